@@ -1,0 +1,401 @@
+"""Pins of the CPU oracle against facts that do not come from the oracle itself.
+
+Each test checks one oracle function against something the format
+definitions or the mathematics fix: library decoders of the same format,
+exhaustive enumeration, brute force on tiny inputs, hand-worked blocks
+(tests/golden/handworked_blocks.json), closed forms of the matmul on
+grid-valued inputs, and invariants of Eq. 2 / Eq. 3 of "Mix-Quant: Quantized
+Prefilling, Precise Decoding for Agentic LLMs", section 3.3.
+"""
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from phase_aware_nvfp4_b200 import workloads as wl
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+E2M1_POS = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]   # OCP FP4 E2M1 magnitudes
+
+
+def bf16(vals):
+    return wl.f32_to_bf16_bits(np.asarray(vals, dtype=np.float32))
+
+
+# ------------------------------------------------------------------ formats
+
+def test_e2m1_decode_table():
+    vals = [oracle.e2m1_value(c) for c in range(16)]
+    assert vals[:8] == E2M1_POS
+    assert vals[8:] == [-v for v in E2M1_POS]
+    assert math.copysign(1.0, vals[8]) == -1.0        # code 0x8 is -0
+
+
+def test_e4m3_decode_matches_torch_for_all_codes():
+    codes = torch.arange(256, dtype=torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    mine = np.array([oracle.e4m3_value(c) for c in range(256)])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(mine), nan)
+    assert set(np.nonzero(nan)[0].tolist()) == {0x7F, 0xFF}
+    assert np.array_equal(mine[~nan], ref[~nan])
+
+
+def test_e4m3_decode_landmarks():
+    assert oracle.e4m3_value(0x7E) == 448.0
+    assert oracle.e4m3_value(0x38) == 1.0
+    assert oracle.e4m3_value(0x08) == 2.0 ** -6      # smallest normal
+    assert oracle.e4m3_value(0x01) == 2.0 ** -9      # smallest subnormal
+    assert oracle.e4m3_value(0x07) == 7 * 2.0 ** -9  # largest subnormal
+
+
+def _finite_e4m3_sorted():
+    return [(oracle.e4m3_value(c), c) for c in range(0x7F)]
+
+
+def test_e4m3_round_matches_torch_rne():
+    """Pi_E4M3 (Eq. 3) = torch's float32 -> float8_e4m3fn cast (RNE) on [0, 448]."""
+    rng = np.random.default_rng(11)
+    s = np.exp2(rng.uniform(-14, 9, 200000)).astype(np.float32)
+    grid = np.array([v for v, _ in _finite_e4m3_sorted()], dtype=np.float64)
+    mids = ((grid[1:] + grid[:-1]) / 2).astype(np.float32)          # every tie, exact in fp32
+    s = np.concatenate([s, mids, grid.astype(np.float32), [0.0, 448.0]]).astype(np.float32)
+    s = s[s <= 448.0]
+    ref = torch.from_numpy(s).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    mine = np.array([oracle.e4m3_round(float(v)) for v in s], dtype=np.uint8)
+    assert np.array_equal(mine, ref)
+
+
+def test_e4m3_round_saturates():
+    for v in (448.0, 449.0, 463.9, 464.0, 1e6, float("inf")):
+        assert oracle.e4m3_round(v) == 0x7E
+
+
+def test_e2m1_round_brute_force():
+    """Pi_FP4 magnitude = brute-force nearest of the 8 magnitudes, ties to even index."""
+    rng = np.random.default_rng(3)
+    m = np.concatenate([rng.uniform(0, 7, 20000), np.linspace(0, 6.5, 2601),
+                        [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0]]).astype(np.float32)
+    for v in m:
+        x = float(v)
+        d = [abs(p - x) for p in E2M1_POS]
+        best = min(d)
+        cands = [i for i, di in enumerate(d) if di == best]
+        want = 7 if x >= 6.0 else ([i for i in cands if i % 2 == 0] or cands)[0]
+        assert oracle.e2m1_round(x) == want, x
+
+
+def test_e2m1_tie_table():
+    ties = {0.25: 0, 0.75: 2, 1.25: 2, 1.75: 4, 2.5: 4, 3.5: 6, 5.0: 6}
+    for m, idx in ties.items():
+        assert oracle.e2m1_round(m) == idx
+
+
+def test_bf16_rounding_known_values():
+    one = 1.0
+    cases = {
+        one: 0x3F80,
+        one + 2.0 ** -8: 0x3F80,            # tie -> even
+        one + 3 * 2.0 ** -8: 0x3F82,        # tie -> even (up)
+        one + 2.0 ** -8 + 2.0 ** -30: 0x3F81,
+        -2.0: 0xC000,
+        2.0 ** -133: 0x0001,                # smallest subnormal
+        2.0 ** -134: 0x0000,                # tie with 0 -> even (0)
+        3 * 2.0 ** -134: 0x0002,            # tie between 1 and 2 quanta -> 2
+        (2 - 2.0 ** -7) * 2.0 ** 127: 0x7F7F,
+        (2 - 2.0 ** -8) * 2.0 ** 127: 0x7F80,  # rounds to +inf
+    }
+    for v, bits in cases.items():
+        assert int(oracle.round_bf16(np.array([v]))[0]) == bits, v
+
+
+def test_bf16_rounding_matches_torch_on_fp32_values():
+    rng = np.random.default_rng(5)
+    v = (rng.standard_normal(100000) * np.exp2(rng.uniform(-20, 20, 100000))).astype(np.float32)
+    ref = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().astype(np.uint16)
+    assert np.array_equal(oracle.round_bf16(v.astype(np.float64)), ref)
+
+
+# ------------------------------------------------------------- Eq. 2 / 3
+
+def _golden_row():
+    g = json.load(open(os.path.join(GOLDEN, "handworked_blocks.json")))
+    x = np.concatenate([bf16(b["x"]) for b in g["blocks"]])[None, :]
+    return g, x
+
+
+def test_handworked_blocks():
+    g, x = _golden_row()
+    amax, alpha, bad = oracle.tensor_alpha(x)
+    assert (amax, alpha, bad) == (2688.0, g["alpha"], False)
+    codes, scales = oracle.quantize(x, alpha)
+    xhat = oracle.dequantize(codes, scales, alpha)[0]
+    for i, b in enumerate(g["blocks"]):
+        assert scales[0, i] == b["sigma_code"], b["name"]
+        assert oracle.e4m3_value(int(scales[0, i])) == b["sigma"]
+        got = []
+        for j in range(16):
+            byte = int(codes[0, i * 8 + j // 2])
+            got.append(byte & 15 if j % 2 == 0 else byte >> 4)
+        assert got == b["codes"], b["name"]
+        assert list(xhat[16 * i:16 * i + 16]) == [float(v) for v in b["xhat"]], b["name"]
+
+
+def test_nibble_order_even_k_low():
+    x = np.zeros((1, 16), dtype=np.uint16)
+    x[0, :2] = bf16([6.0, -3.0])     # amax 6; alpha = 6/2688
+    _, alpha, _ = oracle.tensor_alpha(x)
+    codes, _ = oracle.quantize(x, alpha)
+    assert codes[0, 0] == 0x7 | (0xD << 4)
+
+
+def test_tensor_alpha_special_cases():
+    z = np.zeros((4, 32), dtype=np.uint16)
+    assert oracle.tensor_alpha(z) == (0.0, 1.0, False)
+    x = bf16(np.linspace(-3, 5, 64)).reshape(2, 32)
+    x[1, 3] = 0x7FC0  # NaN
+    amax, _, bad = oracle.tensor_alpha(x)
+    assert bad and amax == 5.0
+    x[1, 3] = 0xFF80  # -inf
+    assert oracle.tensor_alpha(x)[2]
+
+
+def test_alpha_prevents_global_saturation():
+    """With alpha = amax/(6*448) the block holding the tensor amax gets sigma = 448 and no block exceeds it."""
+    for seed in range(5):
+        x = wl.heavy_tailed_bf16(64, 256, seed)
+        amax, alpha, _ = oracle.tensor_alpha(x)
+        _, scales = oracle.quantize(x, alpha)
+        sig = np.array([oracle.e4m3_value(int(c)) for c in np.unique(scales)])
+        assert sig.max() == 448.0
+        flat = np.abs(wl.bf16_bits_to_f32(x)).reshape(64, -1, 16).max(axis=2)
+        r, b = np.unravel_index(np.argmax(flat), flat.shape)
+        assert scales[r, b] == 0x7E
+
+
+def test_block_scale_is_nearest_e4m3_of_exact_quotient():
+    """Eq. 3 in fp32 picks the E4M3 value nearest to the exact quotient amax_b/(6 alpha).
+
+    The only allowed difference is at a near-tie: when the exact quotient lies
+    within a few fp32 ulps of the midpoint of two E4M3 neighbours, the two
+    fp32 roundings (of alpha*6 and of the quotient) may land on the tie and
+    pick the even neighbour.  Both candidates are then the two neighbours.
+    """
+    x = wl.heavy_tailed_bf16(256, 256, 7)
+    amax, alpha, _ = oracle.tensor_alpha(x)
+    _, scales = oracle.quantize(x, alpha)
+    grid = _finite_e4m3_sorted()
+    vals = [Fraction(v) for v, _ in grid]
+    xf = np.abs(wl.bf16_bits_to_f32(x)).reshape(256, 16, 16).max(axis=2)
+    a6 = Fraction(float(np.float32(alpha))) * 6
+    near_ties = 0
+    for r in range(256):
+        for b in range(16):
+            q = Fraction(float(xf[r, b])) / a6
+            best = min(grid, key=lambda vc: (abs(Fraction(vc[0]) - q), vc[1] & 1))
+            want = best[1] if q < 448 else 0x7E
+            if scales[r, b] == want:
+                continue
+            # must be a near-tie between two adjacent E4M3 values
+            i = int(np.searchsorted(np.array([float(v) for v in vals]), float(q)))
+            lo, hi = vals[i - 1], vals[i]
+            mid = (lo + hi) / 2
+            assert abs(q - mid) <= mid * Fraction(1, 2 ** 21), (float(q), float(mid))
+            assert int(scales[r, b]) in (grid[i - 1][1], grid[i][1])
+            near_ties += 1
+    assert near_ties < 0.02 * 256 * 16
+
+
+def test_elements_on_grid_and_error_bound():
+    """Every xhat = +-alpha*sigma*v, and |x - xhat| <= d*(half local step) for normal unsaturated scales."""
+    x = wl.heavy_tailed_bf16(128, 512, 9)
+    _, alpha, _ = oracle.tensor_alpha(x)
+    codes, scales = oracle.quantize(x, alpha)
+    xhat = oracle.dequantize(codes, scales, alpha)
+    xf = wl.bf16_bits_to_f32(x).astype(np.float64)
+    sig = np.vectorize(oracle.e4m3_value)(scales.astype(np.int64)).repeat(16, axis=1)
+    d = (np.float32(alpha) * sig.astype(np.float32)).astype(np.float64)   # fl32(alpha*sigma)
+    d_exact = np.float64(np.float32(alpha)) * sig                         # alpha*sigma, exact in fp64
+    with np.errstate(divide="ignore", invalid="ignore"):
+        v = np.where(d_exact > 0, xhat / np.where(d_exact > 0, d_exact, 1.0), 0.0)
+    assert np.all(np.isin(np.abs(v), E2M1_POS))
+    # half the local grid step at |x|/d
+    m = np.where(d > 0, np.abs(xf) / d, 0.0)
+    half = np.where(m <= 2.0, 0.25, np.where(m <= 4.0, 0.5, 1.0))
+    normal = sig >= 2.0 ** -6
+    err = np.abs(xf - xhat)
+    bound = d * half * (1 + 2.0 ** -20) + np.abs(xf) * 2.0 ** -22
+    clipped = m > 6.0
+    ok = (err <= bound) | ~normal | clipped
+    assert ok.all()
+    # clipped elements: rounding sigma to E4M3 costs at most 2^-4 relative, so |x|/d <= 6.4
+    assert np.all(m[normal] <= 6.0 * (1 + 2.0 ** -4) + 1e-6)
+
+
+def test_frobenius_error_bound():
+    x = wl.heavy_tailed_bf16(64, 1024, 4)
+    _, alpha, _ = oracle.tensor_alpha(x)
+    c, s = oracle.quantize(x, alpha)
+    xhat = oracle.dequantize(c, s, alpha)
+    xf = wl.bf16_bits_to_f32(x).astype(np.float64)
+    amax_b = np.abs(xf).reshape(64, -1, 16).max(axis=2)
+    assert np.sum((xf - xhat) ** 2) <= 16 * np.sum((1.0625 * amax_b / 6) ** 2)
+
+
+def test_requantize_is_idempotent():
+    """Re-quantizing xhat of blocks whose max code is +-6 returns the same codes and scales."""
+    x = wl.heavy_tailed_bf16(32, 256, 12)
+    x[0, 0] = bf16([2688.0])[0]          # amax = 6*448 -> alpha = 1, so xhat = sigma*v is BF16-exact
+    amax, alpha, _ = oracle.tensor_alpha(x)
+    assert amax == 2688.0 and alpha == 1.0
+    c, s = oracle.quantize(x, alpha)
+    xhat = oracle.dequantize(c, s, alpha)
+    xh = oracle.round_bf16(xhat)
+    assert np.array_equal(oracle.bf16_to_f64(xh), xhat)
+    c2, s2 = oracle.quantize(xh, alpha)
+    lo, hi = c & 15, c >> 4
+    mags = np.stack([lo & 7, hi & 7], axis=-1).reshape(32, -1, 16)
+    full = mags.max(axis=2) == 7
+    assert np.array_equal(s2[full], s[full])
+    cm = c.reshape(32, -1, 8)
+    assert np.array_equal(c2.reshape(32, -1, 8)[full], cm[full])
+
+
+def test_rtn_quotient_reading_agrees_with_exact_division():
+    """|x| * fl(1/fl(alpha*sigma)) picks the same code as the exact quotient except at near-ties."""
+    x = wl.heavy_tailed_bf16(256, 512, 21)
+    _, alpha, _ = oracle.tensor_alpha(x)
+    c, s = oracle.quantize(x, alpha)
+    xf = wl.bf16_bits_to_f32(x).astype(np.float64)
+    sig = np.vectorize(oracle.e4m3_value)(s.astype(np.int64)).repeat(16, axis=1)
+    d = np.float64(np.float32(np.float32(alpha) * sig.astype(np.float32)))
+    m = np.where(d > 0, np.abs(xf) / np.where(d > 0, d, 1), 0)
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+    idx = np.searchsorted(mids, m, side="left")
+    tie = np.isin(m, mids)
+    idx = np.where(tie & (idx % 2 == 1), idx + 1, idx)   # exact ties -> even index
+    idx = np.minimum(idx, 7)
+    lo, hi = c & 15, c >> 4
+    got = np.stack([lo & 7, hi & 7], axis=-1).reshape(idx.shape)
+    frac = np.mean(got != idx)
+    assert frac <= 1e-5
+
+
+# ------------------------------------------------------------------ matmuls
+
+def _grid_matrix(rows, K, rng, with_anchor):
+    """Values on the E2M1 grid, each 16-block holding a +-6, so sigma = 1 when alpha = 1."""
+    v = rng.choice(np.array(E2M1_POS + [-p for p in E2M1_POS[1:]]), size=(rows, K))
+    v = v.reshape(rows, K // 16, 16)
+    v[:, :, 0] = rng.choice([6.0, -6.0], size=(rows, K // 16))
+    v = v.reshape(rows, K)
+    if with_anchor:                        # one block [2688, 0...] makes amax = 6*448 -> alpha = 1
+        v[0, :16] = 0.0
+        v[0, 0] = 2688.0
+    return v
+
+
+def test_gemm_closed_form_on_grid_inputs():
+    rng = np.random.default_rng(17)
+    M, N, K = 24, 40, 256
+    xv = _grid_matrix(M, K, rng, True)
+    wv = _grid_matrix(N, K, rng, True)
+    xb, wb = bf16(xv), bf16(wv)
+    ax, aw = oracle.tensor_alpha(xb)[1], oracle.tensor_alpha(wb)[1]
+    assert ax == 1.0 and aw == 1.0
+    xq = (*oracle.quantize(xb, ax), ax)
+    wq = (*oracle.quantize(wb, aw), aw)
+    y, sabs = oracle.nvfp4_linear_rows(xq, wq)
+    # exact: every value is a multiple of 1/2, so 4*x*w sums are integers
+    xi = [[int(Fraction(v) * 2) for v in row] for row in xv]
+    wi = [[int(Fraction(v) * 2) for v in row] for row in wv]
+    for m in range(M):
+        for n in range(N):
+            exact = Fraction(sum(a * b for a, b in zip(xi[m], wi[n])), 4)
+            assert y[m, n] == float(exact)
+            assert sabs[m, n] == float(Fraction(sum(abs(a * b) for a, b in zip(xi[m], wi[n])), 4))
+    assert np.array_equal(oracle.round_bf16(y), oracle.round_bf16(np.array(y)))
+
+
+def test_gemm_tensor_scales_multiply_out():
+    """Scaling X by 2^e scales alpha_x by 2^e and leaves codes/scales unchanged (exact)."""
+    x = wl.heavy_tailed_bf16(16, 128, 30)
+    w = wl.normal_bf16(8, 128, 0.02, 31)
+    xs = wl.f32_to_bf16_bits(wl.bf16_bits_to_f32(x) * np.float32(8.0))
+    a1, a2 = oracle.tensor_alpha(x)[1], oracle.tensor_alpha(xs)[1]
+    assert a2 == 8 * a1
+    c1, s1 = oracle.quantize(x, a1)
+    c2, s2 = oracle.quantize(xs, a2)
+    assert np.array_equal(c1, c2) and np.array_equal(s1, s2)
+    aw = oracle.tensor_alpha(w)[1]
+    wq = (*oracle.quantize(w, aw), aw)
+    y1, _ = oracle.nvfp4_linear_rows((c1, s1, a1), wq)
+    y2, _ = oracle.nvfp4_linear_rows((c2, s2, a2), wq)
+    assert np.array_equal(8 * y1, y2)
+
+
+def test_bf16_linear_exact_on_small_integers():
+    rng = np.random.default_rng(2)
+    xi = rng.integers(-8, 9, size=(5, 64))
+    wi = rng.integers(-8, 9, size=(7, 64))
+    y = oracle.bf16_linear_rows(bf16(xi), bf16(wi))
+    assert np.array_equal(y, (xi @ wi.T).astype(np.float64))
+
+
+def test_nvfp4_vs_bf16_error_is_bounded_by_quantization_error():
+    """|Y_nvfp4 - Y_exact| <= |X - Xhat||W| + |Xhat||W - What| row by row (Cauchy-Schwarz)."""
+    x = wl.heavy_tailed_bf16(32, 512, 40)
+    w = wl.normal_bf16(48, 512, 0.02, 41)
+    ax, aw = oracle.tensor_alpha(x)[1], oracle.tensor_alpha(w)[1]
+    xq = (*oracle.quantize(x, ax), ax)
+    wq = (*oracle.quantize(w, aw), aw)
+    y, _ = oracle.nvfp4_linear_rows(xq, wq)
+    yb = oracle.bf16_linear_rows(x, w)
+    xf, wf = oracle.bf16_to_f64(x), oracle.bf16_to_f64(w)
+    xh, wh = oracle.dequantize(*xq), oracle.dequantize(*wq)
+    ex = np.linalg.norm(xf - xh, axis=1)[:, None] * np.linalg.norm(wf, axis=1)[None, :]
+    ew = np.linalg.norm(xh, axis=1)[:, None] * np.linalg.norm(wf - wh, axis=1)[None, :]
+    assert np.all(np.abs(y - yb) <= (ex + ew) * (1 + 1e-9))
+    assert oracle.rel_frobenius(y, yb) < 0.2
+
+
+def test_silu_mul_against_torch():
+    rng = np.random.default_rng(8)
+    g = rng.standard_normal(50000) * 6
+    u = rng.standard_normal(50000) * 3
+    h = oracle.bf16_to_f64(oracle.silu_mul(g, u))
+    gf = torch.from_numpy(g.astype(np.float32).astype(np.float64))
+    ref = (torch.nn.functional.silu(gf) * torch.from_numpy(u.astype(np.float32).astype(np.float64))).numpy()
+    assert np.all(np.abs(h - ref) <= oracle.bf16_ulp(ref) * 0.5 + np.abs(ref) * 2.0 ** -22)
+    assert oracle.silu_mul(np.array([0.0]), np.array([5.0]))[0] == 0
+
+
+def test_bf16_ulp():
+    assert oracle.bf16_ulp(np.array([1.0]))[0] == 2.0 ** -7
+    assert oracle.bf16_ulp(np.array([3.0]))[0] == 2.0 ** -6
+    assert oracle.bf16_ulp(np.array([0.0]))[0] == 2.0 ** -133
+
+
+@pytest.mark.parametrize("mutation", ["drop_sign", "ties_away"])
+def test_pins_catch_planted_mistakes(mutation):
+    """A plausible slip in the encode step is caught by the hand-worked golden blocks."""
+    g, x = _golden_row()
+    _, alpha, _ = oracle.tensor_alpha(x)
+    codes, _ = oracle.quantize(x, alpha)
+    lo, hi = codes & 15, codes >> 4
+    got = np.stack([lo, hi], axis=-1).reshape(-1)
+    want = np.concatenate([b["codes"] for b in g["blocks"]])
+    assert np.array_equal(got, want)
+    if mutation == "drop_sign":
+        planted = got & 7
+    else:  # round ties away from zero instead of to even
+        xf = np.abs(wl.bf16_bits_to_f32(x[0]).astype(np.float64))
+        planted = got.copy()
+        for i, v in enumerate(xf[16:32]):   # block B has alpha = sigma = 1
+            planted[16 + i] = (got[16 + i] & 8) | int(np.argmin([abs(p - v) - 1e-9 * p for p in E2M1_POS]))
+    assert not np.array_equal(planted, want)
