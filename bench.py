@@ -1,0 +1,452 @@
+#!/usr/bin/env python
+"""Benchmark of the NVFP4 prefill linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {mixquant,reference}]
+
+One step = one prefill pass over the linear projections of a Qwen3-8B-shaped
+transformer layer at M = 8192 tokens (the four projection shapes of the
+workload: q-proj K=4096 N=4096 and k-proj K=4096 N=1024 on the attention
+input, up-proj K=4096 N=12288 on the MLP input, down-proj K=12288 N=4096 on
+the MLP intermediate).  Every activation is quantized on the fly (dynamic
+tensor amax + NVFP4 block quantizer, once per distinct input), then each
+projection runs the tcgen05 block-scaled FP4 GEMM with a BF16 output.  The
+weights are quantized once, before timing (offline, as the method does).
+
+The metric is prefill-linear TFLOP/s counting 2*M*N*K per projection over
+the time of quantization + GEMM.  L2 (126 MB) is flushed by a 512 MiB write
+before every timed step; the flush is outside the per-step CUDA events.
+
+Multi-GPU: one process per GPU (torchrun), each rank runs its own independent
+prefill batch -- the linear layer is token-parallel, so there is no
+data-path collective ("weak" scaling).  A barrier brackets the timed region
+and the per-step time is the max over ranks.
+
+--impl reference times the CPU oracle (oracle/), as it stands, on the host
+cores, on a bounded sample of the same workload, and prints the same line
+with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "NVFP4 prefill linear TFLOP/s (quant+GEMM) and fraction of B200 dense FP4 peak"
+UNIT = "TFLOP/s"
+FP4_PER_BF16 = 4.0          # nominal dense FP4 : dense BF16 tensor throughput on B200
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+GEMM_SOURCES = ("phase_aware_nvfp4_b200/csrc/mq_gemm.cu", "phase_aware_nvfp4_b200/csrc/mq_device.cuh")
+QUANT_SOURCES = ("phase_aware_nvfp4_b200/csrc/mq_quant.cu", "phase_aware_nvfp4_b200/csrc/mq_device.cuh")
+COUNTERS = os.path.join(ROOT, "profiles", "ncu_counters.json")
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="mixquant", choices=["mixquant", "reference"])
+    ap.add_argument("--M", type=int, default=8192, help="prefill tokens per step (per rank)")
+    ap.add_argument("--cpu-baseline-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args(argv)
+
+
+# ---------------------------------------------------------------- helpers
+
+def sources_sha(paths) -> str:
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", 0) or 0), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 0.0, "fallback"
+
+
+def counters_for(kernel: str, sha: str):
+    """DRAM bytes per launch from a committed ncu capture, if the kernel source is unchanged since."""
+    try:
+        with open(COUNTERS) as f:
+            d = json.load(f)
+        k = d.get(kernel, {})
+        if k.get("source_sha") == sha:
+            return k
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while the timed region runs."""
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.period = period_s
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for b, name in self.REASONS.items():
+                    if bits & b:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- workload
+
+def workload(M: int):
+    from phase_aware_nvfp4_b200 import workloads as wl
+    return wl.qwen3_8b_projections(M)
+
+
+def groups_of(w):
+    groups = {}
+    for p in w.projections:
+        groups.setdefault(p.x_group, []).append(p)
+    return groups
+
+
+def host_inputs(w):
+    """Seeded BF16 inputs (numpy uint16): one X per input group, one W per projection."""
+    from phase_aware_nvfp4_b200 import workloads as wl
+    xs = {g: wl.make_x(ps[0]) for g, ps in groups_of(w).items()}
+    ws = {p.name: wl.make_w(p) for p in w.projections}
+    return xs, ws
+
+
+# ---------------------------------------------------------------- oracle timing
+
+def oracle_sample_step(w, xs, wq, rows_per_proj: int, cols_per_proj: int, rng):
+    """One bounded oracle pass: for each projection, the tensor amax of X, the
+    NVFP4 quantization of `rows_per_proj` sampled rows and the FP64 block-scaled
+    matmul against `cols_per_proj` sampled weight rows.  Returns the FLOPs covered."""
+    import oracle
+    flops = 0
+    for g, ps in groups_of(w).items():
+        x = xs[g]
+        _, ax, _ = oracle.tensor_alpha(x)
+        rows = np.sort(rng.choice(x.shape[0], size=min(rows_per_proj, x.shape[0]), replace=False))
+        xc, xsc = oracle.quantize(x[rows], ax)
+        for p in ps:
+            wc, wsc, aw = wq[p.name]
+            cols = np.sort(rng.choice(p.N, size=min(cols_per_proj, p.N), replace=False))
+            oracle.nvfp4_linear_rows((xc, xsc, ax), (wc[cols], wsc[cols], aw))
+            flops += 2 * len(rows) * len(cols) * p.K
+    return flops
+
+
+def oracle_threads():
+    import oracle
+    n = oracle.num_threads()
+    try:
+        from threadpoolctl import threadpool_info
+        n = max([n] + [int(i.get("num_threads", 1)) for i in threadpool_info()])
+    except Exception:
+        pass
+    return n
+
+
+def time_oracle(w, xs, wsh, budget_s: float, steps: int = 1, warmup: int = 0):
+    """Oracle throughput in TFLOP/s on bounded samples sized to `budget_s` seconds per step."""
+    import oracle
+    wq = {}
+    for p in w.projections:
+        _, aw, _ = oracle.tensor_alpha(wsh[p.name])
+        wq[p.name] = (*oracle.quantize(wsh[p.name], aw), aw)
+    rng = np.random.default_rng(0)
+    # calibrate the sample so one step costs about budget_s
+    r, c = 16, 256
+    t0 = time.perf_counter()
+    oracle_sample_step(w, xs, wq, r, c, rng)
+    t1 = time.perf_counter() - t0
+    scale = max(1.0, budget_s / max(t1, 1e-3))
+    r = int(min(w.projections[0].M, r * scale ** 0.5))
+    c = int(min(4096, c * scale ** 0.5))
+    for _ in range(warmup):
+        oracle_sample_step(w, xs, wq, r, c, rng)
+    tot_flops, tot_t = 0, 0.0
+    for _ in range(max(1, steps)):
+        t0 = time.perf_counter()
+        tot_flops += oracle_sample_step(w, xs, wq, r, c, rng)
+        tot_t += time.perf_counter() - t0
+    return {"value": tot_flops / tot_t / 1e12, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+            "sample": f"per step and projection: tensor amax of the full X, NVFP4 quantization of {r} of "
+                      f"{w.projections[0].M} sampled activation rows, FP64 block-scaled matmul against {c} "
+                      f"sampled weight rows (x all K); weights quantized before timing",
+            "seconds": tot_t, "steps": max(1, steps)}
+
+
+# ---------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = workload(args.M)
+    xs, wsh = host_inputs(w)
+    per_step = max(0.05, min(2.0, 120.0 / max(1, args.steps + args.warmup)))
+    res = time_oracle(w, xs, wsh, per_step, steps=args.steps, warmup=args.warmup)
+    line = {"metric": METRIC, "value": res["value"], "unit": UNIT, "impl": "reference", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * res["seconds"] / res["steps"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_of(w),
+            "cpu_baseline": {k: res[k] for k in ("value", "unit", "cores", "kind", "sample")},
+            "e2e": {"value": res["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(w):
+    return {"workload": w.name, "M": w.projections[0].M,
+            "projections": [{"name": p.name, "K": p.K, "N": p.N} for p in w.projections],
+            "activation": "Student-t(3), 1% channels x20, BF16", "weights": "N(0, 0.02^2), BF16",
+            "l2": "flushed with a 512 MiB write before every timed step",
+            "quantization": "dynamic tensor amax per activation, once per distinct input"}
+
+
+# ---------------------------------------------------------------- GPU arm
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    from phase_aware_nvfp4_b200 import mixquant as mq
+
+    w = workload(args.M)
+    groups = groups_of(w)
+    xs_h, ws_h = host_inputs(w)
+    xs_pin = {g: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for g, x in xs_h.items()}
+    X = {g: t.to(dev) for g, t in xs_pin.items()}
+    Wd = {n: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev) for n, a in ws_h.items()}
+    ws = mq.workspace(device=dev)
+    stream = torch.cuda.current_stream()
+
+    # offline weight quantization (timed once, reported separately)
+    Wq = {}
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for p in w.projections:
+        Wq[p.name] = mq.quantize_weight(Wd[p.name], ws=ws)
+    e1.record()
+    torch.cuda.synchronize()
+    weight_quant_ms = e0.elapsed_time(e1)
+
+    Xq = {g: mq.nvfp4_empty(args.M, ps[0].K, dev) for g, ps in groups.items()}
+    Y = {p.name: torch.empty((p.M, p.N), dtype=torch.bfloat16, device=dev) for p in w.projections}
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+
+    ev = {}
+
+    def step(record: bool, i: int = 0):
+        for g, ps in groups.items():
+            if record:
+                ev[("q", g, i)][0].record()
+            mq.quantize_activation(X[g], out=Xq[g], ws=ws)
+            if record:
+                ev[("q", g, i)][1].record()
+            for p in ps:
+                if record:
+                    ev[("g", p.name, i)][0].record()
+                mq.prefill_linear(W=Wq[p.name], Xq=Xq[g], Y=Y[p.name], ws=ws)
+                if record:
+                    ev[("g", p.name, i)][1].record()
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step(False)
+    torch.cuda.synchronize()
+    st = mq.async_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device error during warm-up: {mq.STATUS_NAMES.get(st)}")
+
+    K = args.steps
+    for i in range(K):
+        for g in groups:
+            ev[("q", g, i)] = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+        for p in w.projections:
+            ev[("g", p.name, i)] = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else local) as clk:
+        for i in range(K):
+            flush.zero_()
+            step_ev[i][0].record()
+            step(True, i)
+            step_ev[i][1].record()
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    st = mq.async_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device error in the timed region: {mq.STATUS_NAMES.get(st)}")
+
+    step_ms = [a.elapsed_time(b) for a, b in step_ev]
+    ms = float(np.mean(step_ms))
+    gemm_ms = {p.name: float(np.mean([ev[("g", p.name, i)][0].elapsed_time(ev[("g", p.name, i)][1])
+                                      for i in range(K)])) for p in w.projections}
+    quant_ms = {g: float(np.mean([ev[("q", g, i)][0].elapsed_time(ev[("q", g, i)][1]) for i in range(K)]))
+                for g in groups}
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    flops = w.flops
+    value = flops * world / (ms * 1e-3) / 1e12
+    hbm_gbs, bf16_tf, bf16_tf_sus, peak_src = measured_peaks()
+    fp4_peak = bf16_tf * FP4_PER_BF16
+    gemm_flops = sum(p.flops for p in w.projections)
+    gemm_total_ms = sum(gemm_ms.values())
+    achieved = gemm_flops / (gemm_total_ms * 1e-3) / 1e12
+    gsha = sources_sha(GEMM_SOURCES)
+    cnt = counters_for("gemm_nvfp4", gsha)
+    traffic = None
+    if cnt is not None and "dram_bytes_per_launch" in cnt:
+        traffic = float(np.mean(list(cnt["dram_bytes_per_launch"].values())))
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
+                "frac": achieved / fp4_peak, "traffic": traffic,
+                "kernel": "gemm_nvfp4_kernel<BF16 epilogue>",
+                "peak_source": f"{peak_src} bf16_tflops (burst) x {FP4_PER_BF16:g} nominal FP4:BF16 ratio",
+                "per_projection_tflops": {p.name: p.flops / (gemm_ms[p.name] * 1e-3) / 1e12
+                                          for p in w.projections}}
+    # quantizer: algorithmic bytes = amax read (2 B/elem) + quantize read (2) + codes/scales write (0.5625)
+    q_bytes = {g: ps[0].M * ps[0].K * (2 + 2 + 0.5625) for g, ps in groups.items()}
+    q_gbs = sum(q_bytes.values()) / (sum(quant_ms.values()) * 1e-3) / 1e9
+    roofline_quant = {"bound": "hbm", "achieved": q_gbs, "peak": hbm_gbs, "unit": "GB/s", "frac": q_gbs / hbm_gbs,
+                      "traffic": None, "kernel": "amax_kernel + quantize_kernel",
+                      "bytes_per_elem": 4.5625, "ms": quant_ms}
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "nvfp4", "data": "synthetic", "config": config_of(w),
+            "tokens_per_s": args.M * world / (ms * 1e-3),
+            "fp4_peak_frac": value / world / fp4_peak,
+            "roofline": roofline, "roofline_quant": roofline_quant,
+            "gemm_ms": gemm_ms, "quant_ms": quant_ms, "weight_quant_ms_offline": weight_quant_ms,
+            "gpu_launches": K * (2 * len(groups) + len(w.projections)),
+            "clocks": clk.summary()}
+
+    # end to end through the public API with host buffers: H2D of every
+    # activation from pinned memory, the prefill pass, D2H of every output
+    if not args.no_e2e:
+        y_pin = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for n, t in Y.items()}
+        h2d = sum(t.numel() * 2 for t in xs_pin.values())
+        d2h = sum(t.numel() * 2 for t in Y.values())
+        ke = max(3, min(K, 20))
+
+        def e2e_step():
+            for g in groups:
+                X[g].copy_(xs_pin[g], non_blocking=True)
+            step(False)
+            for n in Y:
+                y_pin[n].copy_(Y[n], non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(ke):
+            e2e_step()
+        b.record()
+        torch.cuda.synchronize()
+        e2e_ms = a.elapsed_time(b) / ke
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        line["e2e"] = {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                       "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": ke}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res = time_oracle(w, xs_h, ws_h, args.cpu_baseline_seconds, steps=1)
+        line["cpu_baseline"] = {k: res[k] for k in ("value", "unit", "cores", "kind", "sample")}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,174 @@
+/*
+ * mixquant.h -- C ABI of libmixquant, the B200 (sm_100a) NVFP4 prefill linear
+ * layer with its BF16 decode counterpart.
+ *
+ * Method: "Mix-Quant: Quantized Prefilling, Precise Decoding for Agentic
+ * LLMs", section 3.3.  The prefill phase runs every linear layer as an NVFP4
+ * W4A4 GEMM: weights are quantized once, activations on the fly, with
+ *   Eq. 2   q_i = Pi_FP4( x_i / (alpha_x sigma_b(i)) ),  xhat_i = alpha_x sigma_b(i) q_i
+ *   Eq. 3   sigma_b = Pi_E4M3( max_{i in b} |x_i| / (alpha_x q_max) ),  q_max = 6
+ * over blocks b of g = 16 consecutive elements along the GEMM K dimension.
+ * The decode phase keeps the BF16 weights ("Prefill-Decode Disaggregation
+ * Deployment", same section).  Readings of the steps the paper leaves open:
+ *   alpha  = amax(|X|) / (6 * 448) in FP32 (1 for an all-zero tensor);
+ *   Pi_E4M3, Pi_FP4: round to nearest, ties to even, saturating (448, 6);
+ *   the quotient of Eq. 2 is |x| * fl(1 / fl(alpha * sigma)); the sign of x
+ *   is kept on a zero code.
+ *
+ * Conventions for every call
+ *   - All pointers are DEVICE pointers owned by the caller, except where a
+ *     parameter says "host".  The library allocates no memory.
+ *   - Calls are asynchronous on `stream`.  Argument errors are returned
+ *     synchronously before anything is launched.  Errors found on the device
+ *     (a NaN/Inf in a tensor being quantized, a pipeline wait that timed out)
+ *     are posted to the control block of the workspace `ws` and returned by
+ *     mq_async_status().
+ *   - BF16 tensors are row-major with a 16-byte aligned base.
+ *   - Shapes: K (the reduction dimension) is a multiple of 64; N is a
+ *     multiple of 16 (128 for the fused MLP epilogue); M >= 1.
+ *
+ * NVFP4 tensor storage (mq_nvfp4), for a logical [rows, cols] matrix:
+ *   codes   rows x cols/2 bytes, row-major; element k of a row is in byte
+ *           k/2, even k in the low nibble; E2M1 code = sign bit 3 + index of
+ *           the magnitude in {0, 0.5, 1, 1.5, 2, 3, 4, 6}.
+ *   scales  E4M3 block scales in the tcgen05 block-scaled MMA layout: for
+ *           each 128-row block and each 64-column chunk, a 512-byte atom in
+ *           which (row r, block kb) sits at (r%32)*16 + ((r%128)/32)*4 + kb%4;
+ *           atoms are ordered K-fastest, ceil(cols/256)*4 atoms per row
+ *           block; padding rows/atoms hold 0.  Size: mq_nvfp4_sizes().
+ *           mq_unswizzle_scales() converts to plain row-major [rows, cols/16].
+ *   alpha   one FP32 tensor scale (device).
+ */
+#ifndef MIXQUANT_H
+#define MIXQUANT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MQ_API __attribute__((visibility("default")))
+#else
+#define MQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* mq_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+typedef enum mq_status {
+    MQ_OK = 0,
+    MQ_ERR_INVALID_ARG = 1, /* null pointer where one is required, bad enum */
+    MQ_ERR_SHAPE = 2,       /* K % 64, N % 16 (128 with the MLP epilogue), M range */
+    MQ_ERR_ALIGNMENT = 3,   /* a pointer is not 16-byte aligned */
+    MQ_ERR_WORKSPACE = 4,   /* workspace missing or smaller than mq_workspace_bytes() */
+    MQ_ERR_NONFINITE = 5,   /* (async) NaN or Inf in a tensor that was quantized */
+    MQ_ERR_TIMEOUT = 6,     /* (async) a device-side pipeline wait gave up */
+    MQ_ERR_CUDA = 7,        /* a CUDA runtime/driver call failed */
+    MQ_ERR_DEVICE = 8       /* current device is not compute capability 10.0 (B200) */
+} mq_status;
+
+typedef enum mq_epilogue {
+    MQ_EPI_BF16 = 0,         /* Y = bf16(alpha_x alpha_w X W^T) */
+    MQ_EPI_SILU_MUL_NVFP4 = 1 /* h = bf16(silu(gate) * up), stored as NVFP4 with a static alpha_h */
+} mq_epilogue;
+
+/* An NVFP4 tensor: views of caller-owned device buffers (layout above). */
+typedef struct mq_nvfp4 {
+    uint8_t* codes;
+    uint8_t* scales;
+    float* alpha;
+    int64_t rows;
+    int64_t cols;
+} mq_nvfp4;
+
+/* Fixed part of every workspace: control block (error bits, counters) and
+ * the amax partial maxima.  A workspace must be zero-filled once before its
+ * first use; afterwards the library keeps it consistent.  Use one workspace
+ * per stream (concurrent calls must not share one). */
+#define MQ_WS_CONTROL_BYTES 16384
+
+/* Human-readable name of a status code (static string). */
+MQ_API const char* mq_status_string(mq_status s);
+
+/* Library version as "major.minor.patch" (static string). */
+MQ_API const char* mq_version(void);
+
+/* Byte sizes of the codes and scales buffers of an NVFP4 [rows, cols] tensor
+ * (cols a multiple of 64).  Host-only; writes through the two host pointers. */
+MQ_API mq_status mq_nvfp4_sizes(int64_t rows, int64_t cols, size_t* codes_bytes, size_t* scales_bytes);
+
+/* Workspace bytes for mq_prefill_linear / mq_quantize_activation on an
+ * activation of M x K: the control block plus room for the NVFP4 copy of
+ * the activation.  mq_workspace_bytes(0, 0) == MQ_WS_CONTROL_BYTES is enough
+ * for calls that quantize nothing in the workspace. */
+MQ_API size_t mq_workspace_bytes(int64_t M, int64_t K);
+
+/*
+ * Offline weight quantization (section 3.3: the same NVFP4 format is applied
+ * to the weights, so the prefill GEMM is W4A4).  W: BF16 [N, K].  Computes
+ * the tensor scale alpha_w = amax/(6*448), then Eq. 3 block scales and
+ * Eq. 2 codes into `out` (out->rows == N, out->cols == K).
+ * gate_up_interleave != 0 declares W as [2I, K] = [W_gate; W_up] (I = N/2,
+ * I % 64 == 0) and stores the rows interleaved in groups of 16
+ * (out row 32c+t = gate row 16c+t for t < 16, up row 16c+t-16 otherwise), the
+ * B-operand order the MQ_EPI_SILU_MUL_NVFP4 epilogue expects.
+ * ws: >= MQ_WS_CONTROL_BYTES.
+ */
+MQ_API mq_status mq_quantize_weight(const void* W_bf16, int64_t N, int64_t K, int gate_up_interleave,
+                             const mq_nvfp4* out, void* ws, size_t ws_bytes, mq_stream_t stream);
+
+/*
+ * On-the-fly activation quantization (Eq. 2, Eq. 3).  X: BF16 [M, K].
+ * alpha_static: device FP32 tensor scale to use, or NULL to compute the
+ * dynamic alpha = amax(|X|)/(6*448) into out->alpha (one extra read of X).
+ * ws: >= MQ_WS_CONTROL_BYTES.
+ */
+MQ_API mq_status mq_quantize_activation(const void* X_bf16, int64_t M, int64_t K, const float* alpha_static,
+                                 const mq_nvfp4* out, void* ws, size_t ws_bytes, mq_stream_t stream);
+
+/*
+ * The NVFP4 prefill linear layer: quantize X (unless X_q is given), then the
+ * block-scaled FP4 x FP4 GEMM with FP32 accumulation,
+ *   acc[m, n] = sum_k (sigma q)_X[m, k] (sigma q)_W[n, k],
+ * and the epilogue:
+ *   MQ_EPI_BF16            Y[m, n] = bf16(acc * alpha_x * alpha_w), Y BF16 [M, N];
+ *   MQ_EPI_SILU_MUL_NVFP4  W is an interleaved gate/up weight (N = 2I); with
+ *                          g, u = acc * alpha_x * alpha_w of the paired gate/up
+ *                          columns, h = bf16(silu(g) * u) is quantized (Eq. 2,
+ *                          Eq. 3) with the static device scale *alpha_h into
+ *                          H_out ([M, I]; H_out->alpha is not written).
+ *                          h_debug (optional, BF16 [M, I]) also receives h.
+ * Exactly one of X_bf16 / X_q is non-NULL.  With X_bf16, the activation is
+ * quantized into the workspace (ws_bytes >= mq_workspace_bytes(M, K)) with
+ * alpha_x = *alpha_static, or the dynamic amax scale when alpha_static is NULL.
+ * With X_q (already NVFP4, e.g. the H_out of a previous call), ws_bytes >=
+ * MQ_WS_CONTROL_BYTES.
+ */
+MQ_API mq_status mq_prefill_linear(const void* X_bf16, const mq_nvfp4* X_q, int64_t M, const mq_nvfp4* W,
+                            mq_epilogue epi, const float* alpha_static, const float* alpha_h, void* Y,
+                            const mq_nvfp4* H_out, void* h_debug, void* ws, size_t ws_bytes, mq_stream_t stream);
+
+/*
+ * The precise decode path (section 3.3: decoding stays on the original BF16
+ * weights): Y[M, N] = bf16(sum_k X[m, k] W[n, k]) with FP32 accumulation on
+ * the tensor cores.  X BF16 [M, K] with 1 <= M <= 256, W BF16 [N, K], Y BF16
+ * [M, N].  ws: >= MQ_WS_CONTROL_BYTES (error reporting only).
+ */
+MQ_API mq_status mq_decode_linear(const void* X_bf16, int64_t M, const void* W_bf16, int64_t N, int64_t K, void* Y_bf16,
+                           void* ws, size_t ws_bytes, mq_stream_t stream);
+
+/* Copy the block scales of `t` to plain row-major [rows, cols/16] bytes. */
+MQ_API mq_status mq_unswizzle_scales(const mq_nvfp4* t, uint8_t* rowmajor_out, mq_stream_t stream);
+
+/* Synchronize `stream`, then read and clear the asynchronous error bits of
+ * workspace `ws`: MQ_OK, MQ_ERR_NONFINITE, MQ_ERR_TIMEOUT (or MQ_ERR_CUDA if
+ * the synchronization itself failed). */
+MQ_API mq_status mq_async_status(void* ws, mq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MIXQUANT_H */

@@ -1,0 +1,254 @@
+// mq_decode.cu -- the precise decode path: BF16 GEMV / skinny GEMM on the
+// BF16 master weights, FP32 accumulation ("Mix-Quant: Quantized Prefilling,
+// Precise Decoding for Agentic LLMs", section 3.3, "Prefill-Decode
+// Disaggregation Deployment": the decode path keeps the original
+// high-precision weights; section 3.1: decoding is bound by memory access).
+//
+// Y[M, N] = X[M, K] W[N, K]^T with M <= 256 tokens.  The kernel computes the
+// transposed product on the tensor cores, D[n, m] = sum_k W[n, k] X[m, k]:
+// A = a 128-row W tile streamed by TMA, B = the (zero-padded) token tile,
+// D = 128 lanes x MT columns of FP32 in TMEM.  The W stream is the whole
+// cost, so the grid must cover every SM: the K dimension is split across the
+// CTAs of a thread-block cluster and the partial sums are reduced through
+// distributed shared memory (no global scratch, deterministic order).
+#include "mq_device.cuh"
+
+namespace mq {
+namespace {
+
+constexpr int DBM = 128;                 // W rows per tile (UMMA M)
+constexpr int DBK = 64;                  // K elements per stage (128 bytes of BF16)
+constexpr int D_THREADS = 192;
+constexpr int W_STAGE = DBM * DBK * 2;   // 16 KiB
+
+struct DParams {
+    int M, N, K, MT;
+    int k_stages;       // total K stages
+    int split;          // cluster size along K
+    int stages;         // pipeline depth
+    int bar_offset;     // barriers sit after both the pipeline and the partial-sum buffer
+    uint32_t tmem_cols;
+    uint16_t* y;
+    WsControl* ctrl;
+};
+
+__device__ __forceinline__ uint32_t cluster_rank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all()
+{
+    asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t local_addr, uint32_t rank)
+{
+    uint32_t raddr;
+    float v;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(raddr) : "r"(local_addr), "r"(rank));
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(raddr) : "memory");
+    return v;
+}
+
+__global__ void __launch_bounds__(D_THREADS, 1)
+    decode_bf16_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
+                       const DParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int x_stage = p.MT * DBK * 2;
+    const int stage_bytes = W_STAGE + x_stage;
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + p.bar_offset);
+    uint64_t* empty_bar = full_bar + p.stages;
+    uint64_t* acc_full = empty_bar + p.stages;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+    volatile uint32_t* abort_flag = tmem_slot + 1;
+    float* red = reinterpret_cast<float*>(smem);  // [MT][128] partials, reuses the pipeline buffers
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = (p.split > 1) ? cluster_rank() : 0u;
+    const int n_tile = blockIdx.x / p.split;
+    const int ks_begin = (int)(((int64_t)p.k_stages * rank) / p.split);
+    const int ks_end = (int)(((int64_t)p.k_stages * (rank + 1)) / p.split);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < p.stages; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], 1);
+        }
+        mbar_init(acc_full, 1);
+        *abort_flag = 0;
+        fence_mbarrier_init();
+        prefetch_tensormap(&tmap_w);
+        prefetch_tensormap(&tmap_x);
+    }
+    if (warp == 1) tmem_alloc(tmem_slot, p.tmem_cols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            int last_stage = -1;
+            uint32_t last_parity = 0;
+            for (int ks = ks_begin; ks < ks_end; ++ks) {
+                if (*abort_flag || !mbar_wait(&empty_bar[stage], phase ^ 1u)) {
+                    ok = false;
+                    break;
+                }
+                mbar_arrive_expect_tx(&full_bar[stage], (uint32_t)stage_bytes);
+                uint8_t* sw = smem + stage * stage_bytes;
+                tma_load_2d(sw, &tmap_w, &full_bar[stage], ks * DBK, n_tile * DBM);
+                tma_load_2d(sw + W_STAGE, &tmap_x, &full_bar[stage], ks * DBK, 0);
+                last_stage = stage;
+                last_parity = phase;
+                if (++stage == p.stages) stage = 0, phase ^= 1u;
+            }
+            if (!ok) {
+                post_error(p.ctrl, kErrTimeout);
+                *abort_flag = 1;
+                // stages are consumed in order, so the newest issue lands last
+                if (last_stage >= 0) (void)mbar_wait(&full_bar[last_stage], last_parity);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16(DBM, p.MT);
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int ks = ks_begin; ks < ks_end; ++ks) {
+                if (*abort_flag || !mbar_wait(&full_bar[stage], phase)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t w_addr = smem_u32(smem + stage * stage_bytes);
+                const uint32_t x_addr = w_addr + W_STAGE;
+#pragma unroll
+                for (int kb = 0; kb < 4; ++kb)
+                    umma_bf16(tmem_base, sdesc_kmajor_sw128(w_addr + 32 * kb), sdesc_kmajor_sw128(x_addr + 32 * kb),
+                              idesc, (ks > ks_begin || kb > 0) ? 1u : 0u);
+                tc_commit(&empty_bar[stage]);
+                if (++stage == p.stages) stage = 0, phase ^= 1u;
+            }
+            if (!ok) {
+                post_error(p.ctrl, kErrTimeout);
+                *abort_flag = 1;
+            }
+            tc_commit(acc_full);  // also the "all MMAs done" signal before TMEM is freed
+        }
+    } else {
+        const int lg = warp & 3;
+        const int row = 32 * lg + lane;  // W row within the tile = TMEM lane
+        const int64_t n = (int64_t)n_tile * DBM + row;
+        const bool have_acc = ks_end > ks_begin;
+        bool ok = mbar_wait(acc_full, 0);
+        if (!ok) post_error(p.ctrl, kErrTimeout);
+        tc_fence_after();
+        const uint32_t t_row = tmem_base + ((uint32_t)(32 * lg) << 16);
+        for (int c = 0; c < p.MT / 16; ++c) {
+            uint32_t r[16];
+            tmem_ld_32x32b_x16(t_row + 16 * c, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int m = 16 * c + j;
+                const float v = (have_acc && ok) ? __uint_as_float(r[j]) : 0.0f;
+                if (p.split > 1) {
+                    red[m * DBM + row] = v;
+                } else if (m < p.M && n < p.N) {
+                    p.y[(int64_t)m * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+                }
+            }
+        }
+    }
+
+    if (p.split > 1) {
+        // Every CTA of the cluster has its partial tile in shared memory; CTA
+        // `rank` reduces tokens m = rank, rank + split, ... in rank order.
+        cluster_sync_all();
+        if (warp >= 2) {
+            const int row = 32 * (warp & 3) + lane;
+            const int64_t n = (int64_t)n_tile * DBM + row;
+            for (int m = (int)rank; m < p.M; m += p.split) {
+                float acc = 0.0f;
+                const uint32_t laddr = smem_u32(&red[m * DBM + row]);
+                for (int q = 0; q < p.split; ++q) acc += ld_dsmem_f32(laddr, (uint32_t)q);
+                if (n < p.N) p.y[(int64_t)m * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(acc));
+            }
+        }
+        cluster_sync_all();  // keep every partial alive until all readers are done
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, p.tmem_cols);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_decode_bf16(const void* x, int64_t M, const void* w, int64_t N, int64_t K, void* y,
+                               WsControl* ctrl, const DeviceInfo& di, cudaStream_t s)
+{
+    DParams p{};
+    p.M = (int)M;
+    p.N = (int)N;
+    p.K = (int)K;
+    p.MT = (int)((M + 15) / 16 * 16);
+    p.k_stages = (int)((K + DBK - 1) / DBK);
+    p.tmem_cols = 32;
+    while ((int)p.tmem_cols < p.MT) p.tmem_cols <<= 1;
+    p.y = static_cast<uint16_t*>(y);
+    p.ctrl = ctrl;
+    const int n_tiles = (int)((N + DBM - 1) / DBM);
+    const int x_stage = p.MT * DBK * 2;
+    const int stage_bytes = W_STAGE + x_stage;
+    // ~100 KB of pipeline per CTA: two CTAs share an SM and keep ~190 KB of W in flight
+    p.stages = std::max(2, std::min(8, 100 * 1024 / stage_bytes));
+    const int red_bytes = p.MT * DBM * 4;
+    p.bar_offset = std::max(p.stages * stage_bytes, red_bytes);
+    const int smem = p.bar_offset + 256 + 1024;
+    // split K so the grid covers the SMs about twice (cluster size <= 8)
+    int split = (2 * di.num_sms + n_tiles - 1) / n_tiles;
+    split = std::max(1, std::min(8, std::min(split, p.k_stages)));
+    p.split = split;
+
+    CUtensorMap tw, tx;
+    if (!make_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w, (uint64_t)K, (uint64_t)N, (uint64_t)K * 2, DBK, DBM,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    if (!make_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, DBK,
+                      (uint32_t)p.MT, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+
+    cudaError_t e = cudaFuncSetAttribute(decode_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)(n_tiles * split), 1, 1);
+    cfg.blockDim = dim3(D_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)split;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, decode_bf16_kernel, tw, tx, p);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+}  // namespace mq

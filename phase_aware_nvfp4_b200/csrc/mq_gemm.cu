@@ -1,0 +1,397 @@
+// mq_gemm.cu -- block-scaled NVFP4 x NVFP4 GEMM on sm_100a tensor cores.
+//
+// Y[M, N] = alpha_a * alpha_b * sum_k (sigma_a q_a)[m, k] (sigma_b q_b)[n, k]
+// with FP32 accumulation in TMEM and a BF16 (or fused SiLU-mul + NVFP4
+// requantize) epilogue: the prefill linear layer of "Mix-Quant: Quantized
+// Prefilling, Precise Decoding for Agentic LLMs", section 3.3 (NVFP4 W4A4
+// prefill; Eq. 2 gives xhat = alpha * sigma * q, so the matmul of the
+// dequantized operands factors into the block-scaled MMA times the two
+// tensor scales).
+//
+// Design (one persistent CTA per SM, 192 threads):
+//   warp 0      TMA producer: per K stage, A and B code tiles by tensor-map
+//               TMA (128-byte swizzle), and the A/B scale atoms by bulk copy,
+//               all completing on one mbarrier.
+//   warp 1      TMEM owner and MMA issuer: copies the stage's scale atoms to
+//               TMEM (tcgen05.cp) and issues 4 x tcgen05.mma kind::mxf4nvf4
+//               (128 x 256 x 64 each) per stage; commits free the stage and,
+//               at the end of a tile, signal the epilogue.
+//   warps 2-5   epilogue: drain the 128 x 256 FP32 accumulator from TMEM
+//               (one row per thread), release it to the MMA warp, then apply
+//               the tensor scales and store BF16 (or SiLU-mul -> NVFP4).
+// Stage = 256 K-elements (128 bytes per row, one swizzle row); 4 stages in
+// flight.  TMEM: accumulator in columns [0, 256), scale factors in two
+// alternating 48-column buffers from column 256 (per stage: 4 x 4 columns
+// for A, 4 x 8 columns for B, one 32-bit column per 32 rows per MMA).
+#include "mq_device.cuh"
+
+namespace mq {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 256;                  // K elements per stage
+constexpr int BK_BYTES = BK / 2;         // packed FP4 bytes per row per stage
+constexpr int STAGES = 4;
+constexpr int A_STAGE = BM * BK_BYTES;   // 16 KiB
+constexpr int B_STAGE = BN * BK_BYTES;   // 32 KiB
+constexpr int SFA_STAGE = 2048;          // 1 row block x 4 atoms
+constexpr int SFB_STAGE = 4096;          // 2 row blocks x 4 atoms
+constexpr int OFF_A = 0;
+constexpr int OFF_B = OFF_A + STAGES * A_STAGE;
+constexpr int OFF_SFA = OFF_B + STAGES * B_STAGE;
+constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_STAGE;
+constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_STAGE;
+constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;  // + barriers + alignment slack
+constexpr int NUM_THREADS = 192;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t TMEM_SF = 256;        // two scale-factor buffers of 48 columns
+constexpr uint32_t TMEM_SF_BUF = 48;     // SFA 16 columns + SFB 32 columns per stage
+constexpr uint32_t IDESC = idesc_nvfp4(BM, BN);
+
+struct Params {
+    const uint8_t* sfa;
+    const uint8_t* sfb;
+    const float* alpha_a;
+    const float* alpha_b;
+    int M, N, K;
+    int num_m_blk, num_tiles, k_stages;
+    int sfa_atoms, sfb_atoms, sfb_rowblks;
+    void* y;
+    uint8_t* h_codes;
+    uint8_t* h_scales;
+    const float* h_alpha;
+    uint16_t* h_debug;
+    int h_atoms;
+    WsControl* ctrl;
+};
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&p);
+}
+
+// Fused MLP epilogue for one 32-column chunk of a row: columns 0..15 are
+// gate values and 16..31 the matching up values (the weight rows were
+// interleaved in 16-row groups when quantized).  Produces 16 values of
+// h = bf16(silu(g) * u) and quantizes them as one NVFP4 block with the
+// static tensor scale alpha_h (Eq. 2 / Eq. 3 with alpha = alpha_h).
+__device__ __forceinline__ void silu_mul_quant_chunk(const uint32_t (&acc)[32], float alpha_ab, float alpha_h,
+                                                     float alpha_h_qmax, uint32_t (&codes)[2], uint32_t& scale,
+                                                     uint32_t (&hbits)[8])
+{
+    float h[16];
+    float amax = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        const float g = __fmul_rn(__uint_as_float(acc[j]), alpha_ab);
+        const float u = __fmul_rn(__uint_as_float(acc[16 + j]), alpha_ab);
+        const float sg = __fdiv_rn(g, 1.0f + expf(-g));
+        const float hv = __bfloat162float(__float2bfloat16_rn(__fmul_rn(sg, u)));
+        h[j] = hv;
+        amax = fmaxf(amax, fabsf(hv));
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) hbits[j] = pack_bf16x2(h[2 * j], h[2 * j + 1]);
+    const uint32_t sc = e4m3_round_sat(__fdiv_rn(amax, alpha_h_qmax));
+    const float d = __fmul_rn(alpha_h, e4m3_to_float(sc));
+    const float enc = (d == 0.0f) ? 0.0f : __fdiv_rn(1.0f, d);
+    codes[0] = codes[1] = 0;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) codes[j >> 3] |= e2m1_code(h[j], enc) << (4 * (j & 7));
+    scale = sc;
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                      const Params p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+    uint64_t* empty_bar = full_bar + STAGES;
+    uint64_t* acc_full = empty_bar + STAGES;
+    uint64_t* acc_empty = acc_full + 1;
+    uint64_t* mma_done = acc_empty + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+    volatile uint32_t* abort_flag = tmem_slot + 1;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], 1);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, 128);
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        fence_mbarrier_init();
+        prefetch_tensormap(&tmap_a);
+        prefetch_tensormap(&tmap_b);
+    }
+    if (warp == 1) tmem_alloc(tmem_slot, TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t issued_parity[STAGES];
+            bool issued[STAGES];
+            for (int s = 0; s < STAGES; ++s) issued[s] = false, issued_parity[s] = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
+                const int m_blk = tile % p.num_m_blk;
+                const int n_blk = tile / p.num_m_blk;
+                const bool two_sfb = (2 * n_blk + 1) < p.sfb_rowblks;
+                const uint32_t tx = A_STAGE + B_STAGE + SFA_STAGE + (two_sfb ? SFB_STAGE : SFB_STAGE / 2);
+                for (int ks = 0; ks < p.k_stages; ++ks) {
+                    if (*abort_flag || !mbar_wait(&empty_bar[stage], phase ^ 1u)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&full_bar[stage], tx);
+                    tma_load_2d(smem + OFF_A + stage * A_STAGE, &tmap_a, &full_bar[stage], ks * BK_BYTES,
+                                m_blk * BM);
+                    tma_load_2d(smem + OFF_B + stage * B_STAGE, &tmap_b, &full_bar[stage], ks * BK_BYTES,
+                                n_blk * BN);
+                    bulk_load(smem + OFF_SFA + stage * SFA_STAGE,
+                              p.sfa + ((int64_t)m_blk * p.sfa_atoms + ks * 4) * 512, SFA_STAGE, &full_bar[stage]);
+                    bulk_load(smem + OFF_SFB + stage * SFB_STAGE,
+                              p.sfb + ((int64_t)(2 * n_blk) * p.sfb_atoms + ks * 4) * 512, 2048, &full_bar[stage]);
+                    if (two_sfb)
+                        bulk_load(smem + OFF_SFB + stage * SFB_STAGE + 2048,
+                                  p.sfb + ((int64_t)(2 * n_blk + 1) * p.sfb_atoms + ks * 4) * 512, 2048,
+                                  &full_bar[stage]);
+                    issued[stage] = true;
+                    issued_parity[stage] = phase;
+                    if (++stage == STAGES) stage = 0, phase ^= 1u;
+                }
+            }
+            if (!ok) {
+                post_error(p.ctrl, kErrTimeout);
+                *abort_flag = 1;
+                // let every copy already in flight land before the CTA exits
+                for (int s = 0; s < STAGES; ++s)
+                    if (issued[s]) (void)mbar_wait(&full_bar[s], issued_parity[s]);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            bool ok = true;
+            const uint32_t d_tmem = tmem_base;
+            uint32_t sf_buf = 0;
+            for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
+                if (*abort_flag || !mbar_wait(acc_empty, acc_phase ^ 1u)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                for (int ks = 0; ks < p.k_stages; ++ks) {
+                    if (*abort_flag || !mbar_wait(&full_bar[stage], phase)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_base = smem_u32(smem + OFF_A + stage * A_STAGE);
+                    const uint32_t b_base = smem_u32(smem + OFF_B + stage * B_STAGE);
+                    const uint32_t sfa_base = smem_u32(smem + OFF_SFA + stage * SFA_STAGE);
+                    const uint32_t sfb_base = smem_u32(smem + OFF_SFB + stage * SFB_STAGE);
+                    // scale factors alternate between two TMEM buffers from stage to stage
+                    const uint32_t sfa_tmem = tmem_base + TMEM_SF + sf_buf * TMEM_SF_BUF;
+                    const uint32_t sfb_tmem = sfa_tmem + 16;
+                    sf_buf ^= 1u;
+#pragma unroll
+                    for (int kb = 0; kb < 4; ++kb) {
+                        tmem_cp_32x128b_x4(sfa_tmem + 4 * kb, sdesc_sf_block(sfa_base + kb * 512));
+                        tmem_cp_32x128b_x4(sfb_tmem + 8 * kb, sdesc_sf_block(sfb_base + kb * 512));
+                        tmem_cp_32x128b_x4(sfb_tmem + 8 * kb + 4, sdesc_sf_block(sfb_base + 2048 + kb * 512));
+                    }
+#pragma unroll
+                    for (int kb = 0; kb < 4; ++kb) {
+                        umma_nvfp4(d_tmem, sdesc_kmajor_sw128(a_base + kb * 32), sdesc_kmajor_sw128(b_base + kb * 32),
+                                   IDESC, sfa_tmem + 4 * kb, sfb_tmem + 8 * kb, (ks | kb) != 0 ? 1u : 0u);
+                    }
+                    tc_commit(&empty_bar[stage]);
+                    if (++stage == STAGES) stage = 0, phase ^= 1u;
+                }
+                if (!ok) break;
+                tc_commit(acc_full);
+                acc_phase ^= 1u;
+            }
+            if (!ok) {
+                post_error(p.ctrl, kErrTimeout);
+                *abort_flag = 1;
+            }
+            // every MMA / copy issued above has finished before TMEM is freed
+            tc_commit(mma_done);
+            (void)mbar_wait(mma_done, 0);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int lg = warp & 3;  // TMEM lane group this warp may access
+        const float alpha_ab = __fmul_rn(*p.alpha_a, *p.alpha_b);
+        float alpha_h = 1.0f, alpha_h_qmax = 6.0f;
+        if (EPI == 1) {
+            alpha_h = *p.h_alpha;
+            alpha_h_qmax = __fmul_rn(alpha_h, 6.0f);
+        }
+        uint32_t acc_phase = 0;
+        for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+            const int m_blk = tile % p.num_m_blk;
+            const int n_blk = tile / p.num_m_blk;
+            if (*abort_flag || !mbar_wait(acc_full, acc_phase)) {
+                post_error(p.ctrl, kErrTimeout);
+                *abort_flag = 1;
+                break;
+            }
+            acc_phase ^= 1u;
+            tc_fence_after();
+            const uint32_t t_row = tmem_base + ((uint32_t)(32 * lg) << 16);
+            const int64_t row = (int64_t)m_blk * BM + 32 * lg + lane;
+            if (EPI == 0) {
+                uint32_t out[128];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(t_row + 32 * c, r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        out[16 * c + j] = pack_bf16x2(__fmul_rn(__uint_as_float(r[2 * j]), alpha_ab),
+                                                      __fmul_rn(__uint_as_float(r[2 * j + 1]), alpha_ab));
+                }
+                tc_fence_before();
+                mbar_arrive(acc_empty);
+                if (row < p.M) {
+                    uint16_t* yrow = static_cast<uint16_t*>(p.y) + row * (int64_t)p.N + (int64_t)n_blk * BN;
+                    const int ncols = min(BN, p.N - n_blk * BN);
+#pragma unroll
+                    for (int q = 0; q < 32; ++q)
+                        if (8 * q < ncols)
+                            reinterpret_cast<uint4*>(yrow)[q] =
+                                make_uint4(out[4 * q], out[4 * q + 1], out[4 * q + 2], out[4 * q + 3]);
+                }
+            } else {
+                uint32_t codes[16];
+                uint32_t scl[8];
+                uint32_t hb[64];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(t_row + 32 * c, r);
+                    tmem_wait_ld();
+                    uint32_t cc[2], hbits[8];
+                    silu_mul_quant_chunk(r, alpha_ab, alpha_h, alpha_h_qmax, cc, scl[c], hbits);
+                    codes[2 * c] = cc[0];
+                    codes[2 * c + 1] = cc[1];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) hb[8 * c + j] = hbits[j];
+                }
+                tc_fence_before();
+                mbar_arrive(acc_empty);
+                const int hN = p.N / 2;
+                const int hcol0 = n_blk * (BN / 2);  // first h column of this tile
+                if (row < p.M && hcol0 < hN) {
+                    const int nch = min(8, (hN - hcol0) / 16);
+                    uint8_t* crow = p.h_codes + row * (int64_t)(hN / 2) + hcol0 / 2;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        if (c < nch)
+                            *reinterpret_cast<uint2*>(crow + 8 * c) = make_uint2(codes[2 * c], codes[2 * c + 1]);
+#pragma unroll
+                    for (int g = 0; g < 2; ++g)
+                        if (4 * g < nch) {
+                            const int kb = hcol0 / 16 + 4 * g;
+                            const uint32_t v =
+                                scl[4 * g] | (scl[4 * g + 1] << 8) | (scl[4 * g + 2] << 16) | (scl[4 * g + 3] << 24);
+                            *reinterpret_cast<uint32_t*>(p.h_scales + sf_offset(row, kb, p.h_atoms)) = v;
+                        }
+                    if (p.h_debug != nullptr) {
+                        uint16_t* hrow = p.h_debug + row * (int64_t)hN + hcol0;
+#pragma unroll
+                        for (int c = 0; c < 8; ++c)
+                            if (c < nch) {
+                                reinterpret_cast<uint4*>(hrow)[2 * c] =
+                                    make_uint4(hb[8 * c], hb[8 * c + 1], hb[8 * c + 2], hb[8 * c + 3]);
+                                reinterpret_cast<uint4*>(hrow)[2 * c + 1] =
+                                    make_uint4(hb[8 * c + 4], hb[8 * c + 5], hb[8 * c + 6], hb[8 * c + 7]);
+                            }
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_nvfp4(const GemmArgs& a, const DeviceInfo& di, cudaStream_t s)
+{
+    CUtensorMap ta, tb;
+    // A codes: [M rows, K/2 bytes], B codes: [N rows, K/2 bytes]; 128 x 128-byte
+    // and 256 x 128-byte boxes with the 128-byte swizzle the UMMA descriptors use.
+    if (!make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.a_codes, (uint64_t)(a.K / 2), (uint64_t)a.M,
+                      (uint64_t)(a.K / 2), BK_BYTES, BM, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    if (!make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.b_codes, (uint64_t)(a.K / 2), (uint64_t)a.N,
+                      (uint64_t)(a.K / 2), BK_BYTES, BN, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    Params p{};
+    p.sfa = a.a_scales;
+    p.sfb = a.b_scales;
+    p.alpha_a = a.a_alpha;
+    p.alpha_b = a.b_alpha;
+    p.M = (int)a.M;
+    p.N = (int)a.N;
+    p.K = (int)a.K;
+    p.num_m_blk = (int)((a.M + BM - 1) / BM);
+    const int num_n_blk = (int)((a.N + BN - 1) / BN);
+    p.num_tiles = p.num_m_blk * num_n_blk;
+    p.k_stages = (int)((a.K + BK - 1) / BK);
+    p.sfa_atoms = (int)sf_atoms_per_rowblk(a.K);
+    p.sfb_atoms = (int)sf_atoms_per_rowblk(a.K);
+    p.sfb_rowblks = (int)sf_rowblks(a.N);
+    p.y = a.y;
+    p.h_codes = a.h_codes;
+    p.h_scales = a.h_scales;
+    p.h_alpha = a.h_alpha;
+    p.h_debug = a.h_debug;
+    p.h_atoms = (int)sf_atoms_per_rowblk(a.N / 2);
+    p.ctrl = a.ctrl;
+
+    const int grid = std::min(p.num_tiles, di.num_sms);
+    if (a.epilogue == 0) {
+        auto k = gemm_nvfp4_kernel<0>;
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        k<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, tb, p);
+    } else {
+        auto k = gemm_nvfp4_kernel<1>;
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        k<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, tb, p);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace mq

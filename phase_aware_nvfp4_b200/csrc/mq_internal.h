@@ -1,0 +1,98 @@
+// mq_internal.h -- declarations shared by the CUDA sources of libmixquant
+// (not part of the public ABI; the public header is include/mixquant.h).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace mq {
+
+// Bounded waits: a device-side wait on an mbarrier gives up after this much
+// wall time, posts kErrTimeout and unwinds.
+constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s
+
+// Asynchronous error bits posted by kernels into the workspace control block.
+constexpr uint32_t kErrNonFinite = 1u;  // NaN / Inf in a tensor being quantized
+constexpr uint32_t kErrTimeout = 2u;    // a pipeline wait gave up
+
+// Control block at the start of every workspace (zero-filled by the caller
+// once, before first use; kernels keep the counters consistent afterwards).
+struct WsControl {
+    uint32_t error_bits;   // OR of kErr* posted since the last status query
+    uint32_t amax_ticket;  // blocks of the running amax pass that have finished
+    uint32_t reserved[6];
+    float alpha;           // tensor scale of the activation quantized in-workspace
+    uint32_t pad[55];
+};
+static_assert(sizeof(WsControl) == 256, "control block is 256 bytes");
+
+constexpr int kAmaxMaxBlocks = 2048;          // partial maxima slots
+constexpr size_t kWsPartialsOffset = 256;     // uint32 partials follow the control block
+constexpr size_t kWsControlBytes = 16384;     // control + partials, rounded up
+constexpr size_t kWsAlign = 256;
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// NVFP4 storage geometry (see include/mixquant.h for the layout).
+inline int64_t sf_atoms_per_rowblk(int64_t cols) { return ((cols + 255) / 256) * 4; }
+inline int64_t sf_rowblks(int64_t rows) { return (rows + 127) / 128; }
+inline size_t nvfp4_codes_bytes(int64_t rows, int64_t cols) { return (size_t)rows * (size_t)(cols / 2); }
+inline size_t nvfp4_scales_bytes(int64_t rows, int64_t cols)
+{
+    return (size_t)sf_rowblks(rows) * (size_t)sf_atoms_per_rowblk(cols) * 512u;
+}
+
+struct DeviceInfo {
+    int device;
+    int num_sms;
+    int cc_major, cc_minor;
+    size_t max_smem_optin;
+};
+// Cached per device; returns cudaSuccess or the error of the attribute query.
+cudaError_t device_info(DeviceInfo* out);
+
+// ----- launchers (stream-ordered, no host synchronisation) -----
+
+// amax of n BF16 values (n % 8 == 0, 16-byte aligned) -> *alpha_out = amax/2688
+// (1 if amax == 0); kErrNonFinite posted on NaN/Inf.
+cudaError_t launch_amax(const void* x, int64_t n, float* alpha_out, WsControl* ctrl, uint32_t* partials,
+                        const DeviceInfo& di, cudaStream_t s);
+
+// NVFP4 quantization of X [rows, K] (ld = K) with tensor scale *alpha.
+// interleave_half: 0, or I (= rows/2) to interleave gate/up rows in 16-row
+// groups (output row 32c+t <- input row 16c+t for t<16, I+16c+t-16 else).
+cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float* alpha, uint8_t* codes,
+                            uint8_t* scales, int64_t interleave_half, const DeviceInfo& di, cudaStream_t s);
+
+cudaError_t launch_unswizzle(const uint8_t* scales, int64_t rows, int64_t K, uint8_t* out, cudaStream_t s);
+
+// Block-scaled NVFP4 GEMM: Y[M,N] = alpha_a*alpha_b * A[M,K] B[N,K]^T.
+struct GemmArgs {
+    const uint8_t* a_codes;
+    const uint8_t* a_scales;
+    const float* a_alpha;
+    const uint8_t* b_codes;
+    const uint8_t* b_scales;
+    const float* b_alpha;
+    int64_t M, N, K;
+    int epilogue;          // 0: BF16 Y; 1: SiLU-mul + NVFP4 requantize
+    void* y;               // epilogue 0: BF16 [M, N]
+    uint8_t* h_codes;      // epilogue 1: [M, N/4] bytes (h has N/2 columns)
+    uint8_t* h_scales;     // epilogue 1: scale layout for [M, N/2]
+    const float* h_alpha;  // epilogue 1: static tensor scale of h
+    uint16_t* h_debug;     // epilogue 1, optional: BF16 h [M, N/2]
+    WsControl* ctrl;
+};
+cudaError_t launch_gemm_nvfp4(const GemmArgs& a, const DeviceInfo& di, cudaStream_t s);
+
+// BF16 decode linear: Y[M,N] = X[M,K] W[N,K]^T, FP32 accumulation.
+cudaError_t launch_decode_bf16(const void* x, int64_t M, const void* w, int64_t N, int64_t K, void* y,
+                               WsControl* ctrl, const DeviceInfo& di, cudaStream_t s);
+
+// cuTensorMapEncodeTiled obtained from the driver at run time.
+bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t outer,
+                  uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz);
+
+}  // namespace mq

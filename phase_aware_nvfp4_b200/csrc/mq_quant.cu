@@ -1,0 +1,241 @@
+// mq_quant.cu -- NVFP4 quantization on sm_100a: tensor amax (the tensor-level
+// scale) and the block quantizer, after "Mix-Quant: Quantized Prefilling,
+// Precise Decoding for Agentic LLMs", section 3.3, Eq. 2 and Eq. 3.
+//
+// Both kernels are HBM-bound streams: 128-bit coalesced loads, a handful of
+// FP32 operations per element, no shared-memory staging of the input.
+#include "mq_device.cuh"
+
+namespace mq {
+
+// ==========================================================================
+// Tensor amax -> alpha = amax / (q_max * 448)
+// ==========================================================================
+
+constexpr int kAmaxThreads = 512;
+constexpr int kAmaxUnroll = 4;
+
+// Per-halfword |bf16| maximum over the finite values of a 32-bit word pair,
+// plus a flag word that is non-zero if a NaN/Inf was seen.
+__device__ __forceinline__ void amax_accum(uint32_t w, uint32_t& mx, uint32_t& bad)
+{
+    const uint32_t mag = w & 0x7FFF7FFFu;
+    const uint32_t nonfin = __vcmpgeu2(mag, 0x7F807F80u);  // 0xFFFF per NaN/Inf halfword
+    bad |= nonfin;
+    mx = __vmaxu2(mx, mag & ~nonfin);
+}
+
+__global__ void __launch_bounds__(kAmaxThreads) amax_kernel(const uint4* __restrict__ x, int64_t n_vec,
+                                                            float* __restrict__ alpha_out, WsControl* ctrl,
+                                                            uint32_t* __restrict__ partials)
+{
+    uint32_t mx = 0, bad = 0;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    for (; i + (kAmaxUnroll - 1) * stride < n_vec; i += kAmaxUnroll * stride) {
+        uint4 v[kAmaxUnroll];
+#pragma unroll
+        for (int u = 0; u < kAmaxUnroll; ++u) v[u] = __ldcs(x + i + u * stride);
+#pragma unroll
+        for (int u = 0; u < kAmaxUnroll; ++u) {
+            amax_accum(v[u].x, mx, bad);
+            amax_accum(v[u].y, mx, bad);
+            amax_accum(v[u].z, mx, bad);
+            amax_accum(v[u].w, mx, bad);
+        }
+    }
+    for (; i < n_vec; i += stride) {
+        const uint4 v = __ldcs(x + i);
+        amax_accum(v.x, mx, bad);
+        amax_accum(v.y, mx, bad);
+        amax_accum(v.z, mx, bad);
+        amax_accum(v.w, mx, bad);
+    }
+    uint32_t m = max(mx & 0xFFFFu, mx >> 16) | (bad ? 0x80000000u : 0u);
+    // block reduction (the non-finite flag rides in bit 31)
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const uint32_t other = __shfl_xor_sync(0xFFFFFFFFu, m, o);
+        m = max(m & 0x7FFFFFFFu, other & 0x7FFFFFFFu) | ((m | other) & 0x80000000u);
+    }
+    __shared__ uint32_t warp_max[kAmaxThreads / 32];
+    __shared__ bool is_last;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (lane == 0) warp_max[warp] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t b = 0;
+        for (int w = 0; w < kAmaxThreads / 32; ++w)
+            b = max(b & 0x7FFFFFFFu, warp_max[w] & 0x7FFFFFFFu) | ((b | warp_max[w]) & 0x80000000u);
+        partials[blockIdx.x] = b;
+        __threadfence();
+        const uint32_t ticket = atomicAdd(&ctrl->amax_ticket, 1u);
+        is_last = (ticket == gridDim.x - 1);
+    }
+    __syncthreads();
+    if (!is_last) return;
+    // The last block to finish folds all partial maxima.
+    __threadfence();
+    uint32_t b = 0;
+    for (int j = threadIdx.x; j < (int)gridDim.x; j += blockDim.x) {
+        const uint32_t p = __ldcg(partials + j);
+        b = max(b & 0x7FFFFFFFu, p & 0x7FFFFFFFu) | ((b | p) & 0x80000000u);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const uint32_t other = __shfl_xor_sync(0xFFFFFFFFu, b, o);
+        b = max(b & 0x7FFFFFFFu, other & 0x7FFFFFFFu) | ((b | other) & 0x80000000u);
+    }
+    __syncthreads();
+    if (lane == 0) warp_max[warp] = b;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t r = 0;
+        for (int w = 0; w < kAmaxThreads / 32; ++w)
+            r = max(r & 0x7FFFFFFFu, warp_max[w] & 0x7FFFFFFFu) | ((r | warp_max[w]) & 0x80000000u);
+        const float amax = __uint_as_float((r & 0x7FFFu) << 16);
+        // tensor scale: amax / (q_max * E4M3_max) = amax / 2688, or 1 for an all-zero tensor
+        *alpha_out = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
+        if (r & 0x80000000u) post_error(ctrl, kErrNonFinite);
+        ctrl->amax_ticket = 0;  // ready for the next pass on this workspace
+        __threadfence();
+    }
+}
+
+cudaError_t launch_amax(const void* x, int64_t n, float* alpha_out, WsControl* ctrl, uint32_t* partials,
+                        const DeviceInfo& di, cudaStream_t s)
+{
+    const int64_t n_vec = n / 8;
+    int64_t blocks = (n_vec + kAmaxThreads * kAmaxUnroll - 1) / (kAmaxThreads * kAmaxUnroll);
+    const int64_t cap = (int64_t)di.num_sms * 4;
+    if (blocks > cap) blocks = cap;
+    if (blocks > kAmaxMaxBlocks) blocks = kAmaxMaxBlocks;
+    if (blocks < 1) blocks = 1;
+    amax_kernel<<<(unsigned)blocks, kAmaxThreads, 0, s>>>(static_cast<const uint4*>(x), n_vec, alpha_out, ctrl,
+                                                         partials);
+    return cudaGetLastError();
+}
+
+// ==========================================================================
+// Block quantizer: BF16 [rows, K] -> NVFP4 codes + E4M3 block scales
+// ==========================================================================
+//
+// One CTA tile = 128 rows x 256 columns = 4 scale atoms (2048 contiguous
+// bytes of the scale layout).  Warp w owns rows 32w..32w+31 of the tile and
+// walks them one row per step: lane l loads columns 8l..8l+7 (16 bytes), so
+// a warp step reads 512 contiguous bytes of one row and writes 128 contiguous
+// bytes of codes.  Lanes l and l^1 hold one 16-element block; one shuffle
+// gives the block amax.  Scales are staged in shared memory and written out
+// as 16-byte stores.
+
+constexpr int kQuantThreads = 128;
+constexpr int kQuantRowUnroll = 8;
+
+__global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const uint16_t* __restrict__ x, int64_t rows,
+                                                                 int64_t K, const float* __restrict__ alpha_ptr,
+                                                                 uint8_t* __restrict__ codes,
+                                                                 uint8_t* __restrict__ scales,
+                                                                 int64_t interleave_half)
+{
+    __shared__ __align__(16) uint8_t sf_stage[2048];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const float alpha = *alpha_ptr;
+    const float alpha_qmax = __fmul_rn(alpha, 6.0f);
+    const int64_t chunks = (K + 255) / 256;              // 256-column chunks per row block
+    const int64_t tiles = ((rows + 127) / 128) * chunks;
+
+    for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+        const int64_t rb = tile / chunks, kc = tile % chunks;
+        const int64_t col = kc * 256 + 8 * lane;
+        const bool col_ok = col < K;
+        for (int i0 = 0; i0 < 32; i0 += kQuantRowUnroll) {
+            uint4 v[kQuantRowUnroll];
+#pragma unroll
+            for (int u = 0; u < kQuantRowUnroll; ++u) {
+                const int64_t r = rb * 128 + 32 * warp + i0 + u;
+                v[u] = make_uint4(0u, 0u, 0u, 0u);
+                if (r < rows && col_ok) {
+                    int64_t src = r;
+                    if (interleave_half > 0) {
+                        const int64_t c = r >> 5, t = r & 31;
+                        src = (t < 16) ? (16 * c + t) : (interleave_half + 16 * c + (t - 16));
+                    }
+                    v[u] = __ldcs(reinterpret_cast<const uint4*>(x + src * K + col));
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kQuantRowUnroll; ++u) {
+                const int i = i0 + u;
+                const int64_t r = rb * 128 + 32 * warp + i;
+                const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+                float f[8];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    f[2 * j] = bf16_lo(w[j]);
+                    f[2 * j + 1] = bf16_hi(w[j]);
+                }
+                float amax = 0.0f;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(f[j]));
+                amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+                // Eq. 3: sigma_b = Pi_E4M3(amax_b / (alpha * q_max))
+                const uint32_t sc = e4m3_round_sat(__fdiv_rn(amax, alpha_qmax));
+                // Eq. 2: q_i = Pi_FP4(x_i / (alpha * sigma_b)), as |x| * fl(1/fl(alpha*sigma))
+                const float d = __fmul_rn(alpha, e4m3_to_float(sc));
+                const float enc = (d == 0.0f) ? 0.0f : __fdiv_rn(1.0f, d);
+                uint32_t packed = 0;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) packed |= e2m1_code(f[j], enc) << (4 * j);
+                const bool ok = (r < rows) && col_ok;
+                if (ok) *reinterpret_cast<uint32_t*>(codes + r * (K / 2) + col / 2) = packed;
+                if ((lane & 1) == 0) {
+                    const int kb = lane >> 1;  // 16-element block within the 256-column chunk
+                    sf_stage[(kb >> 2) * 512 + i * 16 + warp * 4 + (kb & 3)] = ok ? (uint8_t)sc : (uint8_t)0;
+                }
+            }
+        }
+        __syncthreads();
+        uint4* dst = reinterpret_cast<uint4*>(scales + (rb * chunks + kc) * 2048);
+        dst[threadIdx.x] = reinterpret_cast<const uint4*>(sf_stage)[threadIdx.x];
+        __syncthreads();
+    }
+}
+
+cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float* alpha, uint8_t* codes,
+                            uint8_t* scales, int64_t interleave_half, const DeviceInfo& di, cudaStream_t s)
+{
+    const int64_t tiles = ((rows + 127) / 128) * ((K + 255) / 256);
+    int64_t blocks = (int64_t)di.num_sms * 12;
+    if (blocks > tiles) blocks = tiles;
+    if (blocks < 1) blocks = 1;
+    quantize_kernel<<<(unsigned)blocks, kQuantThreads, 0, s>>>(static_cast<const uint16_t*>(x), rows, K, alpha,
+                                                               codes, scales, interleave_half);
+    return cudaGetLastError();
+}
+
+// ==========================================================================
+// Scale layout -> plain row-major [rows, K/16] (test and inspection helper)
+// ==========================================================================
+
+__global__ void unswizzle_kernel(const uint8_t* __restrict__ scales, int64_t rows, int64_t nb,
+                                 int64_t atoms_per_rowblk, uint8_t* __restrict__ out)
+{
+    const int64_t total = rows * nb;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = i / nb, b = i % nb;
+        out[i] = scales[sf_offset(r, b, atoms_per_rowblk)];
+    }
+}
+
+cudaError_t launch_unswizzle(const uint8_t* scales, int64_t rows, int64_t K, uint8_t* out, cudaStream_t s)
+{
+    const int64_t total = rows * (K / 16);
+    int64_t blocks = (total + 255) / 256;
+    if (blocks > 65535) blocks = 65535;
+    if (blocks < 1) blocks = 1;
+    unswizzle_kernel<<<(unsigned)blocks, 256, 0, s>>>(scales, rows, K / 16, sf_atoms_per_rowblk(K), out);
+    return cudaGetLastError();
+}
+
+}  // namespace mq

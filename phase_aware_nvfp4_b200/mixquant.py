@@ -1,0 +1,232 @@
+"""Thin ctypes binding of libmixquant (include/mixquant.h).
+
+Argument marshalling only: every step of the path runs in the CUDA library.
+PyTorch provides the device buffers (``torch.empty`` on the current CUDA
+device) and the stream (``torch.cuda.current_stream()``).  The binding never
+computes anything itself and has no fallback: if ``libmixquant.so`` is
+missing or a call returns an error, it raises.
+
+Names mirror the C ABI: ``quantize_weight``, ``quantize_activation``,
+``prefill_linear``, ``decode_linear``, ``unswizzle_scales``,
+``async_status``, ``nvfp4_sizes``, ``workspace_bytes``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from dataclasses import dataclass
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmixquant.so")
+
+MQ_OK = 0
+MQ_EPI_BF16 = 0
+MQ_EPI_SILU_MUL_NVFP4 = 1
+WS_CONTROL_BYTES = 16384
+
+STATUS_NAMES = {0: "MQ_OK", 1: "MQ_ERR_INVALID_ARG", 2: "MQ_ERR_SHAPE", 3: "MQ_ERR_ALIGNMENT",
+                4: "MQ_ERR_WORKSPACE", 5: "MQ_ERR_NONFINITE", 6: "MQ_ERR_TIMEOUT", 7: "MQ_ERR_CUDA",
+                8: "MQ_ERR_DEVICE"}
+
+# Every symbol the header declares (checked by the ABI tests).
+EXPORTS = ("mq_status_string", "mq_version", "mq_nvfp4_sizes", "mq_workspace_bytes", "mq_quantize_weight",
+           "mq_quantize_activation", "mq_prefill_linear", "mq_decode_linear", "mq_unswizzle_scales",
+           "mq_async_status")
+
+
+class MQError(RuntimeError):
+    def __init__(self, status: int, call: str):
+        self.status = int(status)
+        super().__init__(f"{call} failed: {STATUS_NAMES.get(self.status, self.status)}")
+
+
+class _NVFP4(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("alpha", ctypes.c_void_p),
+                ("rows", ctypes.c_int64), ("cols", ctypes.c_int64)]
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Load libmixquant.so (raises FileNotFoundError if it was not built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(path):
+                raise FileNotFoundError(
+                    f"{path} is missing: build it with `python -m phase_aware_nvfp4_b200.build`")
+            lib = ctypes.CDLL(path)
+            vp, i64, sz, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int
+            nvp = ctypes.POINTER(_NVFP4)
+            lib.mq_status_string.argtypes = [i32]
+            lib.mq_status_string.restype = ctypes.c_char_p
+            lib.mq_version.argtypes = []
+            lib.mq_version.restype = ctypes.c_char_p
+            lib.mq_nvfp4_sizes.argtypes = [i64, i64, ctypes.POINTER(sz), ctypes.POINTER(sz)]
+            lib.mq_nvfp4_sizes.restype = i32
+            lib.mq_workspace_bytes.argtypes = [i64, i64]
+            lib.mq_workspace_bytes.restype = sz
+            lib.mq_quantize_weight.argtypes = [vp, i64, i64, i32, nvp, vp, sz, vp]
+            lib.mq_quantize_weight.restype = i32
+            lib.mq_quantize_activation.argtypes = [vp, i64, i64, vp, nvp, vp, sz, vp]
+            lib.mq_quantize_activation.restype = i32
+            lib.mq_prefill_linear.argtypes = [vp, nvp, i64, nvp, i32, vp, vp, vp, nvp, vp, vp, sz, vp]
+            lib.mq_prefill_linear.restype = i32
+            lib.mq_decode_linear.argtypes = [vp, i64, vp, i64, i64, vp, vp, sz, vp]
+            lib.mq_decode_linear.restype = i32
+            lib.mq_unswizzle_scales.argtypes = [nvp, vp, vp]
+            lib.mq_unswizzle_scales.restype = i32
+            lib.mq_async_status.argtypes = [vp, vp]
+            lib.mq_async_status.restype = i32
+            _lib = lib
+    return _lib
+
+
+def _check(status: int, call: str):
+    if status != MQ_OK:
+        raise MQError(status, call)
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream(stream=None):
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+# ----------------------------------------------------------------- tensors
+
+@dataclass
+class NVFP4Tensor:
+    """Device buffers of an NVFP4 [rows, cols] tensor (layout in include/mixquant.h)."""
+    codes: object    # torch.uint8 [rows, cols/2]
+    scales: object   # torch.uint8 [scales_bytes] in the MMA scale layout
+    alpha: object    # torch.float32 [1]
+    rows: int
+    cols: int
+
+    def c(self) -> _NVFP4:
+        return _NVFP4(self.codes.data_ptr(), self.scales.data_ptr(), self.alpha.data_ptr(), self.rows, self.cols)
+
+
+def nvfp4_sizes(rows: int, cols: int):
+    cb, sb = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    _check(load().mq_nvfp4_sizes(rows, cols, ctypes.byref(cb), ctypes.byref(sb)), "mq_nvfp4_sizes")
+    return cb.value, sb.value
+
+
+def workspace_bytes(M: int = 0, K: int = 0) -> int:
+    return int(load().mq_workspace_bytes(M, K))
+
+
+def nvfp4_empty(rows: int, cols: int, device=None) -> NVFP4Tensor:
+    torch = _torch()
+    device = device or torch.device("cuda", torch.cuda.current_device())
+    cb, sb = nvfp4_sizes(rows, cols)
+    return NVFP4Tensor(torch.empty((rows, cols // 2), dtype=torch.uint8, device=device),
+                       torch.zeros(sb, dtype=torch.uint8, device=device),
+                       torch.zeros(1, dtype=torch.float32, device=device), rows, cols)
+
+
+def workspace(M: int = 0, K: int = 0, device=None):
+    """A zero-filled workspace for an M x K activation (16-byte aligned)."""
+    torch = _torch()
+    device = device or torch.device("cuda", torch.cuda.current_device())
+    return torch.zeros(workspace_bytes(M, K), dtype=torch.uint8, device=device)
+
+
+def _ws_args(ws):
+    return _ptr(ws), ctypes.c_size_t(ws.numel())
+
+
+# ----------------------------------------------------------------- calls
+
+def quantize_weight(W, gate_up_interleave: bool = False, out: NVFP4Tensor | None = None, ws=None,
+                    stream=None) -> NVFP4Tensor:
+    """mq_quantize_weight: BF16 [N, K] -> NVFP4 (offline, dynamic alpha_w)."""
+    N, K = W.shape
+    out = out or nvfp4_empty(N, K, W.device)
+    ws = ws if ws is not None else workspace(device=W.device)
+    cs = out.c()
+    _check(load().mq_quantize_weight(_ptr(W), N, K, int(bool(gate_up_interleave)), ctypes.byref(cs),
+                                     *_ws_args(ws), _stream(stream)), "mq_quantize_weight")
+    return out
+
+
+def quantize_activation(X, alpha_static=None, out: NVFP4Tensor | None = None, ws=None,
+                        stream=None) -> NVFP4Tensor:
+    """mq_quantize_activation: BF16 [M, K] -> NVFP4 (dynamic alpha unless alpha_static)."""
+    M, K = X.shape
+    out = out or nvfp4_empty(M, K, X.device)
+    ws = ws if ws is not None else workspace(device=X.device)
+    cs = out.c()
+    _check(load().mq_quantize_activation(_ptr(X), M, K, _ptr(alpha_static), ctypes.byref(cs), *_ws_args(ws),
+                                         _stream(stream)), "mq_quantize_activation")
+    return out
+
+
+def prefill_linear(X=None, W: NVFP4Tensor = None, *, Xq: NVFP4Tensor | None = None, epilogue: int = MQ_EPI_BF16,
+                   alpha_static=None, alpha_h=None, Y=None, H: NVFP4Tensor | None = None, h_debug=None, ws=None,
+                   stream=None):
+    """mq_prefill_linear.  Returns Y (BF16 [M, N]) or H (NVFP4 [M, N/2])."""
+    torch = _torch()
+    if (X is None) == (Xq is None):
+        raise ValueError("give exactly one of X (BF16) and Xq (NVFP4)")
+    M = X.shape[0] if X is not None else Xq.rows
+    K = W.cols
+    N = W.rows
+    dev = W.codes.device
+    if ws is None:
+        ws = workspace(M, K, dev) if X is not None else workspace(device=dev)
+    xq_c = Xq.c() if Xq is not None else None
+    w_c = W.c()
+    h_c = None
+    if epilogue == MQ_EPI_BF16:
+        Y = Y if Y is not None else torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    else:
+        H = H or nvfp4_empty(M, N // 2, dev)
+        h_c = H.c()
+    _check(load().mq_prefill_linear(_ptr(X), ctypes.byref(xq_c) if xq_c is not None else None, M,
+                                    ctypes.byref(w_c), int(epilogue), _ptr(alpha_static), _ptr(alpha_h),
+                                    _ptr(Y) if epilogue == MQ_EPI_BF16 else None,
+                                    ctypes.byref(h_c) if h_c is not None else None, _ptr(h_debug), *_ws_args(ws),
+                                    _stream(stream)), "mq_prefill_linear")
+    return Y if epilogue == MQ_EPI_BF16 else H
+
+
+def decode_linear(X, W, Y=None, ws=None, stream=None):
+    """mq_decode_linear: BF16 Y[M, N] = X[M, K] W[N, K]^T (M <= 256)."""
+    torch = _torch()
+    M, K = X.shape
+    N = W.shape[0]
+    Y = Y if Y is not None else torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    ws = ws if ws is not None else workspace(device=X.device)
+    _check(load().mq_decode_linear(_ptr(X), M, _ptr(W), N, K, _ptr(Y), *_ws_args(ws), _stream(stream)),
+           "mq_decode_linear")
+    return Y
+
+
+def unswizzle_scales(t: NVFP4Tensor, out=None, stream=None):
+    """mq_unswizzle_scales: MMA scale layout -> row-major uint8 [rows, cols/16]."""
+    torch = _torch()
+    out = out if out is not None else torch.empty((t.rows, t.cols // 16), dtype=torch.uint8,
+                                                  device=t.scales.device)
+    cs = t.c()
+    _check(load().mq_unswizzle_scales(ctypes.byref(cs), _ptr(out), _stream(stream)), "mq_unswizzle_scales")
+    return out
+
+
+def async_status(ws, stream=None) -> int:
+    """mq_async_status: synchronize the stream, return and clear the device error bits."""
+    return int(load().mq_async_status(_ptr(ws), _stream(stream)))

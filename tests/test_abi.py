@@ -1,0 +1,127 @@
+"""The C ABI library on a machine without a GPU: it loads, exports every
+declared symbol, and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from phase_aware_nvfp4_b200 import mixquant as mqb
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mixquant.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(mqb.LIB_PATH):
+        from phase_aware_nvfp4_b200 import build
+        build.build()
+    return mqb.load()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"MQ_API\s+[\w\s\*]+?\b(mq_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_exports():
+    assert declared_symbols() == sorted(mqb.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+
+
+def test_only_mq_symbols_are_exported(lib):
+    out = os.popen(f"nm -D --defined-only {mqb.LIB_PATH}").read()
+    names = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+    assert set(declared_symbols()) <= names
+    assert all(n.startswith("mq_") for n in names), sorted(n for n in names if not n.startswith("mq_"))
+
+
+def test_status_strings_and_version(lib):
+    for code, name in mqb.STATUS_NAMES.items():
+        assert lib.mq_status_string(code).decode() == name
+    assert lib.mq_version().decode() == "0.1.0"
+
+
+def test_sizes(lib):
+    cb, sb = mqb.nvfp4_sizes(8192, 4096)
+    assert cb == 8192 * 2048
+    assert sb == 64 * 16 * 2048            # 64 row blocks x 16 chunks of 4 atoms
+    cb, sb = mqb.nvfp4_sizes(200, 320)
+    assert cb == 200 * 160
+    assert sb == 2 * 8 * 512               # 320 cols -> 2 chunks of 256 -> 8 atoms per row block
+    assert mqb.workspace_bytes(0, 0) == mqb.WS_CONTROL_BYTES
+    assert mqb.workspace_bytes(8192, 4096) >= mqb.WS_CONTROL_BYTES + cb
+    with pytest.raises(mqb.MQError):
+        mqb.nvfp4_sizes(8, 100)
+
+
+class _NV(ctypes.Structure):
+    _fields_ = mqb._NVFP4._fields_
+
+
+def _nv(rows, cols, base=0x10000000):
+    return mqb._NVFP4(base, base + 0x1000000, base + 0x2000000, rows, cols)
+
+
+def test_argument_errors_are_synchronous(lib):
+    """Validation happens on the host before any launch; no GPU is needed to see it."""
+    P = 0x7F0000000000
+    ws, wsb = ctypes.c_void_p(P), ctypes.c_size_t(1 << 30)
+    w = _nv(256, 256)
+    # null / bad enum
+    assert lib.mq_prefill_linear(None, None, 128, ctypes.byref(w), 0, None, None, P, None, None, ws, wsb, None) == 1
+    assert lib.mq_prefill_linear(P, None, 128, ctypes.byref(w), 7, None, None, P, None, None, ws, wsb, None) == 1
+    # shapes: K % 64, N % 16, M range
+    bad_k = _nv(256, 200)
+    assert lib.mq_prefill_linear(P, None, 128, ctypes.byref(bad_k), 0, None, None, P, None, None, ws, wsb, None) == 2
+    bad_n = _nv(250, 256)
+    assert lib.mq_prefill_linear(P, None, 128, ctypes.byref(bad_n), 0, None, None, P, None, None, ws, wsb, None) == 2
+    assert lib.mq_prefill_linear(P, None, 0, ctypes.byref(w), 0, None, None, P, None, None, ws, wsb, None) == 2
+    # alignment
+    assert lib.mq_prefill_linear(P + 2, None, 128, ctypes.byref(w), 0, None, None, P, None, None, ws, wsb,
+                                 None) == 3
+    # workspace too small for in-workspace activation quantization
+    assert lib.mq_prefill_linear(P, None, 128, ctypes.byref(w), 0, None, None, P, None, None, ws,
+                                 ctypes.c_size_t(100), None) == 4
+    # fused epilogue needs N % 128 and an H_out of [M, N/2]
+    h = _nv(128, 128)
+    assert lib.mq_prefill_linear(P, None, 128, ctypes.byref(w), 1, None, P, None, None, None, ws, wsb, None) == 1
+    h_bad = _nv(128, 64)
+    assert lib.mq_prefill_linear(P, None, 128, ctypes.byref(w), 1, None, P, None, ctypes.byref(h_bad), None, ws,
+                                 wsb, None) == 2
+    # decode: M in [1, 256]
+    assert lib.mq_decode_linear(P, 300, P, 256, 256, P, ws, wsb, None) == 2
+    assert lib.mq_decode_linear(P, 4, P, 256, 100, P, ws, wsb, None) == 2
+    assert lib.mq_decode_linear(None, 4, P, 256, 256, P, ws, wsb, None) == 1
+    # weight quantization: interleave needs N % 128
+    out = _nv(200, 256)
+    assert lib.mq_quantize_weight(P, 200, 256, 1, ctypes.byref(out), ws, wsb, None) == 2
+    assert lib.mq_quantize_weight(P, 200, 256, 0, None, ws, wsb, None) == 1
+    assert lib.mq_async_status(None, None) == 1
+    del h
+
+
+def test_valid_call_without_gpu_reports_cuda_or_device_error(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    P = 0x7F0000000000
+    w = _nv(256, 256)
+    st = lib.mq_prefill_linear(P, None, 128, ctypes.byref(w), 0, None, None, P, None, None, ctypes.c_void_p(P),
+                               ctypes.c_size_t(1 << 30), None)
+    assert st in (7, 8)
+
+
+def test_binding_raises_when_library_missing(tmp_path):
+    saved = mqb._lib
+    try:
+        mqb._lib = None
+        with pytest.raises(FileNotFoundError):
+            mqb.load(str(tmp_path / "nope.so"))
+    finally:
+        mqb._lib = saved

@@ -1,0 +1,159 @@
+"""GPU quantizer (tensor amax + Eq. 2 / Eq. 3 block quantizer) vs the oracle:
+codes, block scales and the tensor scale must be bit-exact."""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from phase_aware_nvfp4_b200 import mixquant as mq
+from phase_aware_nvfp4_b200 import workloads as wl
+
+from gpu_helpers import nvfp4_host, require_gpu, scales_from_layout, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    require_gpu()
+
+
+def _check_quant(x_bits, t, alpha_expected=None):
+    codes, scales, alpha = nvfp4_host(t)
+    if alpha_expected is None:
+        _, alpha_expected, _ = oracle.tensor_alpha(x_bits)
+    assert np.float32(alpha) == np.float32(alpha_expected)
+    rc, rs = oracle.quantize(x_bits, alpha_expected)
+    assert np.array_equal(scales, rs), f"{int((scales != rs).sum())} scale mismatches"
+    assert np.array_equal(codes, rc), f"{int((codes != rc).sum())} code byte mismatches"
+
+
+@pytest.mark.parametrize("M,K,kind", [(128, 256, "normal"), (200, 320, "heavy"), (1, 64, "heavy"),
+                                      (129, 4096, "heavy"), (513, 1088, "heavy")])
+def test_quantize_activation_bit_exact(M, K, kind):
+    x = wl.normal_bf16(M, K, 1.0, 3) if kind == "normal" else wl.heavy_tailed_bf16(M, K, 5)
+    t = mq.quantize_activation(to_dev(x))
+    torch.cuda.synchronize()
+    _check_quant(x, t)
+
+
+def test_tiny_workload_quantization():
+    """The tiny 128x256x256 workload: X ~ N(0,1), W ~ N(0, 0.02^2), seed 0."""
+    p = wl.tiny().projections[0]
+    x, w = wl.make_x(p), wl.make_w(p)
+    _check_quant(x, mq.quantize_activation(to_dev(x)))
+    _check_quant(w, mq.quantize_weight(to_dev(w)))
+
+
+def test_golden_blocks_on_gpu():
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "handworked_blocks.json")))
+    x = np.concatenate([wl.f32_to_bf16_bits(np.asarray(b["x"], np.float32)) for b in g["blocks"]])[None, :]
+    t = mq.quantize_activation(to_dev(x))
+    codes, scales, alpha = nvfp4_host(t)
+    assert alpha == 1.0
+    for i, b in enumerate(g["blocks"]):
+        assert scales[0, i] == b["sigma_code"], b["name"]
+        got = [(int(codes[0, 8 * i + j // 2]) >> (4 * (j % 2))) & 15 for j in range(16)]
+        assert got == b["codes"], b["name"]
+
+
+def test_every_e2m1_tie_and_e4m3_midpoint():
+    """Blocks built so that |x|/(alpha sigma) hits every E2M1 tie and the block
+    quotient hits E4M3 midpoints (alpha = 1 via a 2688 anchor)."""
+    rng = np.random.default_rng(1)
+    grid = np.array([oracle.e4m3_value(c) for c in range(0x7F)])
+    mids = (grid[1:] + grid[:-1]) / 2
+    rows = []
+    anchor = np.zeros(16, np.float32)
+    anchor[0] = 2688.0
+    rows.append(anchor)
+    for m in mids[mids * 6 < 2000][::2]:
+        blk = np.zeros(16, np.float32)
+        blk[0] = m * 6           # amax_b / 6 = midpoint (not always BF16-exact; rounding is part of the test)
+        ties = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0]) * m
+        blk[1:8] = ties
+        blk[8:15] = -ties
+        blk[15] = rng.standard_normal() * m
+        rows.append(blk)
+    v = np.concatenate(rows)
+    pad = (-len(v)) % 64
+    v = np.concatenate([v, np.zeros(pad, np.float32)]).reshape(1, -1)
+    x = wl.f32_to_bf16_bits(v)
+    _check_quant(x, mq.quantize_activation(to_dev(x)))
+
+
+def test_static_alpha_and_saturation():
+    x = wl.heavy_tailed_bf16(256, 512, 8)
+    alpha = np.float32(0.01)   # far too small: many blocks clip at sigma = 448 and codes at 6
+    t = mq.quantize_activation(to_dev(x), alpha_static=torch.tensor([alpha], device="cuda"))
+    _check_quant(x, t, alpha_expected=float(alpha))
+    _, scales, _ = nvfp4_host(t)
+    assert (scales == 0x7E).any()
+
+
+def test_zero_and_negative_zero_and_tiny():
+    x = np.zeros((128, 256), np.uint16)
+    x[0, 1] = 0x8000                       # -0.0
+    x[1, :16] = wl.f32_to_bf16_bits(np.full(16, 2.0 ** -12, np.float32))
+    x[2, :] = wl.f32_to_bf16_bits(np.full(256, -1e-30, np.float32))
+    t = mq.quantize_activation(to_dev(x))
+    _check_quant(x, t)
+    z = mq.quantize_activation(to_dev(np.zeros((64, 64), np.uint16)))
+    assert float(z.alpha.cpu()[0]) == 1.0
+
+
+def test_weight_quantization_and_gate_up_interleave():
+    I, K = 256, 512
+    w = wl.normal_bf16(2 * I, K, 0.02, 77)
+    plain = mq.quantize_weight(to_dev(w))
+    _check_quant(w, plain)
+    inter = mq.quantize_weight(to_dev(w), gate_up_interleave=True)
+    perm = np.empty(2 * I, np.int64)
+    for r in range(2 * I):
+        c, t = divmod(r, 32)
+        perm[r] = 16 * c + t if t < 16 else I + 16 * c + (t - 16)
+    codes, scales, alpha = nvfp4_host(inter)
+    _, a_ref, _ = oracle.tensor_alpha(w)
+    rc, rs = oracle.quantize(w, a_ref)
+    assert alpha == a_ref
+    assert np.array_equal(codes, rc[perm]) and np.array_equal(scales, rs[perm])
+
+
+def test_unswizzle_matches_layout_mapping_and_padding_is_zero():
+    x = wl.heavy_tailed_bf16(200, 320, 9)
+    t = mq.quantize_activation(to_dev(x))
+    dev_rm = mq.unswizzle_scales(t).cpu().numpy()
+    buf = t.scales.cpu().numpy()
+    assert np.array_equal(dev_rm, scales_from_layout(buf, 200, 320))
+    mask = np.zeros(buf.size, bool)
+    atoms = 8
+    r = np.arange(200)[:, None]
+    kb = np.arange(20)[None, :]
+    off = ((r // 128) * atoms + kb // 4) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + (kb % 4)
+    mask[off.ravel()] = True
+    assert not buf[~mask].any(), "padding rows / atoms must hold zero scales"
+
+
+def test_nonfinite_input_is_reported():
+    x = wl.heavy_tailed_bf16(128, 256, 2)
+    x[5, 7] = 0x7FC0
+    ws = mq.workspace()
+    mq.quantize_activation(to_dev(x), ws=ws)
+    assert mq.async_status(ws) == 5        # MQ_ERR_NONFINITE
+    assert mq.async_status(ws) == 0        # cleared
+    mq.quantize_activation(to_dev(wl.heavy_tailed_bf16(128, 256, 2)), ws=ws)
+    assert mq.async_status(ws) == 0
+
+
+def test_repeated_amax_on_one_workspace():
+    """The amax pass resets its block counter: back-to-back calls on one workspace stay exact."""
+    ws = mq.workspace()
+    for seed in range(4):
+        x = wl.heavy_tailed_bf16(300, 1024, 100 + seed)
+        t = mq.quantize_activation(to_dev(x), ws=ws)
+        torch.cuda.synchronize()
+        _check_quant(x, t)
+    assert mq.async_status(ws) == 0
