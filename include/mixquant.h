@@ -159,6 +159,35 @@ MQ_API mq_status mq_prefill_linear(const void* X_bf16, const mq_nvfp4* X_q, int6
 MQ_API mq_status mq_decode_linear(const void* X_bf16, int64_t M, const void* W_bf16, int64_t N, int64_t K, void* Y_bf16,
                            void* ws, size_t ws_bytes, mq_stream_t stream);
 
+/*
+ * mq_prefill_linear_noalloc -- the same NVFP4 prefill linear layer (dynamic
+ * or static activation scale, BF16 epilogue) for callers that cannot
+ * allocate device memory and so cannot pass a workspace: for example a
+ * plugin of an inference engine that owns all device memory and may not
+ * allocate when it is enqueued, or a latency-critical serving loop that must
+ * not call cudaMalloc (it can synchronize the whole device).  The paper has
+ * no counterpart of this call; it is a deployment convenience.
+ *
+ * The scratch this call needs (control block + the NVFP4 copy of X) lives in
+ * a static device array of MQ_NOALLOC_SCRATCH_BYTES that every GPU loading
+ * the library holds until the process exits.  Arguments are those of
+ * mq_prefill_linear with X_bf16 given and epi = MQ_EPI_BF16; inputs and
+ * outputs are still caller-owned device buffers.
+ *   - M x K activations whose NVFP4 copy does not fit the array are rejected
+ *     with MQ_ERR_WORKSPACE (the limit admits e.g. M = 8192 with K = 12288).
+ *   - The first call on a device sets the array up (looks up its address,
+ *     zeroes its control block, synchronizes that device); make that first
+ *     call before any stream capture.
+ *   - All calls share the one array: calls that overlap on the GPU (other
+ *     streams, other host threads) race.  Serialize them.
+ *   - Device-side errors (NaN/Inf in X, a pipeline timeout) are not reported
+ *     by this call; mq_prefill_linear with a workspace reports them.
+ * It calls no cudaMalloc, cudaFree or allocating library routine.
+ */
+#define MQ_NOALLOC_SCRATCH_BYTES (64u << 20)
+MQ_API mq_status mq_prefill_linear_noalloc(const void* X_bf16, int64_t M, const mq_nvfp4* W,
+                                           const float* alpha_static, void* Y_bf16, mq_stream_t stream);
+
 /* Copy the block scales of `t` to plain row-major [rows, cols/16] bytes. */
 MQ_API mq_status mq_unswizzle_scales(const mq_nvfp4* t, uint8_t* rowmajor_out, mq_stream_t stream);
 

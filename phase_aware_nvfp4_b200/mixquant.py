@@ -32,7 +32,8 @@ STATUS_NAMES = {0: "MQ_OK", 1: "MQ_ERR_INVALID_ARG", 2: "MQ_ERR_SHAPE", 3: "MQ_E
 # Every symbol the header declares (checked by the ABI tests).
 EXPORTS = ("mq_status_string", "mq_version", "mq_nvfp4_sizes", "mq_workspace_bytes", "mq_quantize_weight",
            "mq_quantize_activation", "mq_prefill_linear", "mq_decode_linear", "mq_unswizzle_scales",
-           "mq_async_status")
+           "mq_async_status", "mq_prefill_linear_noalloc")
+NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
 class MQError(RuntimeError):
@@ -81,6 +82,8 @@ def load(path: str = LIB_PATH):
             lib.mq_unswizzle_scales.restype = i32
             lib.mq_async_status.argtypes = [vp, vp]
             lib.mq_async_status.restype = i32
+            lib.mq_prefill_linear_noalloc.argtypes = [vp, i64, nvp, vp, vp, vp]
+            lib.mq_prefill_linear_noalloc.restype = i32
             _lib = lib
     return _lib
 
@@ -203,6 +206,17 @@ def prefill_linear(X=None, W: NVFP4Tensor = None, *, Xq: NVFP4Tensor | None = No
                                     ctypes.byref(h_c) if h_c is not None else None, _ptr(h_debug), *_ws_args(ws),
                                     _stream(stream)), "mq_prefill_linear")
     return Y if epilogue == MQ_EPI_BF16 else H
+
+
+def prefill_linear_noalloc(X, W: NVFP4Tensor, alpha_static=None, Y=None, stream=None):
+    """mq_prefill_linear_noalloc: prefill linear without a workspace (static device scratch)."""
+    torch = _torch()
+    M = X.shape[0]
+    Y = Y if Y is not None else torch.empty((M, W.rows), dtype=torch.bfloat16, device=X.device)
+    w_c = W.c()
+    _check(load().mq_prefill_linear_noalloc(_ptr(X), M, ctypes.byref(w_c), _ptr(alpha_static), _ptr(Y),
+                                            _stream(stream)), "mq_prefill_linear_noalloc")
+    return Y
 
 
 def decode_linear(X, W, Y=None, ws=None, stream=None):
