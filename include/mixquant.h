@@ -191,6 +191,14 @@ MQ_API mq_status mq_prefill_linear_noalloc(const void* X_bf16, int64_t M, const 
 /* Copy the block scales of `t` to plain row-major [rows, cols/16] bytes. */
 MQ_API mq_status mq_unswizzle_scales(const mq_nvfp4* t, uint8_t* rowmajor_out, mq_stream_t stream);
 
+/* Self-test of the device E2M1 rounding used by the quantizers: for every
+ * FP32 value v in [0, 8] and -v, compares the sm_100 conversion instruction
+ * (cvt.rn.satfinite.e2m1x2.f32) with the definition of Pi_FP4 in Eq. 2
+ * (nearest E2M1 magnitude, ties to even, clipped at 6, sign kept) and ADDS the
+ * numbers of mismatches to mismatch_counts[0] (positive v) and [1] (negative
+ * v), two device uint64 the caller zero-fills.  Both must stay 0. */
+MQ_API mq_status mq_selftest_e2m1(unsigned long long* mismatch_counts, mq_stream_t stream);
+
 /* Synchronize `stream`, then read and clear the asynchronous error bits of
  * workspace `ws`: MQ_OK, MQ_ERR_NONFINITE, MQ_ERR_TIMEOUT (or MQ_ERR_CUDA if
  * the synchronization itself failed). */

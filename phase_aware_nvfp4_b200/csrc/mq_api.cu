@@ -317,6 +317,16 @@ mq_status mq_unswizzle_scales(const mq_nvfp4* t, uint8_t* rowmajor_out, mq_strea
                                         reinterpret_cast<cudaStream_t>(stream)));
 }
 
+mq_status mq_selftest_e2m1(unsigned long long* mismatch_counts, mq_stream_t stream)
+{
+    if (mismatch_counts == nullptr) return MQ_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(mismatch_counts) & 7u) != 0) return MQ_ERR_ALIGNMENT;
+    DeviceInfo di;
+    mq_status st = check_device(&di);
+    if (st != MQ_OK) return st;
+    return cuda_status(launch_selftest_e2m1(mismatch_counts, di, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 mq_status mq_async_status(void* ws, mq_stream_t stream)
 {
     if (ws == nullptr) return MQ_ERR_INVALID_ARG;

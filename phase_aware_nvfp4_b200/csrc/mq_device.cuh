@@ -292,11 +292,61 @@ __device__ __forceinline__ uint32_t e2m1_index(float m)
 }
 
 // 4-bit code of one element: sign bit of x, magnitude index of |x| * enc.
+// (Definition-based form; the kernels use the conversion instruction below,
+// and the self-test checks the two agree on every input.)
 __device__ __forceinline__ uint32_t e2m1_code(float x, float enc)
 {
     const float a = fabsf(x);
     const uint32_t idx = (a == 0.0f) ? 0u : e2m1_index(__fmul_rn(a, enc));
     return ((__float_as_uint(x) >> 28) & 8u) | idx;
+}
+
+// Eight E2M1 codes packed into 32 bits (element j in bits 4j..4j+3) from
+// eight already-scaled values, by the sm_100 conversion instruction: round
+// to nearest even on the E2M1 grid, saturating at +-6, sign kept (also on
+// zero).  Each cvt packs two values: the first source lands in the upper
+// nibble.
+__device__ __forceinline__ uint32_t e2m1x8_cvt(float v0, float v1, float v2, float v3, float v4, float v5,
+                                               float v6, float v7)
+{
+    uint32_t out;
+    asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q3, %8, %7;\n\t"
+        "mov.b32 %0, {q0, q1, q2, q3};\n\t}"
+        : "=r"(out)
+        : "f"(v0), "f"(v1), "f"(v2), "f"(v3), "f"(v4), "f"(v5), "f"(v6), "f"(v7));
+    return out;
+}
+
+// Codes of eight values x[0..7] with encode scale enc = fl(1 / fl(alpha * sigma)):
+// code = Pi_FP4(x * enc) with the sign of x.  When enc overflowed to +inf
+// (alpha * sigma below 2^-128) a zero x would give 0 * inf = NaN, so that rare
+// block takes the element-wise path, which maps zeros to a signed zero code.
+__device__ __forceinline__ uint32_t e2m1x8_encode(const float (&x)[8], float enc)
+{
+    if (isinf(enc)) {
+        uint32_t out = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) out |= e2m1_code(x[j], enc) << (4 * j);
+        return out;
+    }
+    return e2m1x8_cvt(__fmul_rn(x[0], enc), __fmul_rn(x[1], enc), __fmul_rn(x[2], enc), __fmul_rn(x[3], enc),
+                      __fmul_rn(x[4], enc), __fmul_rn(x[5], enc), __fmul_rn(x[6], enc), __fmul_rn(x[7], enc));
+}
+
+// |bf16| maximum of 16 values held as 8 packed words (exact, NaN/Inf not
+// expected: a non-finite input is reported by the amax pass).
+__device__ __forceinline__ float bf16x16_absmax(const uint32_t (&w)[8])
+{
+    uint32_t m = __vmaxu2(w[0] & 0x7FFF7FFFu, w[1] & 0x7FFF7FFFu);
+    m = __vmaxu2(m, __vmaxu2(w[2] & 0x7FFF7FFFu, w[3] & 0x7FFF7FFFu));
+    m = __vmaxu2(m, __vmaxu2(__vmaxu2(w[4] & 0x7FFF7FFFu, w[5] & 0x7FFF7FFFu),
+                             __vmaxu2(w[6] & 0x7FFF7FFFu, w[7] & 0x7FFF7FFFu)));
+    const uint32_t b = max(m & 0xFFFFu, m >> 16);
+    return __uint_as_float(b << 16);
 }
 
 // Byte offset of scale (row r, 16-element block kb) in the MMA scale layout:

@@ -97,9 +97,10 @@ __device__ __forceinline__ void silu_mul_quant_chunk(const uint32_t (&acc)[32], 
     const uint32_t sc = e4m3_round_sat(__fdiv_rn(amax, alpha_h_qmax));
     const float d = __fmul_rn(alpha_h, e4m3_to_float(sc));
     const float enc = (d == 0.0f) ? 0.0f : __fdiv_rn(1.0f, d);
-    codes[0] = codes[1] = 0;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) codes[j >> 3] |= e2m1_code(h[j], enc) << (4 * (j & 7));
+    const float h0[8] = {h[0], h[1], h[2], h[3], h[4], h[5], h[6], h[7]};
+    const float h1[8] = {h[8], h[9], h[10], h[11], h[12], h[13], h[14], h[15]};
+    codes[0] = e2m1x8_encode(h0, enc);
+    codes[1] = e2m1x8_encode(h1, enc);
     scale = sc;
 }
 

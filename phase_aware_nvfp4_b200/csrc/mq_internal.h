@@ -66,6 +66,10 @@ cudaError_t launch_amax(const void* x, int64_t n, float* alpha_out, WsControl* c
 cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float* alpha, uint8_t* codes,
                             uint8_t* scales, int64_t interleave_half, const DeviceInfo& di, cudaStream_t s);
 
+// Sweep of the E2M1 conversion instruction against the definition; adds
+// mismatch counts for positive / negative inputs into counts[0] / counts[1].
+cudaError_t launch_selftest_e2m1(unsigned long long* counts, const DeviceInfo& di, cudaStream_t s);
+
 cudaError_t launch_unswizzle(const uint8_t* scales, int64_t rows, int64_t K, uint8_t* out, cudaStream_t s);
 
 // Block-scaled NVFP4 GEMM: Y[M,N] = alpha_a*alpha_b * A[M,K] B[N,K]^T.

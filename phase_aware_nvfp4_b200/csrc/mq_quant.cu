@@ -35,7 +35,7 @@ __global__ void __launch_bounds__(kAmaxThreads) amax_kernel(const uint4* __restr
     for (; i + (kAmaxUnroll - 1) * stride < n_vec; i += kAmaxUnroll * stride) {
         uint4 v[kAmaxUnroll];
 #pragma unroll
-        for (int u = 0; u < kAmaxUnroll; ++u) v[u] = __ldcs(x + i + u * stride);
+        for (int u = 0; u < kAmaxUnroll; ++u) v[u] = __ldg(x + i + u * stride);
 #pragma unroll
         for (int u = 0; u < kAmaxUnroll; ++u) {
             amax_accum(v[u].x, mx, bad);
@@ -45,7 +45,7 @@ __global__ void __launch_bounds__(kAmaxThreads) amax_kernel(const uint4* __restr
         }
     }
     for (; i < n_vec; i += stride) {
-        const uint4 v = __ldcs(x + i);
+        const uint4 v = __ldg(x + i);
         amax_accum(v.x, mx, bad);
         amax_accum(v.y, mx, bad);
         amax_accum(v.z, mx, bad);
@@ -121,15 +121,20 @@ cudaError_t launch_amax(const void* x, int64_t n, float* alpha_out, WsControl* c
 // ==========================================================================
 //
 // One CTA tile = 128 rows x 256 columns = 4 scale atoms (2048 contiguous
-// bytes of the scale layout).  Warp w owns rows 32w..32w+31 of the tile and
-// walks them one row per step: lane l loads columns 8l..8l+7 (16 bytes), so
-// a warp step reads 512 contiguous bytes of one row and writes 128 contiguous
-// bytes of codes.  Lanes l and l^1 hold one 16-element block; one shuffle
-// gives the block amax.  Scales are staged in shared memory and written out
+// bytes of the scale layout); 8 warps, warp w owns rows 16w..16w+15.  Each
+// thread owns one 16-element block per step: a half-warp covers one row's
+// 256 columns (two 16-byte loads per thread, 512 contiguous bytes per
+// half-warp), so the block amax needs no shuffles and the per-block work
+// (one E4M3 rounding, two divisions) is paid once per 16 elements.  Codes
+// come from the conversion instruction (two per cvt) and leave as one
+// 8-byte store per thread; scales are staged in shared memory and written
 // as 16-byte stores.
+//
+// Tiles are visited in reverse order: when the amax pass has just streamed
+// the tensor front to back, its tail is still in L2 and is consumed first.
 
-constexpr int kQuantThreads = 128;
-constexpr int kQuantRowUnroll = 8;
+constexpr int kQuantThreads = 256;
+constexpr int kQuantStepUnroll = 4;   // steps (2 rows per warp each) with loads in flight
 
 __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const uint16_t* __restrict__ x, int64_t rows,
                                                                  int64_t K, const float* __restrict__ alpha_ptr,
@@ -139,64 +144,68 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const uint16_t*
 {
     __shared__ __align__(16) uint8_t sf_stage[2048];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int half = lane >> 4;   // which of the two rows of a step
+    const int blk = lane & 15;    // 16-element block within the 256-column chunk
     const float alpha = *alpha_ptr;
     const float alpha_qmax = __fmul_rn(alpha, 6.0f);
     const int64_t chunks = (K + 255) / 256;              // 256-column chunks per row block
     const int64_t tiles = ((rows + 127) / 128) * chunks;
 
-    for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+    for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
+        const int64_t tile = tiles - 1 - t;
         const int64_t rb = tile / chunks, kc = tile % chunks;
-        const int64_t col = kc * 256 + 8 * lane;
+        const int64_t col = kc * 256 + 16 * blk;
         const bool col_ok = col < K;
-        for (int i0 = 0; i0 < 32; i0 += kQuantRowUnroll) {
-            uint4 v[kQuantRowUnroll];
+#pragma unroll 1
+        for (int s0 = 0; s0 < 8; s0 += kQuantStepUnroll) {
+            uint4 v[kQuantStepUnroll][2];
 #pragma unroll
-            for (int u = 0; u < kQuantRowUnroll; ++u) {
-                const int64_t r = rb * 128 + 32 * warp + i0 + u;
-                v[u] = make_uint4(0u, 0u, 0u, 0u);
+            for (int u = 0; u < kQuantStepUnroll; ++u) {
+                const int64_t r = rb * 128 + 16 * warp + 2 * (s0 + u) + half;
+                v[u][0] = v[u][1] = make_uint4(0u, 0u, 0u, 0u);
                 if (r < rows && col_ok) {
                     int64_t src = r;
                     if (interleave_half > 0) {
-                        const int64_t c = r >> 5, t = r & 31;
-                        src = (t < 16) ? (16 * c + t) : (interleave_half + 16 * c + (t - 16));
+                        const int64_t c = r >> 5, tt = r & 31;
+                        src = (tt < 16) ? (16 * c + tt) : (interleave_half + 16 * c + (tt - 16));
                     }
-                    v[u] = __ldcs(reinterpret_cast<const uint4*>(x + src * K + col));
+                    const uint4* p = reinterpret_cast<const uint4*>(x + src * K + col);
+                    v[u][0] = __ldcs(p);
+                    v[u][1] = __ldcs(p + 1);
                 }
             }
 #pragma unroll
-            for (int u = 0; u < kQuantRowUnroll; ++u) {
-                const int i = i0 + u;
-                const int64_t r = rb * 128 + 32 * warp + i;
-                const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-                float f[8];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    f[2 * j] = bf16_lo(w[j]);
-                    f[2 * j + 1] = bf16_hi(w[j]);
-                }
-                float amax = 0.0f;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(f[j]));
-                amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+            for (int u = 0; u < kQuantStepUnroll; ++u) {
+                const int rl = 16 * warp + 2 * (s0 + u) + half;   // row within the 128-row block
+                const int64_t r = rb * 128 + rl;
+                const uint32_t w[8] = {v[u][0].x, v[u][0].y, v[u][0].z, v[u][0].w,
+                                       v[u][1].x, v[u][1].y, v[u][1].z, v[u][1].w};
                 // Eq. 3: sigma_b = Pi_E4M3(amax_b / (alpha * q_max))
+                const float amax = bf16x16_absmax(w);
                 const uint32_t sc = e4m3_round_sat(__fdiv_rn(amax, alpha_qmax));
-                // Eq. 2: q_i = Pi_FP4(x_i / (alpha * sigma_b)), as |x| * fl(1/fl(alpha*sigma))
+                // Eq. 2: q_i = Pi_FP4(x_i / (alpha * sigma_b)), as x * fl(1/fl(alpha*sigma))
                 const float d = __fmul_rn(alpha, e4m3_to_float(sc));
                 const float enc = (d == 0.0f) ? 0.0f : __fdiv_rn(1.0f, d);
-                uint32_t packed = 0;
+                float f0[8], f1[8];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) packed |= e2m1_code(f[j], enc) << (4 * j);
-                const bool ok = (r < rows) && col_ok;
-                if (ok) *reinterpret_cast<uint32_t*>(codes + r * (K / 2) + col / 2) = packed;
-                if ((lane & 1) == 0) {
-                    const int kb = lane >> 1;  // 16-element block within the 256-column chunk
-                    sf_stage[(kb >> 2) * 512 + i * 16 + warp * 4 + (kb & 3)] = ok ? (uint8_t)sc : (uint8_t)0;
+                for (int j = 0; j < 4; ++j) {
+                    f0[2 * j] = bf16_lo(w[j]);
+                    f0[2 * j + 1] = bf16_hi(w[j]);
+                    f1[2 * j] = bf16_lo(w[4 + j]);
+                    f1[2 * j + 1] = bf16_hi(w[4 + j]);
                 }
+                const uint32_t c0 = e2m1x8_encode(f0, enc);
+                const uint32_t c1 = e2m1x8_encode(f1, enc);
+                const bool ok = (r < rows) && col_ok;
+                if (ok) *reinterpret_cast<uint2*>(codes + r * (K / 2) + col / 2) = make_uint2(c0, c1);
+                sf_stage[(blk >> 2) * 512 + (rl & 31) * 16 + (rl >> 5) * 4 + (blk & 3)] = ok ? (uint8_t)sc : 0;
             }
         }
         __syncthreads();
-        uint4* dst = reinterpret_cast<uint4*>(scales + (rb * chunks + kc) * 2048);
-        dst[threadIdx.x] = reinterpret_cast<const uint4*>(sf_stage)[threadIdx.x];
+        if (threadIdx.x < 128) {
+            uint4* dst = reinterpret_cast<uint4*>(scales + (rb * chunks + kc) * 2048);
+            dst[threadIdx.x] = reinterpret_cast<const uint4*>(sf_stage)[threadIdx.x];
+        }
         __syncthreads();
     }
 }
@@ -205,11 +214,42 @@ cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float*
                             uint8_t* scales, int64_t interleave_half, const DeviceInfo& di, cudaStream_t s)
 {
     const int64_t tiles = ((rows + 127) / 128) * ((K + 255) / 256);
-    int64_t blocks = (int64_t)di.num_sms * 12;
+    int64_t blocks = (int64_t)di.num_sms * 4;
     if (blocks > tiles) blocks = tiles;
     if (blocks < 1) blocks = 1;
     quantize_kernel<<<(unsigned)blocks, kQuantThreads, 0, s>>>(static_cast<const uint16_t*>(x), rows, K, alpha,
                                                                codes, scales, interleave_half);
+    return cudaGetLastError();
+}
+
+// ==========================================================================
+// Self-test of the E2M1 conversion instruction against the definition
+// ==========================================================================
+//
+// For every FP32 bit pattern p in [0, 0x41000000] (0 .. 8.0) and its
+// negative, compare the conversion instruction with the comparison-chain
+// rounding of the definition (nearest E2M1 magnitude, ties to even, clip at
+// 6, sign kept).  Counts mismatches into counts[0] (positive) / counts[1].
+
+__global__ void selftest_e2m1_kernel(unsigned long long* counts)
+{
+    const uint32_t total = 0x41000000u + 1u;
+    unsigned long long bad_pos = 0, bad_neg = 0;
+    for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
+        const float m = __uint_as_float(i);
+        const float n = -m;
+        const uint32_t hw_p = e2m1x8_cvt(m, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f) & 15u;
+        const uint32_t hw_n = e2m1x8_cvt(n, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f) & 15u;
+        bad_pos += (hw_p != e2m1_code(m, 1.0f));
+        bad_neg += (hw_n != e2m1_code(n, 1.0f));
+    }
+    if (bad_pos) atomicAdd(&counts[0], bad_pos);
+    if (bad_neg) atomicAdd(&counts[1], bad_neg);
+}
+
+cudaError_t launch_selftest_e2m1(unsigned long long* counts, const DeviceInfo& di, cudaStream_t s)
+{
+    selftest_e2m1_kernel<<<di.num_sms * 8, 256, 0, s>>>(counts);
     return cudaGetLastError();
 }
 

@@ -32,7 +32,7 @@ STATUS_NAMES = {0: "MQ_OK", 1: "MQ_ERR_INVALID_ARG", 2: "MQ_ERR_SHAPE", 3: "MQ_E
 # Every symbol the header declares (checked by the ABI tests).
 EXPORTS = ("mq_status_string", "mq_version", "mq_nvfp4_sizes", "mq_workspace_bytes", "mq_quantize_weight",
            "mq_quantize_activation", "mq_prefill_linear", "mq_decode_linear", "mq_unswizzle_scales",
-           "mq_async_status", "mq_prefill_linear_noalloc")
+           "mq_async_status", "mq_prefill_linear_noalloc", "mq_selftest_e2m1")
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
@@ -82,6 +82,8 @@ def load(path: str = LIB_PATH):
             lib.mq_unswizzle_scales.restype = i32
             lib.mq_async_status.argtypes = [vp, vp]
             lib.mq_async_status.restype = i32
+            lib.mq_selftest_e2m1.argtypes = [vp, vp]
+            lib.mq_selftest_e2m1.restype = i32
             lib.mq_prefill_linear_noalloc.argtypes = [vp, i64, nvp, vp, vp, vp]
             lib.mq_prefill_linear_noalloc.restype = i32
             _lib = lib
@@ -239,6 +241,15 @@ def unswizzle_scales(t: NVFP4Tensor, out=None, stream=None):
     cs = t.c()
     _check(load().mq_unswizzle_scales(ctypes.byref(cs), _ptr(out), _stream(stream)), "mq_unswizzle_scales")
     return out
+
+
+def selftest_e2m1(stream=None):
+    """mq_selftest_e2m1: (mismatches on positive inputs, on negative inputs); both should be 0."""
+    torch = _torch()
+    counts = torch.zeros(2, dtype=torch.int64, device=torch.device("cuda", torch.cuda.current_device()))
+    _check(load().mq_selftest_e2m1(_ptr(counts), _stream(stream)), "mq_selftest_e2m1")
+    c = counts.cpu().tolist()
+    return int(c[0]), int(c[1])
 
 
 def async_status(ws, stream=None) -> int:

@@ -132,7 +132,7 @@ def test_fused_mlp_M32768():
     x = wl.heavy_tailed_bf16(32768, 4096, 3000)
     wgu, wdn = wl.mlp_weights(3000)
     rows = sample_rows(32768, 32, seed=3)
-    _mlp(x, wgu, wdn, rows, mq.workspace())
+    _mlp(x, wgu, wdn, rows, mq.workspace(x.shape[0], x.shape[1]))
 
 
 def test_ragged_multiturn_131072_tokens():
@@ -144,7 +144,7 @@ def test_ragged_multiturn_131072_tokens():
     for i in range(len(wl.RAGGED_LENGTHS)):      # every sequence, its first and last token
         a, b = int(off[i]), int(off[i + 1])
         rows |= {a, b - 1, *rng.choice(np.arange(a, b), size=3, replace=False).tolist()}
-    _mlp(x, wgu, wdn, np.array(sorted(rows), dtype=np.int64), mq.workspace())
+    _mlp(x, wgu, wdn, np.array(sorted(rows), dtype=np.int64), mq.workspace(x.shape[0], x.shape[1]))
 
 
 def test_phase_aware_pair_shared_master_weight():

@@ -157,3 +157,8 @@ def test_repeated_amax_on_one_workspace():
         torch.cuda.synchronize()
         _check_quant(x, t)
     assert mq.async_status(ws) == 0
+
+
+def test_e2m1_conversion_instruction_matches_definition():
+    """Every FP32 value in [-8, 8]: the hardware E2M1 rounding equals the comparison-chain definition."""
+    assert mq.selftest_e2m1() == (0, 0)
