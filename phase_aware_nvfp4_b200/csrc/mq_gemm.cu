@@ -20,9 +20,9 @@
 //               (one row per thread), release it to the MMA warp, then apply
 //               the tensor scales and store BF16 (or SiLU-mul -> NVFP4).
 // Stage = 256 K-elements (128 bytes per row, one swizzle row); 4 stages in
-// flight.  TMEM: accumulator in columns [0, 256), scale factors in two
-// alternating 48-column buffers from column 256 (per stage: 4 x 4 columns
-// for A, 4 x 8 columns for B, one 32-bit column per 32 rows per MMA).
+// flight.  TMEM: accumulator in columns [0, 256), scale factors in the 48
+// columns from 256 (per stage: 4 x 4 columns for A, 4 x 8 columns for B, one
+// 32-bit column per 32 rows per MMA).
 #include "mq_device.cuh"
 
 namespace mq {
@@ -45,8 +45,12 @@ constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_STAGE;
 constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;  // + barriers + alignment slack
 constexpr int NUM_THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t TMEM_SF = 256;        // two scale-factor buffers of 48 columns
-constexpr uint32_t TMEM_SF_BUF = 48;     // SFA 16 columns + SFB 32 columns per stage
+// One scale-factor region (SFA 16 columns + SFB 32 columns per stage), rewritten
+// every stage: copies and MMAs from one thread execute in issue order, so the
+// copies of stage s+1 land after the MMAs of stage s have read stage s's
+// scales.  (Alternating two regions measured slower: with a commit per stage
+// the pipe then serialises the copies behind the previous stage's MMAs.)
+constexpr uint32_t TMEM_SF = 256;
 constexpr uint32_t IDESC = idesc_nvfp4(BM, BN);
 
 struct Params {
@@ -102,6 +106,103 @@ __device__ __forceinline__ void silu_mul_quant_chunk(const uint32_t (&acc)[32], 
     codes[0] = e2m1x8_encode(h0, enc);
     codes[1] = e2m1x8_encode(h1, enc);
     scale = sc;
+}
+
+struct EpiScales {
+    float alpha_ab, alpha_h, alpha_h_qmax;
+};
+
+template <int EPI>
+__device__ __forceinline__ EpiScales epi_scales(const Params& p)
+{
+    EpiScales e;
+    e.alpha_ab = __fmul_rn(*p.alpha_a, *p.alpha_b);
+    e.alpha_h = 1.0f;
+    e.alpha_h_qmax = 6.0f;
+    if (EPI == 1) {
+        e.alpha_h = *p.h_alpha;
+        e.alpha_h_qmax = __fmul_rn(e.alpha_h, 6.0f);
+    }
+    return e;
+}
+
+// Epilogue of one 256-column accumulator row block: this thread owns output
+// row `row` and TMEM lane t_row.  Drains the 256 FP32 accumulators into
+// registers, calls release() (the accumulator may then be overwritten by the
+// next tile's MMAs), and only then stores BF16 Y, or (EPI 1) SiLU-mul ->
+// NVFP4 h codes + scales (+ optional BF16 h).
+template <int EPI, class Release>
+__device__ __forceinline__ void epilogue_tile(const Params& p, const EpiScales& es, uint32_t t_row, int64_t row,
+                                              int n_blk, Release release)
+{
+    const int lane_ok = row < p.M;
+    if (EPI == 0) {
+        uint32_t out[128];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(t_row + 32 * c, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                out[16 * c + j] = pack_bf16x2(__fmul_rn(__uint_as_float(r[2 * j]), es.alpha_ab),
+                                              __fmul_rn(__uint_as_float(r[2 * j + 1]), es.alpha_ab));
+        }
+        tc_fence_before();
+        release();
+        if (lane_ok) {
+            uint16_t* yrow = static_cast<uint16_t*>(p.y) + row * (int64_t)p.N + (int64_t)n_blk * BN;
+            const int ncols = min(BN, p.N - n_blk * BN);
+#pragma unroll
+            for (int q = 0; q < 32; ++q)
+                if (8 * q < ncols)
+                    reinterpret_cast<uint4*>(yrow)[q] = make_uint4(out[4 * q], out[4 * q + 1], out[4 * q + 2], out[4 * q + 3]);
+        }
+    } else {
+        uint32_t codes[16];
+        uint32_t scl[8];
+        uint32_t hb[64];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(t_row + 32 * c, r);
+            tmem_wait_ld();
+            uint32_t cc[2], hbits[8];
+            silu_mul_quant_chunk(r, es.alpha_ab, es.alpha_h, es.alpha_h_qmax, cc, scl[c], hbits);
+            codes[2 * c] = cc[0];
+            codes[2 * c + 1] = cc[1];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) hb[8 * c + j] = hbits[j];
+        }
+        tc_fence_before();
+        release();
+        const int hN = p.N / 2;
+        const int hcol0 = n_blk * (BN / 2);  // first h column of this tile
+        if (lane_ok && hcol0 < hN) {
+            const int nch = min(8, (hN - hcol0) / 16);
+            uint8_t* crow = p.h_codes + row * (int64_t)(hN / 2) + hcol0 / 2;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                if (c < nch) *reinterpret_cast<uint2*>(crow + 8 * c) = make_uint2(codes[2 * c], codes[2 * c + 1]);
+#pragma unroll
+            for (int g = 0; g < 2; ++g)
+                if (4 * g < nch) {
+                    const int kb = hcol0 / 16 + 4 * g;
+                    const uint32_t v = scl[4 * g] | (scl[4 * g + 1] << 8) | (scl[4 * g + 2] << 16) | (scl[4 * g + 3] << 24);
+                    *reinterpret_cast<uint32_t*>(p.h_scales + sf_offset(row, kb, p.h_atoms)) = v;
+                }
+            if (p.h_debug != nullptr) {
+                uint16_t* hrow = p.h_debug + row * (int64_t)hN + hcol0;
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    if (c < nch) {
+                        reinterpret_cast<uint4*>(hrow)[2 * c] = make_uint4(hb[8 * c], hb[8 * c + 1], hb[8 * c + 2], hb[8 * c + 3]);
+                        reinterpret_cast<uint4*>(hrow)[2 * c + 1] =
+                            make_uint4(hb[8 * c + 4], hb[8 * c + 5], hb[8 * c + 6], hb[8 * c + 7]);
+                    }
+            }
+        }
+    }
 }
 
 template <int EPI>
@@ -193,7 +294,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
             const uint32_t d_tmem = tmem_base;
-            uint32_t sf_buf = 0;
             for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
                 if (*abort_flag || !mbar_wait(acc_empty, acc_phase ^ 1u)) {
                     ok = false;
@@ -210,10 +310,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     const uint32_t b_base = smem_u32(smem + OFF_B + stage * B_STAGE);
                     const uint32_t sfa_base = smem_u32(smem + OFF_SFA + stage * SFA_STAGE);
                     const uint32_t sfb_base = smem_u32(smem + OFF_SFB + stage * SFB_STAGE);
-                    // scale factors alternate between two TMEM buffers from stage to stage
-                    const uint32_t sfa_tmem = tmem_base + TMEM_SF + sf_buf * TMEM_SF_BUF;
+                    const uint32_t sfa_tmem = tmem_base + TMEM_SF;
                     const uint32_t sfb_tmem = sfa_tmem + 16;
-                    sf_buf ^= 1u;
 #pragma unroll
                     for (int kb = 0; kb < 4; ++kb) {
                         tmem_cp_32x128b_x4(sfa_tmem + 4 * kb, sdesc_sf_block(sfa_base + kb * 512));
@@ -243,12 +341,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     } else {
         // ------------------------------------------------------------ epilogue
         const int lg = warp & 3;  // TMEM lane group this warp may access
-        const float alpha_ab = __fmul_rn(*p.alpha_a, *p.alpha_b);
-        float alpha_h = 1.0f, alpha_h_qmax = 6.0f;
-        if (EPI == 1) {
-            alpha_h = *p.h_alpha;
-            alpha_h_qmax = __fmul_rn(alpha_h, 6.0f);
-        }
+        EpiScales es = epi_scales<EPI>(p);
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
             const int m_blk = tile % p.num_m_blk;
@@ -262,77 +355,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tc_fence_after();
             const uint32_t t_row = tmem_base + ((uint32_t)(32 * lg) << 16);
             const int64_t row = (int64_t)m_blk * BM + 32 * lg + lane;
-            if (EPI == 0) {
-                uint32_t out[128];
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    uint32_t r[32];
-                    tmem_ld_32x32b_x32(t_row + 32 * c, r);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        out[16 * c + j] = pack_bf16x2(__fmul_rn(__uint_as_float(r[2 * j]), alpha_ab),
-                                                      __fmul_rn(__uint_as_float(r[2 * j + 1]), alpha_ab));
-                }
-                tc_fence_before();
-                mbar_arrive(acc_empty);
-                if (row < p.M) {
-                    uint16_t* yrow = static_cast<uint16_t*>(p.y) + row * (int64_t)p.N + (int64_t)n_blk * BN;
-                    const int ncols = min(BN, p.N - n_blk * BN);
-#pragma unroll
-                    for (int q = 0; q < 32; ++q)
-                        if (8 * q < ncols)
-                            reinterpret_cast<uint4*>(yrow)[q] =
-                                make_uint4(out[4 * q], out[4 * q + 1], out[4 * q + 2], out[4 * q + 3]);
-                }
-            } else {
-                uint32_t codes[16];
-                uint32_t scl[8];
-                uint32_t hb[64];
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    uint32_t r[32];
-                    tmem_ld_32x32b_x32(t_row + 32 * c, r);
-                    tmem_wait_ld();
-                    uint32_t cc[2], hbits[8];
-                    silu_mul_quant_chunk(r, alpha_ab, alpha_h, alpha_h_qmax, cc, scl[c], hbits);
-                    codes[2 * c] = cc[0];
-                    codes[2 * c + 1] = cc[1];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) hb[8 * c + j] = hbits[j];
-                }
-                tc_fence_before();
-                mbar_arrive(acc_empty);
-                const int hN = p.N / 2;
-                const int hcol0 = n_blk * (BN / 2);  // first h column of this tile
-                if (row < p.M && hcol0 < hN) {
-                    const int nch = min(8, (hN - hcol0) / 16);
-                    uint8_t* crow = p.h_codes + row * (int64_t)(hN / 2) + hcol0 / 2;
-#pragma unroll
-                    for (int c = 0; c < 8; ++c)
-                        if (c < nch)
-                            *reinterpret_cast<uint2*>(crow + 8 * c) = make_uint2(codes[2 * c], codes[2 * c + 1]);
-#pragma unroll
-                    for (int g = 0; g < 2; ++g)
-                        if (4 * g < nch) {
-                            const int kb = hcol0 / 16 + 4 * g;
-                            const uint32_t v =
-                                scl[4 * g] | (scl[4 * g + 1] << 8) | (scl[4 * g + 2] << 16) | (scl[4 * g + 3] << 24);
-                            *reinterpret_cast<uint32_t*>(p.h_scales + sf_offset(row, kb, p.h_atoms)) = v;
-                        }
-                    if (p.h_debug != nullptr) {
-                        uint16_t* hrow = p.h_debug + row * (int64_t)hN + hcol0;
-#pragma unroll
-                        for (int c = 0; c < 8; ++c)
-                            if (c < nch) {
-                                reinterpret_cast<uint4*>(hrow)[2 * c] =
-                                    make_uint4(hb[8 * c], hb[8 * c + 1], hb[8 * c + 2], hb[8 * c + 3]);
-                                reinterpret_cast<uint4*>(hrow)[2 * c + 1] =
-                                    make_uint4(hb[8 * c + 4], hb[8 * c + 5], hb[8 * c + 6], hb[8 * c + 7]);
-                            }
-                    }
-                }
-            }
+            epilogue_tile<EPI>(p, es, t_row, row, n_blk, [&] { mbar_arrive(acc_empty); });
         }
     }
 
@@ -344,19 +367,265 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
 }
 
+// ==========================================================================
+// CTA-pair kernel: 256 x 256 output tile per cluster of two CTAs
+// ==========================================================================
+//
+// Each CTA of the pair loads its own 128 rows of A, its own 128 of the 256
+// rows of B, the scale atoms of its A rows and all 256 rows of B scales; all
+// loads signal the full barrier of the leader CTA (rank 0).  The leader
+// alone issues the pair MMAs (tcgen05 cta_group::2, 256 x 256 x 64): each SM
+// multiplies its A rows by the whole B tile, half of which it receives from
+// the peer, and accumulates its 128 x 256 quarter... half of the tile in its
+// own TMEM.  Per CTA and stage this moves 38 KB instead of 54 KB for the
+// same FLOPs per SM, and five stages fit in shared memory.
+constexpr int P_STAGES = 5;
+constexpr int P_B_STAGE = 128 * BK_BYTES;  // this CTA's half of the B tile
+constexpr int P_STAGE_BYTES = A_STAGE + P_B_STAGE + SFA_STAGE + SFB_STAGE;
+constexpr int P_OFF_A = 0;
+constexpr int P_OFF_B = P_OFF_A + P_STAGES * A_STAGE;
+constexpr int P_OFF_SFA = P_OFF_B + P_STAGES * P_B_STAGE;
+constexpr int P_OFF_SFB = P_OFF_SFA + P_STAGES * SFA_STAGE;
+constexpr int P_STG_BYTES = 32 * 64 * 2;   // one warp's 32-row x 64-column BF16 output subtile
+constexpr int P_OFF_STG = P_OFF_SFB + P_STAGES * SFB_STAGE;   // 4 warps x 2 buffers
+constexpr int P_OFF_BAR = P_OFF_STG + 8 * P_STG_BYTES;
+constexpr int P_SMEM_BYTES = P_OFF_BAR + 256 + 1024;
+constexpr uint32_t P_IDESC = idesc_nvfp4(2 * BM, BN);
+static_assert(P_SMEM_BYTES <= 232448, "pair kernel shared memory");
+
+// BF16 epilogue through shared memory: drain the 128 x 256 FP32 accumulator
+// into registers (one row per thread), release TMEM, then each warp writes
+// its 32 rows in four 64-column subtiles into two alternating 4 KiB staging
+// buffers of its own (128-byte swizzle) and stores each with one TMA tile
+// store.  The global writes become full 128-byte lines instead of one 16-byte
+// piece of 32 different rows per warp store, which keeps the L1 / shared
+// memory port free for the tensor cores.  Only warp-level synchronisation is
+// used, so a warp that leaves early (wait timeout) cannot block the others.
+// (x0, y0): first output column and first row of this warp's 32 rows.
+template <class Release>
+__device__ __forceinline__ void epilogue_tile_bf16_tma(const EpiScales& es, uint32_t t_row, int lane, uint8_t* stg,
+                                                       const CUtensorMap* tmap_y, int32_t x0, int32_t y0,
+                                                       Release release)
+{
+    uint32_t out[128];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(t_row + 32 * c, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            out[16 * c + j] = pack_bf16x2(__fmul_rn(__uint_as_float(r[2 * j]), es.alpha_ab),
+                                          __fmul_rn(__uint_as_float(r[2 * j + 1]), es.alpha_ab));
+    }
+    tc_fence_before();
+    release();
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        uint8_t* buf = stg + (q & 1) * P_STG_BYTES;
+        // the store that last read this buffer (two subtiles ago) is done reading it
+        if (lane == 0) bulk_wait_group_read<1>();
+        __syncwarp();
+        uint8_t* rowp = buf + lane * 128;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int w = 32 * q + 4 * j;
+            *reinterpret_cast<uint4*>(rowp + ((j ^ (lane & 7)) << 4)) =
+                make_uint4(out[w], out[w + 1], out[w + 2], out[w + 3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_2d(tmap_y, buf, x0 + 64 * q, y0);
+            bulk_commit_group();
+        }
+    }
+}
+
+template <int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+    gemm_nvfp4_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                           const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
+                           const __grid_constant__ CUtensorMap tmap_y, const Params p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + P_OFF_BAR);
+    uint64_t* empty_bar = full_bar + P_STAGES;
+    uint64_t* acc_full = empty_bar + P_STAGES;
+    uint64_t* acc_empty = acc_full + 1;   // used in the leader: both CTAs' epilogues arrive
+    uint64_t* mma_done = acc_empty + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+    volatile uint32_t* abort_flag = tmem_slot + 1;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int pair = blockIdx.x >> 1;
+    const int npairs = gridDim.x >> 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < P_STAGES; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], 1);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, 256);
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        fence_mbarrier_init();
+        prefetch_tensormap(&tmap_a);
+        prefetch_tensormap(&tmap_b);
+        prefetch_tensormap(&tmap_sfa);
+        prefetch_tensormap(&tmap_sfb);
+        if (EPI == 0) prefetch_tensormap(&tmap_y);
+    }
+    if (warp == 1) tmem_alloc_pair(tmem_slot, TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    cluster_barrier();   // both CTAs' barriers initialised and TMEM allocated
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer (both CTAs)
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int tile = pair; tile < p.num_tiles && ok; tile += npairs) {
+                const int m_blk = tile % p.num_m_blk;
+                const int n_blk = tile / p.num_m_blk;
+                for (int ks = 0; ks < p.k_stages; ++ks) {
+                    if (*abort_flag || !mbar_wait(&empty_bar[stage], phase ^ 1u)) {
+                        ok = false;
+                        break;
+                    }
+                    if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2u * P_STAGE_BYTES);
+                    const uint32_t bar = map_to_cta(smem_u32(&full_bar[stage]), 0);
+                    tma_load_2d_pair(smem + P_OFF_A + stage * A_STAGE, &tmap_a, bar, ks * BK_BYTES,
+                                     m_blk * 2 * BM + (int)rank * BM);
+                    tma_load_2d_pair(smem + P_OFF_B + stage * P_B_STAGE, &tmap_b, bar, ks * BK_BYTES,
+                                     n_blk * BN + (int)rank * 128);
+                    tma_load_2d_pair(smem + P_OFF_SFA + stage * SFA_STAGE, &tmap_sfa, bar, 0,
+                                     (m_blk * 2 + (int)rank) * p.sfa_atoms + ks * 4);
+                    tma_load_2d_pair(smem + P_OFF_SFB + stage * SFB_STAGE, &tmap_sfb, bar, 0,
+                                     (n_blk * 2) * p.sfb_atoms + ks * 4);
+                    tma_load_2d_pair(smem + P_OFF_SFB + stage * SFB_STAGE + 2048, &tmap_sfb, bar, 0,
+                                     (n_blk * 2 + 1) * p.sfb_atoms + ks * 4);
+                    if (++stage == P_STAGES) stage = 0, phase ^= 1u;
+                }
+            }
+            if (!ok) {
+                post_error(p.ctrl, kErrTimeout);
+                *abort_flag = 1;
+            }
+            // Every load issued above has landed before this CTA may leave:
+            // the stage it last filled is released by the leader only after
+            // the MMAs that read it (and so after the copy completed).
+            if (ok) {
+                for (int s = 0; s < P_STAGES; ++s) {
+                    (void)mbar_wait(&empty_bar[stage], phase ^ 1u);
+                    if (++stage == P_STAGES) stage = 0, phase ^= 1u;
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer (leader only)
+        if (leader && lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            bool ok = true;
+            for (int tile = pair; tile < p.num_tiles && ok; tile += npairs) {
+                if (*abort_flag || !mbar_wait(acc_empty, acc_phase ^ 1u)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                for (int ks = 0; ks < p.k_stages; ++ks) {
+                    if (*abort_flag || !mbar_wait(&full_bar[stage], phase)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_base = smem_u32(smem + P_OFF_A + stage * A_STAGE);
+                    const uint32_t b_base = smem_u32(smem + P_OFF_B + stage * P_B_STAGE);
+                    const uint32_t sfa_base = smem_u32(smem + P_OFF_SFA + stage * SFA_STAGE);
+                    const uint32_t sfb_base = smem_u32(smem + P_OFF_SFB + stage * SFB_STAGE);
+                    const uint32_t sfa_tmem = tmem_base + TMEM_SF;
+                    const uint32_t sfb_tmem = sfa_tmem + 16;
+#pragma unroll
+                    for (int kb = 0; kb < 4; ++kb) {
+                        tmem_cp_32x128b_x4_pair(sfa_tmem + 4 * kb, sdesc_sf_block(sfa_base + kb * 512));
+                        tmem_cp_32x128b_x4_pair(sfb_tmem + 8 * kb, sdesc_sf_block(sfb_base + kb * 512));
+                        tmem_cp_32x128b_x4_pair(sfb_tmem + 8 * kb + 4, sdesc_sf_block(sfb_base + 2048 + kb * 512));
+                    }
+#pragma unroll
+                    for (int kb = 0; kb < 4; ++kb) {
+                        umma_nvfp4_pair(tmem_base, sdesc_kmajor_sw128(a_base + kb * 32),
+                                        sdesc_kmajor_sw128(b_base + kb * 32), P_IDESC, sfa_tmem + 4 * kb,
+                                        sfb_tmem + 8 * kb, (ks | kb) != 0 ? 1u : 0u);
+                    }
+                    tc_commit_pair_mc(&empty_bar[stage], 0x3);
+                    if (++stage == P_STAGES) stage = 0, phase ^= 1u;
+                }
+                if (!ok) break;
+                tc_commit_pair_mc(acc_full, 0x3);
+                acc_phase ^= 1u;
+            }
+            if (!ok) {
+                post_error(p.ctrl, kErrTimeout);
+                *abort_flag = 1;
+            }
+            tc_commit_pair(mma_done);
+            (void)mbar_wait(mma_done, 0);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue (both CTAs)
+        const int lg = warp & 3;
+        EpiScales es = epi_scales<EPI>(p);
+        const uint32_t leader_acc_empty = map_to_cta(smem_u32(acc_empty), 0);
+        uint32_t acc_phase = 0;
+        for (int tile = pair; tile < p.num_tiles; tile += npairs) {
+            const int m_blk = tile % p.num_m_blk;
+            const int n_blk = tile / p.num_m_blk;
+            if (*abort_flag || !mbar_wait(acc_full, acc_phase)) {
+                post_error(p.ctrl, kErrTimeout);
+                *abort_flag = 1;
+                break;
+            }
+            acc_phase ^= 1u;
+            tc_fence_after();
+            const uint32_t t_row = tmem_base + ((uint32_t)(32 * lg) << 16);
+            const int row_local = 32 * lg + lane;
+            const int64_t row0 = (int64_t)m_blk * 2 * BM + (int64_t)rank * BM;
+            if (EPI == 0) {
+                epilogue_tile_bf16_tma(es, t_row, lane, smem + P_OFF_STG + lg * 2 * P_STG_BYTES, &tmap_y,
+                                       n_blk * BN, (int32_t)(row0 + 32 * lg),
+                                       [&] { mbar_arrive_cluster(leader_acc_empty); });
+            } else {
+                epilogue_tile<EPI>(p, es, t_row, row0 + row_local, n_blk,
+                                   [&] { mbar_arrive_cluster(leader_acc_empty); });
+            }
+        }
+        // every output store has finished before the CTA may leave
+        if (EPI == 0 && lane == 0) bulk_wait_group<0>();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_barrier();   // no CTA leaves while its peer may still read its smem or TMEM
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_gemm_nvfp4(const GemmArgs& a, const DeviceInfo& di, cudaStream_t s)
 {
-    CUtensorMap ta, tb;
-    // A codes: [M rows, K/2 bytes], B codes: [N rows, K/2 bytes]; 128 x 128-byte
-    // and 256 x 128-byte boxes with the 128-byte swizzle the UMMA descriptors use.
-    if (!make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.a_codes, (uint64_t)(a.K / 2), (uint64_t)a.M,
-                      (uint64_t)(a.K / 2), BK_BYTES, BM, CU_TENSOR_MAP_SWIZZLE_128B))
-        return cudaErrorInvalidValue;
-    if (!make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.b_codes, (uint64_t)(a.K / 2), (uint64_t)a.N,
-                      (uint64_t)(a.K / 2), BK_BYTES, BN, CU_TENSOR_MAP_SWIZZLE_128B))
-        return cudaErrorInvalidValue;
     Params p{};
     p.sfa = a.a_scales;
     p.sfb = a.b_scales;
@@ -365,9 +634,7 @@ cudaError_t launch_gemm_nvfp4(const GemmArgs& a, const DeviceInfo& di, cudaStrea
     p.M = (int)a.M;
     p.N = (int)a.N;
     p.K = (int)a.K;
-    p.num_m_blk = (int)((a.M + BM - 1) / BM);
     const int num_n_blk = (int)((a.N + BN - 1) / BN);
-    p.num_tiles = p.num_m_blk * num_n_blk;
     p.k_stages = (int)((a.K + BK - 1) / BK);
     p.sfa_atoms = (int)sf_atoms_per_rowblk(a.K);
     p.sfb_atoms = (int)sf_atoms_per_rowblk(a.K);
@@ -380,6 +647,57 @@ cudaError_t launch_gemm_nvfp4(const GemmArgs& a, const DeviceInfo& di, cudaStrea
     p.h_atoms = (int)sf_atoms_per_rowblk(a.N / 2);
     p.ctrl = a.ctrl;
 
+    CUtensorMap ta, tb;
+    // A codes [M rows, K/2 bytes], B codes [N rows, K/2 bytes]: 128-byte-wide
+    // boxes with the 128-byte swizzle the UMMA descriptors assume.
+    if (!make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.a_codes, (uint64_t)(a.K / 2), (uint64_t)a.M,
+                      (uint64_t)(a.K / 2), BK_BYTES, BM, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+
+    if (a.M > BM) {
+        // CTA-pair kernel: 256 x 256 tiles
+        CUtensorMap tsfa, tsfb;
+        if (!make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.b_codes, (uint64_t)(a.K / 2), (uint64_t)a.N,
+                          (uint64_t)(a.K / 2), BK_BYTES, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
+        // scale buffers viewed as rows of one 512-byte atom (128 x u32); a box is 4 atoms
+        const uint64_t a_atoms = (uint64_t)sf_rowblks(a.M) * (uint64_t)p.sfa_atoms;
+        const uint64_t b_atoms = (uint64_t)sf_rowblks(a.N) * (uint64_t)p.sfb_atoms;
+        if (!make_tmap_2d(&tsfa, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.a_scales, 128, a_atoms, 512, 128, 4,
+                          CU_TENSOR_MAP_SWIZZLE_NONE))
+            return cudaErrorInvalidValue;
+        if (!make_tmap_2d(&tsfb, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.b_scales, 128, b_atoms, 512, 128, 4,
+                          CU_TENSOR_MAP_SWIZZLE_NONE))
+            return cudaErrorInvalidValue;
+        // output Y [M rows, N] BF16 for the TMA-store epilogue: 64-column x 32-row boxes (one warp's rows)
+        CUtensorMap ty = tb;
+        if (a.epilogue == 0 &&
+            !make_tmap_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.y, (uint64_t)a.N, (uint64_t)a.M,
+                          (uint64_t)a.N * 2, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
+        p.num_m_blk = (int)((a.M + 2 * BM - 1) / (2 * BM));
+        p.num_tiles = p.num_m_blk * num_n_blk;
+        const int pairs = std::min(p.num_tiles, di.num_sms / 2);
+        if (a.epilogue == 0) {
+            auto k = gemm_nvfp4_pair_kernel<0>;
+            cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM_BYTES);
+            if (e != cudaSuccess) return e;
+            k<<<2 * pairs, NUM_THREADS, P_SMEM_BYTES, s>>>(ta, tb, tsfa, tsfb, ty, p);
+        } else {
+            auto k = gemm_nvfp4_pair_kernel<1>;
+            cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM_BYTES);
+            if (e != cudaSuccess) return e;
+            k<<<2 * pairs, NUM_THREADS, P_SMEM_BYTES, s>>>(ta, tb, tsfa, tsfb, ty, p);
+        }
+        return cudaGetLastError();
+    }
+
+    // single-CTA kernel for short activations (M <= 128): 128 x 256 tiles
+    if (!make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.b_codes, (uint64_t)(a.K / 2), (uint64_t)a.N,
+                      (uint64_t)(a.K / 2), BK_BYTES, BN, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    p.num_m_blk = (int)((a.M + BM - 1) / BM);
+    p.num_tiles = p.num_m_blk * num_n_blk;
     const int grid = std::min(p.num_tiles, di.num_sms);
     if (a.epilogue == 0) {
         auto k = gemm_nvfp4_kernel<0>;
