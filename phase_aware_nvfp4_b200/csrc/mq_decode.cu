@@ -123,13 +123,18 @@ __global__ void __launch_bounds__(D_THREADS, 1)
             const uint32_t idesc = idesc_bf16(DBM, p.MT);
             int stage = 0;
             uint32_t phase = 0;
-            bool ok = true;
+            bool ok = true, next_ready = false;
+            const int NSTAGES_ = p.stages;
             for (int ks = ks_begin; ks < ks_end; ++ks) {
-                if (*abort_flag || !mbar_wait(&full_bar[stage], phase)) {
+                if (!next_ready && (*abort_flag || !mbar_wait(&full_bar[stage], phase))) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
+                {   // look at the next ring stage now; its result is used next iteration
+                    const int ns = (stage + 1 == NSTAGES_) ? 0 : stage + 1;
+                    next_ready = mbar_test_wait(&full_bar[ns], ns == 0 ? (phase ^ 1u) : phase);
+                }
                 const uint32_t w_addr = smem_u32(smem + stage * stage_bytes);
                 const uint32_t x_addr = w_addr + W_STAGE;
 #pragma unroll

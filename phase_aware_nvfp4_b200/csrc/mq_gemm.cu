@@ -292,7 +292,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0, acc_phase = 0;
-            bool ok = true;
+            bool ok = true, next_ready = false;
+            constexpr int NSTAGES_ = STAGES;
             const uint32_t d_tmem = tmem_base;
             for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
                 if (*abort_flag || !mbar_wait(acc_empty, acc_phase ^ 1u)) {
@@ -301,25 +302,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 }
                 tc_fence_after();
                 for (int ks = 0; ks < p.k_stages; ++ks) {
-                    if (*abort_flag || !mbar_wait(&full_bar[stage], phase)) {
+                    if (!next_ready && (*abort_flag || !mbar_wait(&full_bar[stage], phase))) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
+                    {   // look at the next ring stage now; its result is used next iteration
+                        const int ns = (stage + 1 == NSTAGES_) ? 0 : stage + 1;
+                        next_ready = mbar_test_wait(&full_bar[ns], ns == 0 ? (phase ^ 1u) : phase);
+                    }
                     const uint32_t a_base = smem_u32(smem + OFF_A + stage * A_STAGE);
                     const uint32_t b_base = smem_u32(smem + OFF_B + stage * B_STAGE);
                     const uint32_t sfa_base = smem_u32(smem + OFF_SFA + stage * SFA_STAGE);
                     const uint32_t sfb_base = smem_u32(smem + OFF_SFB + stage * SFB_STAGE);
                     const uint32_t sfa_tmem = tmem_base + TMEM_SF;
                     const uint32_t sfb_tmem = sfa_tmem + 16;
+                    // per k-block: its scale copies, then its MMA (interleaving lets the
+                    // copies overlap the previous MMA in the tensor pipe)
 #pragma unroll
                     for (int kb = 0; kb < 4; ++kb) {
                         tmem_cp_32x128b_x4(sfa_tmem + 4 * kb, sdesc_sf_block(sfa_base + kb * 512));
                         tmem_cp_32x128b_x4(sfb_tmem + 8 * kb, sdesc_sf_block(sfb_base + kb * 512));
                         tmem_cp_32x128b_x4(sfb_tmem + 8 * kb + 4, sdesc_sf_block(sfb_base + 2048 + kb * 512));
-                    }
-#pragma unroll
-                    for (int kb = 0; kb < 4; ++kb) {
                         umma_nvfp4(d_tmem, sdesc_kmajor_sw128(a_base + kb * 32), sdesc_kmajor_sw128(b_base + kb * 32),
                                    IDESC, sfa_tmem + 4 * kb, sfb_tmem + 8 * kb, (ks | kb) != 0 ? 1u : 0u);
                     }
@@ -536,7 +540,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         if (leader && lane == 0) {
             int stage = 0;
             uint32_t phase = 0, acc_phase = 0;
-            bool ok = true;
+            bool ok = true, next_ready = false;
+            constexpr int NSTAGES_ = P_STAGES;
             for (int tile = pair; tile < p.num_tiles && ok; tile += npairs) {
                 if (*abort_flag || !mbar_wait(acc_empty, acc_phase ^ 1u)) {
                     ok = false;
@@ -544,11 +549,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 }
                 tc_fence_after();
                 for (int ks = 0; ks < p.k_stages; ++ks) {
-                    if (*abort_flag || !mbar_wait(&full_bar[stage], phase)) {
+                    if (!next_ready && (*abort_flag || !mbar_wait(&full_bar[stage], phase))) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
+                    {   // look at the next ring stage now; its result is used next iteration
+                        const int ns = (stage + 1 == NSTAGES_) ? 0 : stage + 1;
+                        next_ready = mbar_test_wait(&full_bar[ns], ns == 0 ? (phase ^ 1u) : phase);
+                    }
                     const uint32_t a_base = smem_u32(smem + P_OFF_A + stage * A_STAGE);
                     const uint32_t b_base = smem_u32(smem + P_OFF_B + stage * P_B_STAGE);
                     const uint32_t sfa_base = smem_u32(smem + P_OFF_SFA + stage * SFA_STAGE);
@@ -560,9 +569,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                         tmem_cp_32x128b_x4_pair(sfa_tmem + 4 * kb, sdesc_sf_block(sfa_base + kb * 512));
                         tmem_cp_32x128b_x4_pair(sfb_tmem + 8 * kb, sdesc_sf_block(sfb_base + kb * 512));
                         tmem_cp_32x128b_x4_pair(sfb_tmem + 8 * kb + 4, sdesc_sf_block(sfb_base + 2048 + kb * 512));
-                    }
-#pragma unroll
-                    for (int kb = 0; kb < 4; ++kb) {
                         umma_nvfp4_pair(tmem_base, sdesc_kmajor_sw128(a_base + kb * 32),
                                         sdesc_kmajor_sw128(b_base + kb * 32), P_IDESC, sfa_tmem + 4 * kb,
                                         sfb_tmem + 8 * kb, (ks | kb) != 0 ? 1u : 0u);

@@ -12,8 +12,14 @@ namespace mq {
 // Tensor amax -> alpha = amax / (q_max * 448)
 // ==========================================================================
 
+#ifndef MQ_AMAX_UNROLL
+#define MQ_AMAX_UNROLL 4
+#endif
+#ifndef MQ_AMAX_BLOCKS_PER_SM
+#define MQ_AMAX_BLOCKS_PER_SM 4
+#endif
 constexpr int kAmaxThreads = 512;
-constexpr int kAmaxUnroll = 4;
+constexpr int kAmaxUnroll = MQ_AMAX_UNROLL;
 
 // Per-halfword |bf16| maximum over the finite values of a 32-bit word pair,
 // plus a flag word that is non-zero if a NaN/Inf was seen.
@@ -107,7 +113,7 @@ cudaError_t launch_amax(const void* x, int64_t n, float* alpha_out, WsControl* c
 {
     const int64_t n_vec = n / 8;
     int64_t blocks = (n_vec + kAmaxThreads * kAmaxUnroll - 1) / (kAmaxThreads * kAmaxUnroll);
-    const int64_t cap = (int64_t)di.num_sms * 4;
+    const int64_t cap = (int64_t)di.num_sms * MQ_AMAX_BLOCKS_PER_SM;
     if (blocks > cap) blocks = cap;
     if (blocks > kAmaxMaxBlocks) blocks = kAmaxMaxBlocks;
     if (blocks < 1) blocks = 1;
@@ -133,10 +139,16 @@ cudaError_t launch_amax(const void* x, int64_t n, float* alpha_out, WsControl* c
 // Tiles are visited in reverse order: when the amax pass has just streamed
 // the tensor front to back, its tail is still in L2 and is consumed first.
 
+#ifndef MQ_QUANT_UNROLL
+#define MQ_QUANT_UNROLL 4
+#endif
+#ifndef MQ_QUANT_MIN_BLOCKS
+#define MQ_QUANT_MIN_BLOCKS 4
+#endif
 constexpr int kQuantThreads = 256;
-constexpr int kQuantStepUnroll = 4;   // steps (2 rows per warp each) with loads in flight
+constexpr int kQuantStepUnroll = MQ_QUANT_UNROLL;   // steps (2 rows per warp each) with loads in flight
 
-__global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const uint16_t* __restrict__ x, int64_t rows,
+__global__ void __launch_bounds__(kQuantThreads, MQ_QUANT_MIN_BLOCKS) quantize_kernel(const uint16_t* __restrict__ x, int64_t rows,
                                                                  int64_t K, const float* __restrict__ alpha_ptr,
                                                                  uint8_t* __restrict__ codes,
                                                                  uint8_t* __restrict__ scales,
@@ -185,7 +197,7 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const uint16_t*
                 const uint32_t sc = e4m3_round_sat(__fdiv_rn(amax, alpha_qmax));
                 // Eq. 2: q_i = Pi_FP4(x_i / (alpha * sigma_b)), as x * fl(1/fl(alpha*sigma))
                 const float d = __fmul_rn(alpha, e4m3_to_float(sc));
-                const float enc = (d == 0.0f) ? 0.0f : __fdiv_rn(1.0f, d);
+                const float enc = (d == 0.0f) ? 0.0f : __frcp_rn(d);   // == fl(1/d)
                 float f0[8], f1[8];
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
@@ -214,7 +226,7 @@ cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float*
                             uint8_t* scales, int64_t interleave_half, const DeviceInfo& di, cudaStream_t s)
 {
     const int64_t tiles = ((rows + 127) / 128) * ((K + 255) / 256);
-    int64_t blocks = (int64_t)di.num_sms * 4;
+    int64_t blocks = (int64_t)di.num_sms * (MQ_QUANT_MIN_BLOCKS > 4 ? MQ_QUANT_MIN_BLOCKS : 4);
     if (blocks > tiles) blocks = tiles;
     if (blocks < 1) blocks = 1;
     quantize_kernel<<<(unsigned)blocks, kQuantThreads, 0, s>>>(static_cast<const uint16_t*>(x), rows, K, alpha,
