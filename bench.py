@@ -149,6 +149,24 @@ class ClockSampler:
                 "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
 
 
+# ---------------------------------------------------------------- multi-rank aggregation
+
+def max_over_ranks(value: float, device=None) -> float:
+    """Max of a per-rank scalar over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_rank_step: float, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput: the work of every rank divided by the slowest rank's step time."""
+    return flops_per_rank_step * world / (ms_per_step * 1e-3) / 1e12
+
+
 # ---------------------------------------------------------------- workload
 
 def workload(M: int):
@@ -355,13 +373,10 @@ def run_gpu(args):
                                       for i in range(K)])) for p in w.projections}
     quant_ms = {g: float(np.mean([ev[("q", g, i)][0].elapsed_time(ev[("q", g, i)][1]) for i in range(K)]))
                 for g in groups}
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dev)
 
     flops = w.flops
-    value = flops * world / (ms * 1e-3) / 1e12
+    value = whole_job_tflops(flops, world, ms)
     hbm_gbs, bf16_tf, bf16_tf_sus, peak_src = measured_peaks()
     fp4_peak = bf16_tf * FP4_PER_BF16
     gemm_flops = sum(p.flops for p in w.projections)
@@ -421,12 +436,8 @@ def run_gpu(args):
             e2e_step()
         b.record()
         torch.cuda.synchronize()
-        e2e_ms = a.elapsed_time(b) / ke
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        line["e2e"] = {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
+        e2e_ms = max_over_ranks(a.elapsed_time(b) / ke, dev)
+        line["e2e"] = {"value": whole_job_tflops(flops, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                        "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": ke}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
