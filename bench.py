@@ -389,15 +389,19 @@ def run_gpu(args):
         traffic = float(np.mean(list(cnt["dram_bytes_per_launch"].values())))
     roofline = {"bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
                 "frac": achieved / fp4_peak, "traffic": traffic,
-                "kernel": "gemm_nvfp4_kernel<BF16 epilogue>",
+                "kernel": "gemm_nvfp4_pair_kernel<BF16 epilogue>",
                 "peak_source": f"{peak_src} bf16_tflops (burst) x {FP4_PER_BF16:g} nominal FP4:BF16 ratio",
                 "per_projection_tflops": {p.name: p.flops / (gemm_ms[p.name] * 1e-3) / 1e12
                                           for p in w.projections}}
     # quantizer: algorithmic bytes = amax read (2 B/elem) + quantize read (2) + codes/scales write (0.5625)
     q_bytes = {g: ps[0].M * ps[0].K * (2 + 2 + 0.5625) for g, ps in groups.items()}
     q_gbs = sum(q_bytes.values()) / (sum(quant_ms.values()) * 1e-3) / 1e9
+    qcnt = counters_for("quantize_activation", sources_sha(QUANT_SOURCES))
+    q_traffic = None
+    if qcnt is not None and "dram_bytes_per_launch" in qcnt:
+        q_traffic = float(np.mean(list(qcnt["dram_bytes_per_launch"].values())))
     roofline_quant = {"bound": "hbm", "achieved": q_gbs, "peak": hbm_gbs, "unit": "GB/s", "frac": q_gbs / hbm_gbs,
-                      "traffic": None, "kernel": "amax_kernel + quantize_kernel",
+                      "traffic": q_traffic, "kernel": "amax_kernel + quantize_kernel",
                       "bytes_per_elem": 4.5625, "ms": quant_ms}
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,

@@ -121,6 +121,34 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity)
     }
 }
 
+// Warp-uniform forms, for loops that a whole converged warp runs so that its
+// values stay warp-uniform (the tensor-core instructions issued from such a
+// loop under elect_one() read their operands from uniform registers).
+// Every lane observes the phase itself; the vote makes the result (and so
+// the control flow after it) identical across the warp.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* abort_flag)
+{
+    const bool ok = !*abort_flag && mbar_wait(bar, parity);
+    return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ bool warp_test(uint64_t* bar, uint32_t parity)
+{
+    return __all_sync(0xffffffffu, mbar_test_wait(bar, parity));
+}
+
+// One lane of the converged warp is elected (elect.sync).
+__device__ __forceinline__ bool elect_one()
+{
+    uint32_t pred;
+    asm volatile(
+        "{\n\t.reg .pred P;\n\t"
+        "elect.sync _|P, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, P;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
+}
+
 // --------------------------------------------------------------------------
 // TMA / bulk copies (global -> shared, completion on an mbarrier)
 // --------------------------------------------------------------------------

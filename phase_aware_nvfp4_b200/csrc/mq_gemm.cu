@@ -536,55 +536,67 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             }
         }
     } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer (leader only)
-        if (leader && lane == 0) {
+        // ------------------------------------------------------------ MMA issuer (leader CTA)
+        // The whole warp runs the loop, so every address and descriptor is
+        // warp-uniform; one elected lane issues the copies, MMAs and commits.
+        // Descriptors are formed once and advanced by adding (offset >> 4) to
+        // their 14-bit start-address field (shared addresses stay below 256 KB,
+        // so the field never carries into its neighbours).
+        if (leader) {
+            const uint64_t a_desc0 = sdesc_kmajor_sw128(smem_u32(smem + P_OFF_A));
+            const uint64_t b_desc0 = sdesc_kmajor_sw128(smem_u32(smem + P_OFF_B));
+            const uint64_t sfa_desc0 = sdesc_sf_block(smem_u32(smem + P_OFF_SFA));
+            const uint64_t sfb_desc0 = sdesc_sf_block(smem_u32(smem + P_OFF_SFB));
+            const uint32_t sfa_tmem = tmem_base + TMEM_SF;
+            const uint32_t sfb_tmem = sfa_tmem + 16;
             int stage = 0;
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true, next_ready = false;
-            constexpr int NSTAGES_ = P_STAGES;
             for (int tile = pair; tile < p.num_tiles && ok; tile += npairs) {
-                if (*abort_flag || !mbar_wait(acc_empty, acc_phase ^ 1u)) {
+                if (!warp_wait(acc_empty, acc_phase ^ 1u, abort_flag)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 for (int ks = 0; ks < p.k_stages; ++ks) {
-                    if (!next_ready && (*abort_flag || !mbar_wait(&full_bar[stage], phase))) {
+                    if (!next_ready && !warp_wait(&full_bar[stage], phase, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     {   // look at the next ring stage now; its result is used next iteration
-                        const int ns = (stage + 1 == NSTAGES_) ? 0 : stage + 1;
-                        next_ready = mbar_test_wait(&full_bar[ns], ns == 0 ? (phase ^ 1u) : phase);
+                        const int ns = (stage + 1 == P_STAGES) ? 0 : stage + 1;
+                        next_ready = warp_test(&full_bar[ns], ns == 0 ? (phase ^ 1u) : phase);
                     }
-                    const uint32_t a_base = smem_u32(smem + P_OFF_A + stage * A_STAGE);
-                    const uint32_t b_base = smem_u32(smem + P_OFF_B + stage * P_B_STAGE);
-                    const uint32_t sfa_base = smem_u32(smem + P_OFF_SFA + stage * SFA_STAGE);
-                    const uint32_t sfb_base = smem_u32(smem + P_OFF_SFB + stage * SFB_STAGE);
-                    const uint32_t sfa_tmem = tmem_base + TMEM_SF;
-                    const uint32_t sfb_tmem = sfa_tmem + 16;
+                    const uint64_t a_d = a_desc0 + (uint64_t)((stage * A_STAGE) >> 4);
+                    const uint64_t b_d = b_desc0 + (uint64_t)((stage * P_B_STAGE) >> 4);
+                    const uint64_t sfa_d = sfa_desc0 + (uint64_t)((stage * SFA_STAGE) >> 4);
+                    const uint64_t sfb_d = sfb_desc0 + (uint64_t)((stage * SFB_STAGE) >> 4);
+                    if (elect_one()) {
 #pragma unroll
-                    for (int kb = 0; kb < 4; ++kb) {
-                        tmem_cp_32x128b_x4_pair(sfa_tmem + 4 * kb, sdesc_sf_block(sfa_base + kb * 512));
-                        tmem_cp_32x128b_x4_pair(sfb_tmem + 8 * kb, sdesc_sf_block(sfb_base + kb * 512));
-                        tmem_cp_32x128b_x4_pair(sfb_tmem + 8 * kb + 4, sdesc_sf_block(sfb_base + 2048 + kb * 512));
-                        umma_nvfp4_pair(tmem_base, sdesc_kmajor_sw128(a_base + kb * 32),
-                                        sdesc_kmajor_sw128(b_base + kb * 32), P_IDESC, sfa_tmem + 4 * kb,
-                                        sfb_tmem + 8 * kb, (ks | kb) != 0 ? 1u : 0u);
+                        for (int kb = 0; kb < 4; ++kb) {
+                            tmem_cp_32x128b_x4_pair(sfa_tmem + 4 * kb, sfa_d + (uint64_t)((kb * 512) >> 4));
+                            tmem_cp_32x128b_x4_pair(sfb_tmem + 8 * kb, sfb_d + (uint64_t)((kb * 512) >> 4));
+                            tmem_cp_32x128b_x4_pair(sfb_tmem + 8 * kb + 4, sfb_d + (uint64_t)((2048 + kb * 512) >> 4));
+                            umma_nvfp4_pair(tmem_base, a_d + (uint64_t)((kb * 32) >> 4), b_d + (uint64_t)((kb * 32) >> 4),
+                                            P_IDESC, sfa_tmem + 4 * kb, sfb_tmem + 8 * kb, (ks | kb) != 0 ? 1u : 0u);
+                        }
+                        tc_commit_pair_mc(&empty_bar[stage], 0x3);
                     }
-                    tc_commit_pair_mc(&empty_bar[stage], 0x3);
+                    __syncwarp();
                     if (++stage == P_STAGES) stage = 0, phase ^= 1u;
                 }
                 if (!ok) break;
-                tc_commit_pair_mc(acc_full, 0x3);
+                if (elect_one()) tc_commit_pair_mc(acc_full, 0x3);
+                __syncwarp();
                 acc_phase ^= 1u;
             }
-            if (!ok) {
+            if (!ok && lane == 0) {
                 post_error(p.ctrl, kErrTimeout);
                 *abort_flag = 1;
             }
-            tc_commit_pair(mma_done);
+            if (elect_one()) tc_commit_pair(mma_done);
+            __syncwarp();
             (void)mbar_wait(mma_done, 0);
         }
     } else {
