@@ -391,46 +391,61 @@ constexpr int P_OFF_B = P_OFF_A + P_STAGES * A_STAGE;
 constexpr int P_OFF_SFA = P_OFF_B + P_STAGES * P_B_STAGE;
 constexpr int P_OFF_SFB = P_OFF_SFA + P_STAGES * SFA_STAGE;
 constexpr int P_STG_BYTES = 32 * 64 * 2;   // one warp's 32-row x 64-column BF16 output subtile
-constexpr int P_OFF_STG = P_OFF_SFB + P_STAGES * SFB_STAGE;   // 4 warps x 2 buffers
+constexpr int P_OFF_STG = P_OFF_SFB + P_STAGES * SFB_STAGE;   // 8 epilogue warps x 1 buffer
 constexpr int P_OFF_BAR = P_OFF_STG + 8 * P_STG_BYTES;
 constexpr int P_SMEM_BYTES = P_OFF_BAR + 256 + 1024;
 constexpr uint32_t P_IDESC = idesc_nvfp4(2 * BM, BN);
 static_assert(P_SMEM_BYTES <= 232448, "pair kernel shared memory");
+// Pair kernel warps: 0 TMA producer, 1 MMA issuer, 2-9 epilogue (warp w drains
+// TMEM lane group w % 4, accumulator columns [128 * ((w - 2) / 4), + 128)).
+constexpr int P_NUM_THREADS = 320;
+constexpr int P_EPI_WARPS = 8;
 
-// BF16 epilogue through shared memory: drain the 128 x 256 FP32 accumulator
-// into registers (one row per thread), release TMEM, then each warp writes
-// its 32 rows in four 64-column subtiles into two alternating 4 KiB staging
-// buffers of its own (128-byte swizzle) and stores each with one TMA tile
-// store.  The global writes become full 128-byte lines instead of one 16-byte
-// piece of 32 different rows per warp store, which keeps the L1 / shared
-// memory port free for the tensor cores.  Only warp-level synchronisation is
-// used, so a warp that leaves early (wait timeout) cannot block the others.
-// (x0, y0): first output column and first row of this warp's 32 rows.
-template <class Release>
-__device__ __forceinline__ void epilogue_tile_bf16_tma(const EpiScales& es, uint32_t t_row, int lane, uint8_t* stg,
-                                                       const CUtensorMap* tmap_y, int32_t x0, int32_t y0,
-                                                       Release release)
+// Pair-kernel epilogue: eight warps drain the 128 x 256 FP32 accumulator,
+// two per TMEM lane group, each taking 32 rows x one 128-column half, so the
+// accumulator is released after four TMEM loads per warp instead of eight.
+// The release is per warp: every lane has waited for its loads, the warp
+// synchronises and lane 0 arrives on the leader CTA's acc_empty barrier.
+template <class Barrier>
+__device__ __forceinline__ void release_acc_warp(int lane, Barrier arrive)
 {
-    uint32_t out[128];
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) arrive();
+}
+
+// BF16 half-tile through shared memory: after the release, the warp writes
+// its 32 rows x 128 columns as two 64-column subtiles into its 4 KiB staging
+// buffer (128-byte swizzle) and stores each with one TMA tile store; the
+// buffer is reused once the previous store has finished reading it.  Full
+// 128-byte lines reach global memory instead of 16-byte pieces of 32 rows,
+// which keeps the L1 / shared-memory port free for the tensor cores.  Only
+// warp-level synchronisation is used, so a warp that leaves early (wait
+// timeout) cannot block the others.  (x0, y0): first output column and first
+// row of this warp's 32 x 128 block.
+template <class Barrier>
+__device__ __forceinline__ void epilogue_half_bf16_tma(const EpiScales& es, uint32_t t_col, int lane, uint8_t* stg,
+                                                       const CUtensorMap* tmap_y, int32_t x0, int32_t y0,
+                                                       Barrier arrive)
+{
+    uint32_t out[64];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
+    for (int c = 0; c < 4; ++c) {
         uint32_t r[32];
-        tmem_ld_32x32b_x32(t_row + 32 * c, r);
+        tmem_ld_32x32b_x32(t_col + 32 * c, r);
         tmem_wait_ld();
 #pragma unroll
         for (int j = 0; j < 16; ++j)
             out[16 * c + j] = pack_bf16x2(__fmul_rn(__uint_as_float(r[2 * j]), es.alpha_ab),
                                           __fmul_rn(__uint_as_float(r[2 * j + 1]), es.alpha_ab));
     }
-    tc_fence_before();
-    release();
+    release_acc_warp(lane, arrive);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        uint8_t* buf = stg + (q & 1) * P_STG_BYTES;
-        // the store that last read this buffer (two subtiles ago) is done reading it
-        if (lane == 0) bulk_wait_group_read<1>();
+    for (int q = 0; q < 2; ++q) {
+        // the store that last read the buffer is done reading it
+        if (lane == 0) bulk_wait_group_read<0>();
         __syncwarp();
-        uint8_t* rowp = buf + lane * 128;
+        uint8_t* rowp = stg + lane * 128;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const int w = 32 * q + 4 * j;
@@ -440,14 +455,61 @@ __device__ __forceinline__ void epilogue_tile_bf16_tma(const EpiScales& es, uint
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-            tma_store_2d(tmap_y, buf, x0 + 64 * q, y0);
+            tma_store_2d(tmap_y, stg, x0 + 64 * q, y0);
             bulk_commit_group();
         }
     }
 }
 
+// Fused MLP half-tile (EPI 1): accumulator columns [128*half, 128*half + 128)
+// are four 32-column chunks (16 gate + 16 up each) = 64 h columns = one
+// 64-wide group of four NVFP4 blocks, whose four scale bytes form one 32-bit
+// word of the scale layout.
+template <class Barrier>
+__device__ __forceinline__ void epilogue_half_mlp(const Params& p, const EpiScales& es, uint32_t t_col, int half,
+                                                  int64_t row, int n_blk, int lane, Barrier arrive)
+{
+    uint32_t codes[8];
+    uint32_t scl[4];
+    uint32_t hb[32];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(t_col + 32 * c, r);
+        tmem_wait_ld();
+        uint32_t cc[2], hbits[8];
+        silu_mul_quant_chunk(r, es.alpha_ab, es.alpha_h, es.alpha_h_qmax, cc, scl[c], hbits);
+        codes[2 * c] = cc[0];
+        codes[2 * c + 1] = cc[1];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) hb[8 * c + j] = hbits[j];
+    }
+    release_acc_warp(lane, arrive);
+    const int hN = p.N / 2;
+    const int hcol0 = n_blk * (BN / 2) + 64 * half;   // first h column of this half
+    const int nch = min(4, (hN - hcol0) / 16);
+    if (row < p.M && nch > 0) {
+        uint8_t* crow = p.h_codes + row * (int64_t)(hN / 2) + hcol0 / 2;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+            if (c < nch) *reinterpret_cast<uint2*>(crow + 8 * c) = make_uint2(codes[2 * c], codes[2 * c + 1]);
+        const uint32_t v = scl[0] | (scl[1] << 8) | (scl[2] << 16) | (scl[3] << 24);
+        *reinterpret_cast<uint32_t*>(p.h_scales + sf_offset(row, hcol0 / 16, p.h_atoms)) = v;
+        if (p.h_debug != nullptr) {
+            uint16_t* hrow = p.h_debug + row * (int64_t)hN + hcol0;
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                if (c < nch) {
+                    reinterpret_cast<uint4*>(hrow)[2 * c] = make_uint4(hb[8 * c], hb[8 * c + 1], hb[8 * c + 2], hb[8 * c + 3]);
+                    reinterpret_cast<uint4*>(hrow)[2 * c + 1] =
+                        make_uint4(hb[8 * c + 4], hb[8 * c + 5], hb[8 * c + 6], hb[8 * c + 7]);
+                }
+        }
+    }
+}
+
 template <int EPI>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_NUM_THREADS, 1)
     gemm_nvfp4_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                            const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
                            const __grid_constant__ CUtensorMap tmap_y, const Params p)
@@ -475,7 +537,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             mbar_init(&empty_bar[s], 1);
         }
         mbar_init(acc_full, 1);
-        mbar_init(acc_empty, 256);
+        mbar_init(acc_empty, 2 * P_EPI_WARPS);   // one arrival per epilogue warp of both CTAs
         mbar_init(mma_done, 1);
         *abort_flag = 0;
         fence_mbarrier_init();
@@ -602,29 +664,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     } else {
         // ------------------------------------------------------------ epilogue (both CTAs)
         const int lg = warp & 3;
+        const int half = (warp - 2) >> 2;
         EpiScales es = epi_scales<EPI>(p);
         const uint32_t leader_acc_empty = map_to_cta(smem_u32(acc_empty), 0);
+        const uint32_t t_col = tmem_base + ((uint32_t)(32 * lg) << 16) + (uint32_t)(128 * half);
+        uint8_t* stg = smem + P_OFF_STG + (warp - 2) * P_STG_BYTES;
+        auto arrive = [&] { mbar_arrive_cluster(leader_acc_empty); };
         uint32_t acc_phase = 0;
         for (int tile = pair; tile < p.num_tiles; tile += npairs) {
             const int m_blk = tile % p.num_m_blk;
             const int n_blk = tile / p.num_m_blk;
-            if (*abort_flag || !mbar_wait(acc_full, acc_phase)) {
-                post_error(p.ctrl, kErrTimeout);
-                *abort_flag = 1;
+            if (!warp_wait(acc_full, acc_phase, abort_flag)) {
+                if (lane == 0) {
+                    post_error(p.ctrl, kErrTimeout);
+                    *abort_flag = 1;
+                }
                 break;
             }
             acc_phase ^= 1u;
             tc_fence_after();
-            const uint32_t t_row = tmem_base + ((uint32_t)(32 * lg) << 16);
-            const int row_local = 32 * lg + lane;
-            const int64_t row0 = (int64_t)m_blk * 2 * BM + (int64_t)rank * BM;
+            const int64_t row0 = (int64_t)m_blk * 2 * BM + (int64_t)rank * BM + 32 * lg;
             if (EPI == 0) {
-                epilogue_tile_bf16_tma(es, t_row, lane, smem + P_OFF_STG + lg * 2 * P_STG_BYTES, &tmap_y,
-                                       n_blk * BN, (int32_t)(row0 + 32 * lg),
-                                       [&] { mbar_arrive_cluster(leader_acc_empty); });
+                epilogue_half_bf16_tma(es, t_col, lane, stg, &tmap_y, n_blk * BN + 128 * half, (int32_t)row0, arrive);
             } else {
-                epilogue_tile<EPI>(p, es, t_row, row0 + row_local, n_blk,
-                                   [&] { mbar_arrive_cluster(leader_acc_empty); });
+                epilogue_half_mlp(p, es, t_col, half, row0 + lane, n_blk, lane, arrive);
             }
         }
         // every output store has finished before the CTA may leave
@@ -700,12 +763,12 @@ cudaError_t launch_gemm_nvfp4(const GemmArgs& a, const DeviceInfo& di, cudaStrea
             auto k = gemm_nvfp4_pair_kernel<0>;
             cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM_BYTES);
             if (e != cudaSuccess) return e;
-            k<<<2 * pairs, NUM_THREADS, P_SMEM_BYTES, s>>>(ta, tb, tsfa, tsfb, ty, p);
+            k<<<2 * pairs, P_NUM_THREADS, P_SMEM_BYTES, s>>>(ta, tb, tsfa, tsfb, ty, p);
         } else {
             auto k = gemm_nvfp4_pair_kernel<1>;
             cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM_BYTES);
             if (e != cudaSuccess) return e;
-            k<<<2 * pairs, NUM_THREADS, P_SMEM_BYTES, s>>>(ta, tb, tsfa, tsfb, ty, p);
+            k<<<2 * pairs, P_NUM_THREADS, P_SMEM_BYTES, s>>>(ta, tb, tsfa, tsfb, ty, p);
         }
         return cudaGetLastError();
     }
