@@ -556,34 +556,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_NUM_THREADS, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer (both CTAs)
-        if (lane == 0) {
+        // Whole warp, warp-uniform values; one elected lane issues the copies.
+        {
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
+            const uint32_t full0 = map_to_cta(smem_u32(&full_bar[0]), 0);
             for (int tile = pair; tile < p.num_tiles && ok; tile += npairs) {
                 const int m_blk = tile % p.num_m_blk;
                 const int n_blk = tile / p.num_m_blk;
+                const int a_row = m_blk * 2 * BM + (int)rank * BM;
+                const int b_row = n_blk * BN + (int)rank * 128;
+                const int sfa_row = (m_blk * 2 + (int)rank) * p.sfa_atoms;
+                const int sfb_row0 = (n_blk * 2) * p.sfb_atoms;
+                const int sfb_row1 = sfb_row0 + p.sfb_atoms;
                 for (int ks = 0; ks < p.k_stages; ++ks) {
-                    if (*abort_flag || !mbar_wait(&empty_bar[stage], phase ^ 1u)) {
+                    if (!warp_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) {
                         ok = false;
                         break;
                     }
-                    if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2u * P_STAGE_BYTES);
-                    const uint32_t bar = map_to_cta(smem_u32(&full_bar[stage]), 0);
-                    tma_load_2d_pair(smem + P_OFF_A + stage * A_STAGE, &tmap_a, bar, ks * BK_BYTES,
-                                     m_blk * 2 * BM + (int)rank * BM);
-                    tma_load_2d_pair(smem + P_OFF_B + stage * P_B_STAGE, &tmap_b, bar, ks * BK_BYTES,
-                                     n_blk * BN + (int)rank * 128);
-                    tma_load_2d_pair(smem + P_OFF_SFA + stage * SFA_STAGE, &tmap_sfa, bar, 0,
-                                     (m_blk * 2 + (int)rank) * p.sfa_atoms + ks * 4);
-                    tma_load_2d_pair(smem + P_OFF_SFB + stage * SFB_STAGE, &tmap_sfb, bar, 0,
-                                     (n_blk * 2) * p.sfb_atoms + ks * 4);
-                    tma_load_2d_pair(smem + P_OFF_SFB + stage * SFB_STAGE + 2048, &tmap_sfb, bar, 0,
-                                     (n_blk * 2 + 1) * p.sfb_atoms + ks * 4);
+                    if (elect_one()) {
+                        if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2u * P_STAGE_BYTES);
+                        const uint32_t bar = full0 + 8u * (uint32_t)stage;
+                        tma_load_2d_pair(smem + P_OFF_A + stage * A_STAGE, &tmap_a, bar, ks * BK_BYTES, a_row);
+                        tma_load_2d_pair(smem + P_OFF_B + stage * P_B_STAGE, &tmap_b, bar, ks * BK_BYTES, b_row);
+                        tma_load_2d_pair(smem + P_OFF_SFA + stage * SFA_STAGE, &tmap_sfa, bar, 0, sfa_row + ks * 4);
+                        tma_load_2d_pair(smem + P_OFF_SFB + stage * SFB_STAGE, &tmap_sfb, bar, 0, sfb_row0 + ks * 4);
+                        tma_load_2d_pair(smem + P_OFF_SFB + stage * SFB_STAGE + 2048, &tmap_sfb, bar, 0,
+                                         sfb_row1 + ks * 4);
+                    }
+                    __syncwarp();
                     if (++stage == P_STAGES) stage = 0, phase ^= 1u;
                 }
             }
-            if (!ok) {
+            if (!ok && lane == 0) {
                 post_error(p.ctrl, kErrTimeout);
                 *abort_flag = 1;
             }
