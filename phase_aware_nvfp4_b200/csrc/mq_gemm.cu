@@ -568,8 +568,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_NUM_THREADS, 1)
                 const int a_row = m_blk * 2 * BM + (int)rank * BM;
                 const int b_row = n_blk * BN + (int)rank * 128;
                 const int sfa_row = (m_blk * 2 + (int)rank) * p.sfa_atoms;
-                const int sfb_row0 = (n_blk * 2) * p.sfb_atoms;
-                const int sfb_row1 = sfb_row0 + p.sfb_atoms;
                 for (int ks = 0; ks < p.k_stages; ++ks) {
                     if (!warp_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) {
                         ok = false;
@@ -581,9 +579,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_NUM_THREADS, 1)
                         tma_load_2d_pair(smem + P_OFF_A + stage * A_STAGE, &tmap_a, bar, ks * BK_BYTES, a_row);
                         tma_load_2d_pair(smem + P_OFF_B + stage * P_B_STAGE, &tmap_b, bar, ks * BK_BYTES, b_row);
                         tma_load_2d_pair(smem + P_OFF_SFA + stage * SFA_STAGE, &tmap_sfa, bar, 0, sfa_row + ks * 4);
-                        tma_load_2d_pair(smem + P_OFF_SFB + stage * SFB_STAGE, &tmap_sfb, bar, 0, sfb_row0 + ks * 4);
-                        tma_load_2d_pair(smem + P_OFF_SFB + stage * SFB_STAGE + 2048, &tmap_sfb, bar, 0,
-                                         sfb_row1 + ks * 4);
+                        tma_load_3d_pair(smem + P_OFF_SFB + stage * SFB_STAGE, &tmap_sfb, bar, 0, ks * 4, 2 * n_blk);
                     }
                     __syncwarp();
                     if (++stage == P_STAGES) stage = 0, phase ^= 1u;
@@ -749,12 +745,13 @@ cudaError_t launch_gemm_nvfp4(const GemmArgs& a, const DeviceInfo& di, cudaStrea
             return cudaErrorInvalidValue;
         // scale buffers viewed as rows of one 512-byte atom (128 x u32); a box is 4 atoms
         const uint64_t a_atoms = (uint64_t)sf_rowblks(a.M) * (uint64_t)p.sfa_atoms;
-        const uint64_t b_atoms = (uint64_t)sf_rowblks(a.N) * (uint64_t)p.sfb_atoms;
         if (!make_tmap_2d(&tsfa, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.a_scales, 128, a_atoms, 512, 128, 4,
                           CU_TENSOR_MAP_SWIZZLE_NONE))
             return cudaErrorInvalidValue;
-        if (!make_tmap_2d(&tsfb, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.b_scales, 128, b_atoms, 512, 128, 4,
-                          CU_TENSOR_MAP_SWIZZLE_NONE))
+        // B scales as [row blocks][atoms][128 x u32]: one box = 4 atoms of the two
+        // 128-row blocks of a 256-row tile
+        if (!make_tmap_3d(&tsfb, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.b_scales, 128, (uint64_t)p.sfb_atoms,
+                          (uint64_t)p.sfb_rowblks, 512, (uint64_t)p.sfb_atoms * 512, 128, 4, 2))
             return cudaErrorInvalidValue;
         // output Y [M rows, N] BF16 for the TMA-store epilogue: 64-column x 32-row boxes (one warp's rows)
         CUtensorMap ty = tb;

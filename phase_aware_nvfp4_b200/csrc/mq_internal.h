@@ -98,5 +98,9 @@ cudaError_t launch_decode_bf16(const void* x, int64_t M, const void* w, int64_t 
 // cuTensorMapEncodeTiled obtained from the driver at run time.
 bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t outer,
                   uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz);
+// 3-D tiled map without swizzle: extents d0 (innermost) .. d2, byte strides of
+// dimensions 1 and 2, box b0 x b1 x b2.
+bool make_tmap_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                  uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t b0, uint32_t b1, uint32_t b2);
 
 }  // namespace mq
