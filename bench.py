@@ -61,6 +61,8 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-baseline-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the decode / fused-MLP side measurements reported under 'extras'")
     return ap.parse_args(argv)
 
 
@@ -281,6 +283,126 @@ def config_of(w):
 
 # ---------------------------------------------------------------- GPU arm
 
+def _to_dev(torch, a, dev):
+    return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+
+
+def _time_calls(torch, fn, reps, flush):
+    """Mean device time (ms) of fn() over reps calls, L2 flushed before each."""
+    evs = []
+    for _ in range(reps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        evs.append((a, b))
+    torch.cuda.synchronize()
+    return float(np.mean([a.elapsed_time(b) for a, b in evs]))
+
+
+def measure_extras(mq, torch, dev, flush, hbm_gbs, fp4_peak, reps=10):
+    """Side measurements of the other workloads (the main line is the projection step):
+
+    * phase-aware pair on one BF16 master weight [12288, 4096]: BF16 decode at
+      M = 1, 8, 32, 64 tokens (HBM roofline: 2NK + 2MK + 2MN bytes) and NVFP4
+      prefill (quantize + GEMM) at M = 16384, plus the NVFP4-vs-BF16 output
+      error of the two paths on the first 64 prefill tokens;
+    * fused MLP at M = 32768: activation quantization, gate/up GEMM with the
+      SiLU-mul + NVFP4 requantization epilogue, down GEMM.
+    """
+    from phase_aware_nvfp4_b200 import workloads as wl
+    out = {}
+    N, K = 12288, 4096
+    Wm = _to_dev(torch, wl.normal_bf16(N, K, 0.02, 4001), dev)
+    ws = mq.workspace(16384, K, device=dev)
+    dec = {}
+    for M in (1, 8, 32, 64):
+        x = _to_dev(torch, wl.heavy_tailed_bf16(M, K, 4000 + M), dev)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        for _ in range(3):
+            mq.decode_linear(x, Wm, Y=y, ws=ws)
+        ms = _time_calls(torch, lambda: mq.decode_linear(x, Wm, Y=y, ws=ws), reps, flush)
+        gbs = (2 * N * K + 2 * M * K + 2 * M * N) / (ms * 1e-3) / 1e9
+        dec[str(M)] = {"ms": ms, "GB/s": gbs, "frac": gbs / hbm_gbs}
+    Wq = mq.quantize_weight(Wm, ws=ws)
+    Mp = 16384
+    X = _to_dev(torch, wl.heavy_tailed_bf16(Mp, K, 4000), dev)
+    Xq = mq.nvfp4_empty(Mp, K, dev)
+    Y = torch.empty((Mp, N), dtype=torch.bfloat16, device=dev)
+
+    def prefill():
+        mq.quantize_activation(X, out=Xq, ws=ws)
+        mq.prefill_linear(W=Wq, Xq=Xq, Y=Y, ws=ws)
+    for _ in range(3):
+        prefill()
+    ms = _time_calls(torch, prefill, reps, flush)
+    yb = mq.decode_linear(X[:64], Wm, ws=ws)
+    torch.cuda.synchronize()
+    yq, yr = Y[:64].double(), yb.double()
+    err = float(torch.linalg.norm(yq - yr) / torch.linalg.norm(yr))
+    out["phase_aware_pair"] = {
+        "weight": [N, K], "decode_bf16": dec,
+        "roofline_decode": {"bound": "hbm", "kernel": "decode_bf16_kernel", "unit": "GB/s", "peak": hbm_gbs,
+                            "achieved": dec["64"]["GB/s"], "frac": dec["64"]["frac"], "M": 64},
+        "prefill_nvfp4": {"M": Mp, "ms": ms, "TFLOP/s": 2 * Mp * N * K / (ms * 1e-3) / 1e12},
+        "nvfp4_vs_bf16_rel_frobenius": err}
+    del X, Xq, Y
+    # fused MLP, M = 32768
+    Mm = 32768
+    wgu, wdn = wl.mlp_weights(3000)
+    I = wdn.shape[1]
+    Wgu = mq.quantize_weight(_to_dev(torch, wgu, dev), gate_up_interleave=True, ws=ws)
+    Wdn = mq.quantize_weight(_to_dev(torch, wdn, dev), ws=ws)
+    X = _to_dev(torch, wl.heavy_tailed_bf16(Mm, K, 3000), dev)
+    wsm = mq.workspace(Mm, K, device=dev)
+    Xq = mq.nvfp4_empty(Mm, K, dev)
+    H = mq.nvfp4_empty(Mm, I, dev)
+    Y = torch.empty((Mm, wdn.shape[0]), dtype=torch.bfloat16, device=dev)
+    # static alpha_h, calibrated once (offline step): amax of h over this batch / (6 * 448)
+    mq.quantize_activation(X, out=Xq, ws=wsm)
+    h_dbg = torch.empty((Mm, I), dtype=torch.bfloat16, device=dev)
+    one = torch.ones(1, dtype=torch.float32, device=dev)
+    mq.prefill_linear(W=Wgu, Xq=Xq, epilogue=mq.MQ_EPI_SILU_MUL_NVFP4, alpha_h=one, H=H, h_debug=h_dbg, ws=wsm)
+    amax_h = float(h_dbg.float().abs().max())
+    del h_dbg
+    ah = torch.full((1,), amax_h / 2688.0 if amax_h > 0 else 1.0, dtype=torch.float32, device=dev)
+    H.alpha.copy_(ah)
+
+    parts = {}
+
+    def mlp(record=None):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        e[0].record()
+        mq.quantize_activation(X, out=Xq, ws=wsm)
+        e[1].record()
+        mq.prefill_linear(W=Wgu, Xq=Xq, epilogue=mq.MQ_EPI_SILU_MUL_NVFP4, alpha_h=ah, H=H, ws=wsm)
+        e[2].record()
+        mq.prefill_linear(W=Wdn, Xq=H, Y=Y, ws=wsm)
+        e[3].record()
+        if record is not None:
+            record.append(e)
+    for _ in range(3):
+        mlp()
+    rec = []
+    ms = _time_calls(torch, lambda: mlp(rec), reps, flush)
+    q_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in rec]))
+    gu_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in rec]))
+    dn_ms = float(np.mean([e[2].elapsed_time(e[3]) for e in rec]))
+    fl_gu = 2 * Mm * wgu.shape[0] * K
+    fl_dn = 2 * Mm * wdn.shape[0] * I
+    out["fused_mlp"] = {"M": Mm, "gate_up": [wgu.shape[0], K], "down": [wdn.shape[0], I], "ms": ms,
+                        "TFLOP/s": (fl_gu + fl_dn) / (ms * 1e-3) / 1e12,
+                        "quant_ms": q_ms, "gate_up_silu_requant_ms": gu_ms, "down_ms": dn_ms,
+                        "gate_up_TFLOP/s": fl_gu / (gu_ms * 1e-3) / 1e12,
+                        "down_TFLOP/s": fl_dn / (dn_ms * 1e-3) / 1e12,
+                        "gate_up_frac": fl_gu / (gu_ms * 1e-3) / 1e12 / fp4_peak}
+    st = mq.async_status(wsm)
+    if st != 0:
+        raise RuntimeError(f"device error in the side measurements: {mq.STATUS_NAMES.get(st)}")
+    return out
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -443,6 +565,9 @@ def run_gpu(args):
         e2e_ms = max_over_ranks(a.elapsed_time(b) / ke, dev)
         line["e2e"] = {"value": whole_job_tflops(flops, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                        "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": ke}
+
+    if not args.no_extras:
+        line["extras"] = measure_extras(mq, torch, dev, flush, hbm_gbs, fp4_peak)
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res = time_oracle(w, xs_h, ws_h, args.cpu_baseline_seconds, steps=1)

@@ -92,64 +92,71 @@ __global__ void __launch_bounds__(D_THREADS, 1)
     const uint32_t tmem_base = *tmem_slot;
 
     if (warp == 0) {
-        if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
-            bool ok = true;
-            int last_stage = -1;
-            uint32_t last_parity = 0;
-            for (int ks = ks_begin; ks < ks_end; ++ks) {
-                if (*abort_flag || !mbar_wait(&empty_bar[stage], phase ^ 1u)) {
-                    ok = false;
-                    break;
-                }
+        // TMA producer: whole warp (warp-uniform values), one elected lane issues
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        int last_stage = -1;
+        uint32_t last_parity = 0;
+        for (int ks = ks_begin; ks < ks_end; ++ks) {
+            if (!warp_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) {
+                ok = false;
+                break;
+            }
+            if (elect_one()) {
                 mbar_arrive_expect_tx(&full_bar[stage], (uint32_t)stage_bytes);
                 uint8_t* sw = smem + stage * stage_bytes;
                 tma_load_2d(sw, &tmap_w, &full_bar[stage], ks * DBK, n_tile * DBM);
                 tma_load_2d(sw + W_STAGE, &tmap_x, &full_bar[stage], ks * DBK, 0);
-                last_stage = stage;
-                last_parity = phase;
-                if (++stage == p.stages) stage = 0, phase ^= 1u;
             }
-            if (!ok) {
+            __syncwarp();
+            last_stage = stage;
+            last_parity = phase;
+            if (++stage == p.stages) stage = 0, phase ^= 1u;
+        }
+        if (!ok) {
+            if (lane == 0) {
                 post_error(p.ctrl, kErrTimeout);
                 *abort_flag = 1;
-                // stages are consumed in order, so the newest issue lands last
-                if (last_stage >= 0) (void)mbar_wait(&full_bar[last_stage], last_parity);
             }
+            // stages are consumed in order, so the newest issue lands last
+            if (last_stage >= 0) (void)mbar_wait(&full_bar[last_stage], last_parity);
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            const uint32_t idesc = idesc_bf16(DBM, p.MT);
-            int stage = 0;
-            uint32_t phase = 0;
-            bool ok = true, next_ready = false;
-            const int NSTAGES_ = p.stages;
-            for (int ks = ks_begin; ks < ks_end; ++ks) {
-                if (!next_ready && (*abort_flag || !mbar_wait(&full_bar[stage], phase))) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                {   // look at the next ring stage now; its result is used next iteration
-                    const int ns = (stage + 1 == NSTAGES_) ? 0 : stage + 1;
-                    next_ready = mbar_test_wait(&full_bar[ns], ns == 0 ? (phase ^ 1u) : phase);
-                }
-                const uint32_t w_addr = smem_u32(smem + stage * stage_bytes);
-                const uint32_t x_addr = w_addr + W_STAGE;
+        // MMA issuer: whole warp, one elected lane issues
+        const uint32_t idesc = idesc_bf16(DBM, p.MT);
+        const uint64_t w_desc0 = sdesc_kmajor_sw128(smem_u32(smem));
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true, next_ready = false;
+        for (int ks = ks_begin; ks < ks_end; ++ks) {
+            if (!next_ready && !warp_wait(&full_bar[stage], phase, abort_flag)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            {   // look at the next ring stage now; its result is used next iteration
+                const int ns = (stage + 1 == p.stages) ? 0 : stage + 1;
+                next_ready = warp_test(&full_bar[ns], ns == 0 ? (phase ^ 1u) : phase);
+            }
+            const uint64_t w_d = w_desc0 + (uint64_t)((stage * stage_bytes) >> 4);
+            const uint64_t x_d = w_d + (uint64_t)(W_STAGE >> 4);
+            if (elect_one()) {
 #pragma unroll
                 for (int kb = 0; kb < 4; ++kb)
-                    umma_bf16(tmem_base, sdesc_kmajor_sw128(w_addr + 32 * kb), sdesc_kmajor_sw128(x_addr + 32 * kb),
-                              idesc, (ks > ks_begin || kb > 0) ? 1u : 0u);
+                    umma_bf16(tmem_base, w_d + (uint64_t)((32 * kb) >> 4), x_d + (uint64_t)((32 * kb) >> 4), idesc,
+                              (ks > ks_begin || kb > 0) ? 1u : 0u);
                 tc_commit(&empty_bar[stage]);
-                if (++stage == p.stages) stage = 0, phase ^= 1u;
             }
-            if (!ok) {
-                post_error(p.ctrl, kErrTimeout);
-                *abort_flag = 1;
-            }
-            tc_commit(acc_full);  // also the "all MMAs done" signal before TMEM is freed
+            __syncwarp();
+            if (++stage == p.stages) stage = 0, phase ^= 1u;
         }
+        if (!ok && lane == 0) {
+            post_error(p.ctrl, kErrTimeout);
+            *abort_flag = 1;
+        }
+        if (elect_one()) tc_commit(acc_full);  // also the "all MMAs done" signal before TMEM is freed
+        __syncwarp();
     } else {
         const int lg = warp & 3;
         const int row = 32 * lg + lane;  // W row within the tile = TMEM lane
@@ -162,7 +169,7 @@ __global__ void __launch_bounds__(D_THREADS, 1)
         for (int c = 0; c < p.MT / 16; ++c) {
             uint32_t r[16];
             tmem_ld_32x32b_x16(t_row + 16 * c, r);
-            tmem_wait_ld();
+            tmem_wait_ld(r);
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 const int m = 16 * c + j;
@@ -224,8 +231,9 @@ cudaError_t launch_decode_bf16(const void* x, int64_t M, const void* w, int64_t 
     const int red_bytes = p.MT * DBM * 4;
     p.bar_offset = std::max(p.stages * stage_bytes, red_bytes);
     const int smem = p.bar_offset + 256 + 1024;
-    // split K so the grid covers the SMs about twice (cluster size <= 8)
-    int split = (2 * di.num_sms + n_tiles - 1) / n_tiles;
+    // split K so that the grid fills the two CTA slots of every SM in one
+    // wave without a partial second wave (cluster size <= 8)
+    int split = (2 * di.num_sms) / n_tiles;
     split = std::max(1, std::min(8, std::min(split, p.k_stages)));
     p.split = split;
 

@@ -287,6 +287,17 @@ __device__ __forceinline__ void tmem_wait_ld()
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// Wait for the TMEM loads, then pass the destination registers through empty
+// volatile asm statements: their later uses depend on those, so the compiler
+// cannot move a use of a loaded register above the wait.
+template <int N>
+__device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[N])
+{
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
+}
+
 // Each thread of the warp reads 32 consecutive 32-bit columns of its own
 // TMEM lane (lane = 32 * (warp % 4) + laneid, encoded in taddr[31:16]).
 __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32])

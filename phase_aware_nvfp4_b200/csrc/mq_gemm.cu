@@ -142,7 +142,7 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const EpiScales& 
         for (int c = 0; c < 8; ++c) {
             uint32_t r[32];
             tmem_ld_32x32b_x32(t_row + 32 * c, r);
-            tmem_wait_ld();
+            tmem_wait_ld(r);
 #pragma unroll
             for (int j = 0; j < 16; ++j)
                 out[16 * c + j] = pack_bf16x2(__fmul_rn(__uint_as_float(r[2 * j]), es.alpha_ab),
@@ -166,7 +166,7 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const EpiScales& 
         for (int c = 0; c < 8; ++c) {
             uint32_t r[32];
             tmem_ld_32x32b_x32(t_row + 32 * c, r);
-            tmem_wait_ld();
+            tmem_wait_ld(r);
             uint32_t cc[2], hbits[8];
             silu_mul_quant_chunk(r, es.alpha_ab, es.alpha_h, es.alpha_h_qmax, cc, scl[c], hbits);
             codes[2 * c] = cc[0];
@@ -244,7 +244,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        if (lane == 0) {
+        // Whole warp (warp-uniform values); one elected lane issues the copies.
+        {
             int stage = 0;
             uint32_t phase = 0;
             uint32_t issued_parity[STAGES];
@@ -257,31 +258,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 const bool two_sfb = (2 * n_blk + 1) < p.sfb_rowblks;
                 const uint32_t tx = A_STAGE + B_STAGE + SFA_STAGE + (two_sfb ? SFB_STAGE : SFB_STAGE / 2);
                 for (int ks = 0; ks < p.k_stages; ++ks) {
-                    if (*abort_flag || !mbar_wait(&empty_bar[stage], phase ^ 1u)) {
+                    if (!warp_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) {
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&full_bar[stage], tx);
-                    tma_load_2d(smem + OFF_A + stage * A_STAGE, &tmap_a, &full_bar[stage], ks * BK_BYTES,
-                                m_blk * BM);
-                    tma_load_2d(smem + OFF_B + stage * B_STAGE, &tmap_b, &full_bar[stage], ks * BK_BYTES,
-                                n_blk * BN);
-                    bulk_load(smem + OFF_SFA + stage * SFA_STAGE,
-                              p.sfa + ((int64_t)m_blk * p.sfa_atoms + ks * 4) * 512, SFA_STAGE, &full_bar[stage]);
-                    bulk_load(smem + OFF_SFB + stage * SFB_STAGE,
-                              p.sfb + ((int64_t)(2 * n_blk) * p.sfb_atoms + ks * 4) * 512, 2048, &full_bar[stage]);
-                    if (two_sfb)
-                        bulk_load(smem + OFF_SFB + stage * SFB_STAGE + 2048,
-                                  p.sfb + ((int64_t)(2 * n_blk + 1) * p.sfb_atoms + ks * 4) * 512, 2048,
-                                  &full_bar[stage]);
+                    if (elect_one()) {
+                        mbar_arrive_expect_tx(&full_bar[stage], tx);
+                        tma_load_2d(smem + OFF_A + stage * A_STAGE, &tmap_a, &full_bar[stage], ks * BK_BYTES,
+                                    m_blk * BM);
+                        tma_load_2d(smem + OFF_B + stage * B_STAGE, &tmap_b, &full_bar[stage], ks * BK_BYTES,
+                                    n_blk * BN);
+                        bulk_load(smem + OFF_SFA + stage * SFA_STAGE,
+                                  p.sfa + ((int64_t)m_blk * p.sfa_atoms + ks * 4) * 512, SFA_STAGE, &full_bar[stage]);
+                        bulk_load(smem + OFF_SFB + stage * SFB_STAGE,
+                                  p.sfb + ((int64_t)(2 * n_blk) * p.sfb_atoms + ks * 4) * 512, 2048, &full_bar[stage]);
+                        if (two_sfb)
+                            bulk_load(smem + OFF_SFB + stage * SFB_STAGE + 2048,
+                                      p.sfb + ((int64_t)(2 * n_blk + 1) * p.sfb_atoms + ks * 4) * 512, 2048,
+                                      &full_bar[stage]);
+                    }
+                    __syncwarp();
                     issued[stage] = true;
                     issued_parity[stage] = phase;
                     if (++stage == STAGES) stage = 0, phase ^= 1u;
                 }
             }
             if (!ok) {
-                post_error(p.ctrl, kErrTimeout);
-                *abort_flag = 1;
+                if (lane == 0) {
+                    post_error(p.ctrl, kErrTimeout);
+                    *abort_flag = 1;
+                }
                 // let every copy already in flight land before the CTA exits
                 for (int s = 0; s < STAGES; ++s)
                     if (issued[s]) (void)mbar_wait(&full_bar[s], issued_parity[s]);
@@ -289,57 +295,65 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        // Whole warp; descriptors formed once and advanced by (offset >> 4)
+        // in their 14-bit start-address field; one elected lane issues.
+        {
+            const uint64_t a_desc0 = sdesc_kmajor_sw128(smem_u32(smem + OFF_A));
+            const uint64_t b_desc0 = sdesc_kmajor_sw128(smem_u32(smem + OFF_B));
+            const uint64_t sfa_desc0 = sdesc_sf_block(smem_u32(smem + OFF_SFA));
+            const uint64_t sfb_desc0 = sdesc_sf_block(smem_u32(smem + OFF_SFB));
+            const uint32_t sfa_tmem = tmem_base + TMEM_SF;
+            const uint32_t sfb_tmem = sfa_tmem + 16;
             int stage = 0;
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true, next_ready = false;
-            constexpr int NSTAGES_ = STAGES;
-            const uint32_t d_tmem = tmem_base;
             for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
-                if (*abort_flag || !mbar_wait(acc_empty, acc_phase ^ 1u)) {
+                if (!warp_wait(acc_empty, acc_phase ^ 1u, abort_flag)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 for (int ks = 0; ks < p.k_stages; ++ks) {
-                    if (!next_ready && (*abort_flag || !mbar_wait(&full_bar[stage], phase))) {
+                    if (!next_ready && !warp_wait(&full_bar[stage], phase, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     {   // look at the next ring stage now; its result is used next iteration
-                        const int ns = (stage + 1 == NSTAGES_) ? 0 : stage + 1;
-                        next_ready = mbar_test_wait(&full_bar[ns], ns == 0 ? (phase ^ 1u) : phase);
+                        const int ns = (stage + 1 == STAGES) ? 0 : stage + 1;
+                        next_ready = warp_test(&full_bar[ns], ns == 0 ? (phase ^ 1u) : phase);
                     }
-                    const uint32_t a_base = smem_u32(smem + OFF_A + stage * A_STAGE);
-                    const uint32_t b_base = smem_u32(smem + OFF_B + stage * B_STAGE);
-                    const uint32_t sfa_base = smem_u32(smem + OFF_SFA + stage * SFA_STAGE);
-                    const uint32_t sfb_base = smem_u32(smem + OFF_SFB + stage * SFB_STAGE);
-                    const uint32_t sfa_tmem = tmem_base + TMEM_SF;
-                    const uint32_t sfb_tmem = sfa_tmem + 16;
-                    // per k-block: its scale copies, then its MMA (interleaving lets the
-                    // copies overlap the previous MMA in the tensor pipe)
+                    const uint64_t a_d = a_desc0 + (uint64_t)((stage * A_STAGE) >> 4);
+                    const uint64_t b_d = b_desc0 + (uint64_t)((stage * B_STAGE) >> 4);
+                    const uint64_t sfa_d = sfa_desc0 + (uint64_t)((stage * SFA_STAGE) >> 4);
+                    const uint64_t sfb_d = sfb_desc0 + (uint64_t)((stage * SFB_STAGE) >> 4);
+                    // per k-block: its scale copies, then its MMA
+                    if (elect_one()) {
 #pragma unroll
-                    for (int kb = 0; kb < 4; ++kb) {
-                        tmem_cp_32x128b_x4(sfa_tmem + 4 * kb, sdesc_sf_block(sfa_base + kb * 512));
-                        tmem_cp_32x128b_x4(sfb_tmem + 8 * kb, sdesc_sf_block(sfb_base + kb * 512));
-                        tmem_cp_32x128b_x4(sfb_tmem + 8 * kb + 4, sdesc_sf_block(sfb_base + 2048 + kb * 512));
-                        umma_nvfp4(d_tmem, sdesc_kmajor_sw128(a_base + kb * 32), sdesc_kmajor_sw128(b_base + kb * 32),
-                                   IDESC, sfa_tmem + 4 * kb, sfb_tmem + 8 * kb, (ks | kb) != 0 ? 1u : 0u);
+                        for (int kb = 0; kb < 4; ++kb) {
+                            tmem_cp_32x128b_x4(sfa_tmem + 4 * kb, sfa_d + (uint64_t)((kb * 512) >> 4));
+                            tmem_cp_32x128b_x4(sfb_tmem + 8 * kb, sfb_d + (uint64_t)((kb * 512) >> 4));
+                            tmem_cp_32x128b_x4(sfb_tmem + 8 * kb + 4, sfb_d + (uint64_t)((2048 + kb * 512) >> 4));
+                            umma_nvfp4(tmem_base, a_d + (uint64_t)((kb * 32) >> 4), b_d + (uint64_t)((kb * 32) >> 4),
+                                       IDESC, sfa_tmem + 4 * kb, sfb_tmem + 8 * kb, (ks | kb) != 0 ? 1u : 0u);
+                        }
+                        tc_commit(&empty_bar[stage]);
                     }
-                    tc_commit(&empty_bar[stage]);
+                    __syncwarp();
                     if (++stage == STAGES) stage = 0, phase ^= 1u;
                 }
                 if (!ok) break;
-                tc_commit(acc_full);
+                if (elect_one()) tc_commit(acc_full);
+                __syncwarp();
                 acc_phase ^= 1u;
             }
-            if (!ok) {
+            if (!ok && lane == 0) {
                 post_error(p.ctrl, kErrTimeout);
                 *abort_flag = 1;
             }
             // every MMA / copy issued above has finished before TMEM is freed
-            tc_commit(mma_done);
+            if (elect_one()) tc_commit(mma_done);
+            __syncwarp();
             (void)mbar_wait(mma_done, 0);
         }
     } else {
@@ -433,7 +447,7 @@ __device__ __forceinline__ void epilogue_half_bf16_tma(const EpiScales& es, uint
     for (int c = 0; c < 4; ++c) {
         uint32_t r[32];
         tmem_ld_32x32b_x32(t_col + 32 * c, r);
-        tmem_wait_ld();
+        tmem_wait_ld(r);
 #pragma unroll
         for (int j = 0; j < 16; ++j)
             out[16 * c + j] = pack_bf16x2(__fmul_rn(__uint_as_float(r[2 * j]), es.alpha_ab),
@@ -469,22 +483,27 @@ template <class Barrier>
 __device__ __forceinline__ void epilogue_half_mlp(const Params& p, const EpiScales& es, uint32_t t_col, int half,
                                                   int64_t row, int n_blk, int lane, Barrier arrive)
 {
+    // drain the raw accumulator first and release TMEM, so the next tile's
+    // MMAs run while this warp does the SiLU-mul and requantization
+    uint32_t acc[4][32];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(t_col + 32 * c, acc[c]);
+    tmem_wait_ld(acc[0]);
+#pragma unroll
+    for (int c = 1; c < 4; ++c) tmem_wait_ld(acc[c]);
+    release_acc_warp(lane, arrive);
     uint32_t codes[8];
     uint32_t scl[4];
     uint32_t hb[32];
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(t_col + 32 * c, r);
-        tmem_wait_ld();
         uint32_t cc[2], hbits[8];
-        silu_mul_quant_chunk(r, es.alpha_ab, es.alpha_h, es.alpha_h_qmax, cc, scl[c], hbits);
+        silu_mul_quant_chunk(acc[c], es.alpha_ab, es.alpha_h, es.alpha_h_qmax, cc, scl[c], hbits);
         codes[2 * c] = cc[0];
         codes[2 * c + 1] = cc[1];
 #pragma unroll
         for (int j = 0; j < 8; ++j) hb[8 * c + j] = hbits[j];
     }
-    release_acc_warp(lane, arrive);
     const int hN = p.N / 2;
     const int hcol0 = n_blk * (BN / 2) + 64 * half;   // first h column of this half
     const int nch = min(4, (hN - hcol0) / 16);
