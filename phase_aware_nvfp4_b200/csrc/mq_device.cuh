@@ -546,16 +546,49 @@ __device__ __forceinline__ uint32_t e2m1x8_encode(const float (&x)[8], float enc
                       __fmul_rn(x[4], enc), __fmul_rn(x[5], enc), __fmul_rn(x[6], enc), __fmul_rn(x[7], enc));
 }
 
+// Per-halfword unsigned maximum (PTX max.u16x2).  The magnitude bits of a
+// non-negative bf16 order like the values, so this is a two-wide |bf16| max.
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
 // |bf16| maximum of 16 values held as 8 packed words (exact, NaN/Inf not
 // expected: a non-finite input is reported by the amax pass).
 __device__ __forceinline__ float bf16x16_absmax(const uint32_t (&w)[8])
 {
-    uint32_t m = __vmaxu2(w[0] & 0x7FFF7FFFu, w[1] & 0x7FFF7FFFu);
-    m = __vmaxu2(m, __vmaxu2(w[2] & 0x7FFF7FFFu, w[3] & 0x7FFF7FFFu));
-    m = __vmaxu2(m, __vmaxu2(__vmaxu2(w[4] & 0x7FFF7FFFu, w[5] & 0x7FFF7FFFu),
-                             __vmaxu2(w[6] & 0x7FFF7FFFu, w[7] & 0x7FFF7FFFu)));
+    const uint32_t m01 = max_u16x2(w[0] & 0x7FFF7FFFu, w[1] & 0x7FFF7FFFu);
+    const uint32_t m23 = max_u16x2(w[2] & 0x7FFF7FFFu, w[3] & 0x7FFF7FFFu);
+    const uint32_t m45 = max_u16x2(w[4] & 0x7FFF7FFFu, w[5] & 0x7FFF7FFFu);
+    const uint32_t m67 = max_u16x2(w[6] & 0x7FFF7FFFu, w[7] & 0x7FFF7FFFu);
+    const uint32_t m = max_u16x2(max_u16x2(m01, m23), max_u16x2(m45, m67));
     const uint32_t b = max(m & 0xFFFFu, m >> 16);
     return __uint_as_float(b << 16);
+}
+
+// E4M3 codes (RNE, satfinite) of two non-negative values in one conversion:
+// low byte = code of lo, next byte = code of hi.
+__device__ __forceinline__ uint32_t e4m3x2_round_sat(float lo, float hi)
+{
+    uint16_t pair;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pair) : "f"(fminf(hi, 448.0f)), "f"(fminf(lo, 448.0f)));
+    return pair;
+}
+
+// Eq. 3 block scale code Pi_E4M3(fl(amax / aq)) without a division on the
+// common path.  inv_lo <= 1/aq <= inv_hi are adjacent floats, so the exact
+// quotient lies in [amax*inv_lo, amax*inv_hi]; rounding is monotone, hence
+// fl(amax/aq) lies between the two rounded products and, when both round to
+// the same E4M3 code, so does it.  Otherwise (a product pair straddling an
+// E4M3 rounding boundary) the correctly rounded division decides.
+__device__ __forceinline__ uint32_t e4m3_block_scale(float amax, float aq, float inv_lo, float inv_hi)
+{
+    const uint32_t pair = e4m3x2_round_sat(__fmul_rn(amax, inv_lo), __fmul_rn(amax, inv_hi));
+    const uint32_t c = pair & 0xFFu;
+    if (c == (pair >> 8)) return c;
+    return e4m3_round_sat(__fdiv_rn(amax, aq));
 }
 
 // Byte offset of scale (row r, 16-element block kb) in the MMA scale layout:

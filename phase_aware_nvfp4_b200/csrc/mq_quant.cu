@@ -28,34 +28,54 @@ __device__ __forceinline__ void amax_accum(uint32_t w, uint32_t& mx, uint32_t& b
     const uint32_t mag = w & 0x7FFF7FFFu;
     const uint32_t nonfin = __vcmpgeu2(mag, 0x7F807F80u);  // 0xFFFF per NaN/Inf halfword
     bad |= nonfin;
-    mx = __vmaxu2(mx, mag & ~nonfin);
+    mx = max_u16x2(mx, mag & ~nonfin);
 }
 
-__global__ void __launch_bounds__(kAmaxThreads) amax_kernel(const uint4* __restrict__ x, int64_t n_vec,
+// Fast path: magnitude maximum including NaN/Inf (two operations per word).
+// A maximum halfword >= 0x7F80 means a non-finite value was seen; only then
+// is the thread's range scanned again with amax_accum.
+__device__ __forceinline__ void amax_accum_fast(uint32_t w, uint32_t& mx)
+{
+    mx = max_u16x2(mx, w & 0x7FFF7FFFu);
+}
+
+__global__ void __launch_bounds__(kAmaxThreads, MQ_AMAX_BLOCKS_PER_SM) amax_kernel(const uint4* __restrict__ x, int64_t n_vec,
                                                             float* __restrict__ alpha_out, WsControl* ctrl,
                                                             uint32_t* __restrict__ partials)
 {
     uint32_t mx = 0, bad = 0;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    int64_t i = i0;
     for (; i + (kAmaxUnroll - 1) * stride < n_vec; i += kAmaxUnroll * stride) {
         uint4 v[kAmaxUnroll];
 #pragma unroll
         for (int u = 0; u < kAmaxUnroll; ++u) v[u] = __ldg(x + i + u * stride);
 #pragma unroll
         for (int u = 0; u < kAmaxUnroll; ++u) {
-            amax_accum(v[u].x, mx, bad);
-            amax_accum(v[u].y, mx, bad);
-            amax_accum(v[u].z, mx, bad);
-            amax_accum(v[u].w, mx, bad);
+            amax_accum_fast(v[u].x, mx);
+            amax_accum_fast(v[u].y, mx);
+            amax_accum_fast(v[u].z, mx);
+            amax_accum_fast(v[u].w, mx);
         }
     }
     for (; i < n_vec; i += stride) {
         const uint4 v = __ldg(x + i);
-        amax_accum(v.x, mx, bad);
-        amax_accum(v.y, mx, bad);
-        amax_accum(v.z, mx, bad);
-        amax_accum(v.w, mx, bad);
+        amax_accum_fast(v.x, mx);
+        amax_accum_fast(v.y, mx);
+        amax_accum_fast(v.z, mx);
+        amax_accum_fast(v.w, mx);
+    }
+    if (max(mx & 0xFFFFu, mx >> 16) >= 0x7F80u) {
+        // a NaN/Inf in this thread's range: rescan it for the finite maximum
+        mx = 0;
+        for (i = i0; i < n_vec; i += stride) {
+            const uint4 v = __ldg(x + i);
+            amax_accum(v.x, mx, bad);
+            amax_accum(v.y, mx, bad);
+            amax_accum(v.z, mx, bad);
+            amax_accum(v.w, mx, bad);
+        }
     }
     uint32_t m = max(mx & 0xFFFFu, mx >> 16) | (bad ? 0x80000000u : 0u);
     // block reduction (the non-finite flag rides in bit 31)
@@ -131,7 +151,8 @@ cudaError_t launch_amax(const void* x, int64_t n, float* alpha_out, WsControl* c
 // thread owns one 16-element block per step: a half-warp covers one row's
 // 256 columns (two 16-byte loads per thread, 512 contiguous bytes per
 // half-warp), so the block amax needs no shuffles and the per-block work
-// (one E4M3 rounding, two divisions) is paid once per 16 elements.  Codes
+// (two products and one conversion for the E4M3 scale, one table lookup for
+// its reciprocal) is paid once per 16 elements.  Codes
 // come from the conversion instruction (two per cvt) and leave as one
 // 8-byte store per thread; scales are staged in shared memory and written
 // as 16-byte stores.
@@ -155,11 +176,24 @@ __global__ void __launch_bounds__(kQuantThreads, MQ_QUANT_MIN_BLOCKS) quantize_k
                                                                  int64_t interleave_half)
 {
     __shared__ __align__(16) uint8_t sf_stage[2048];
+    __shared__ float enc_tab[128];   // fl(1 / fl(alpha * sigma)) for every E4M3 code sigma
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int half = lane >> 4;   // which of the two rows of a step
     const int blk = lane & 15;    // 16-element block within the 256-column chunk
     const float alpha = *alpha_ptr;
     const float alpha_qmax = __fmul_rn(alpha, 6.0f);
+    // 1/alpha_qmax bracketed by the floats next to fl(1/alpha_qmax) (see
+    // e4m3_block_scale).  When that reciprocal is not a normal finite float
+    // the bracket [0, inf] sends every block to the exact division.
+    const float inv_near = __frcp_rn(alpha_qmax);
+    const bool inv_normal = inv_near >= 1.17549435e-38f && inv_near < 3.0e38f;
+    const float inv_lo = inv_normal ? __uint_as_float(__float_as_uint(inv_near) - 1u) : 0.0f;
+    const float inv_hi = inv_normal ? __uint_as_float(__float_as_uint(inv_near) + 1u) : __int_as_float(0x7F800000);
+    if (threadIdx.x < 128) {
+        const float d = __fmul_rn(alpha, e4m3_to_float((uint32_t)threadIdx.x));
+        enc_tab[threadIdx.x] = (d == 0.0f) ? 0.0f : __frcp_rn(d);
+    }
+    __syncthreads();
     const int64_t chunks = (K + 255) / 256;              // 256-column chunks per row block
     const int64_t tiles = ((rows + 127) / 128) * chunks;
 
@@ -194,10 +228,9 @@ __global__ void __launch_bounds__(kQuantThreads, MQ_QUANT_MIN_BLOCKS) quantize_k
                                        v[u][1].x, v[u][1].y, v[u][1].z, v[u][1].w};
                 // Eq. 3: sigma_b = Pi_E4M3(amax_b / (alpha * q_max))
                 const float amax = bf16x16_absmax(w);
-                const uint32_t sc = e4m3_round_sat(__fdiv_rn(amax, alpha_qmax));
+                const uint32_t sc = e4m3_block_scale(amax, alpha_qmax, inv_lo, inv_hi);
                 // Eq. 2: q_i = Pi_FP4(x_i / (alpha * sigma_b)), as x * fl(1/fl(alpha*sigma))
-                const float d = __fmul_rn(alpha, e4m3_to_float(sc));
-                const float enc = (d == 0.0f) ? 0.0f : __frcp_rn(d);   // == fl(1/d)
+                const float enc = enc_tab[sc];
                 float f0[8], f1[8];
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {

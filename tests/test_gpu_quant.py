@@ -85,6 +85,36 @@ def test_every_e2m1_tie_and_e4m3_midpoint():
     _check_quant(x, mq.quantize_activation(to_dev(x)))
 
 
+@pytest.mark.parametrize("alpha", [0.125, 0.1, 1.0 / 6.0, 0.0371, 3.3e-3, 7.5])
+def test_block_scale_rounding_near_e4m3_midpoints(alpha):
+    """Block maxima placed on and next to every E4M3 rounding midpoint times
+    alpha*6 (the BF16 values nearest to it and two BF16 steps either side), for
+    several static tensor scales: the block-scale code must match the oracle's
+    Pi_E4M3(fl32(amax_b / fl32(alpha*6))) exactly, ties included."""
+    a32 = np.float32(alpha)
+    aq = np.float32(a32 * np.float32(6.0))
+    grid = np.array([oracle.e4m3_value(c) for c in range(0x7F)])
+    mids = (grid[1:] + grid[:-1]) / 2
+    rng = np.random.default_rng(int(alpha * 1e4))
+    blocks = []
+    for m in mids:
+        centre = wl.f32_to_bf16_bits(np.array([m * float(aq)], np.float32))[0]
+        for d in (-2, -1, 0, 1, 2):
+            b = int(centre) + d
+            if not 0 < b < 0x7F80:
+                continue
+            amax_b = wl.bf16_bits_to_f32(np.array([b], np.uint16))[0]
+            blk = (rng.uniform(-1, 1, 16) * amax_b).astype(np.float32)
+            blk[rng.integers(16)] = -amax_b if d % 2 else amax_b
+            blocks.append(blk)
+    v = np.concatenate(blocks)
+    v = np.concatenate([v, np.zeros((-len(v)) % 64, np.float32)]).reshape(-1, 64)
+    x = wl.f32_to_bf16_bits(v)
+    # block maxima must survive the BF16 rounding of the filler values
+    t = mq.quantize_activation(to_dev(x), alpha_static=torch.tensor([float(a32)], device="cuda"))
+    _check_quant(x, t, alpha_expected=float(a32))
+
+
 def test_static_alpha_and_saturation():
     x = wl.heavy_tailed_bf16(256, 512, 8)
     alpha = np.float32(0.01)   # far too small: many blocks clip at sigma = 448 and codes at 6
