@@ -199,6 +199,17 @@ MQ_API mq_status mq_unswizzle_scales(const mq_nvfp4* t, uint8_t* rowmajor_out, m
  * v), two device uint64 the caller zero-fills.  Both must stay 0. */
 MQ_API mq_status mq_selftest_e2m1(unsigned long long* mismatch_counts, mq_stream_t stream);
 
+/* Self-test of the failure path: one warp waits, with the same bounded
+ * mbarrier wait every pipeline stage uses, for a phase that nothing ever
+ * completes.  After timeout_ns (1 .. 2e9) the wait gives up, MQ_ERR_TIMEOUT is
+ * posted to workspace `ws` (read it with mq_async_status) and the kernel
+ * returns normally: no fault, the context stays usable.  If waited_ns is not
+ * NULL (8-byte aligned device pointer) it receives the nanoseconds waited.
+ * Returns MQ_ERR_INVALID_ARG for a timeout out of range.  The method has no
+ * counterpart: it checks this library's own error reporting. */
+MQ_API mq_status mq_selftest_timeout(void* ws, size_t ws_bytes, uint64_t timeout_ns, unsigned long long* waited_ns,
+                                     mq_stream_t stream);
+
 /* Synchronize `stream`, then read and clear the asynchronous error bits of
  * workspace `ws`: MQ_OK, MQ_ERR_NONFINITE, MQ_ERR_TIMEOUT (or MQ_ERR_CUDA if
  * the synchronization itself failed). */

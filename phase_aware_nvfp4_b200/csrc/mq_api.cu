@@ -342,6 +342,20 @@ mq_status mq_selftest_e2m1(unsigned long long* mismatch_counts, mq_stream_t stre
     return cuda_status(launch_selftest_e2m1(mismatch_counts, di, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+mq_status mq_selftest_timeout(void* ws, size_t ws_bytes, uint64_t timeout_ns, unsigned long long* waited_ns,
+                              mq_stream_t stream)
+{
+    if (timeout_ns == 0 || timeout_ns > kWaitTimeoutNs) return MQ_ERR_INVALID_ARG;
+    if (waited_ns != nullptr && (reinterpret_cast<uintptr_t>(waited_ns) & 7u) != 0) return MQ_ERR_ALIGNMENT;
+    mq_status st = check_ws(ws, ws_bytes, kWsControlBytes);
+    if (st != MQ_OK) return st;
+    DeviceInfo di;
+    st = check_device(&di);
+    if (st != MQ_OK) return st;
+    return cuda_status(launch_selftest_timeout(static_cast<WsControl*>(ws), timeout_ns, waited_ns,
+                                               reinterpret_cast<cudaStream_t>(stream)));
+}
+
 mq_status mq_async_status(void* ws, mq_stream_t stream)
 {
     if (ws == nullptr) return MQ_ERR_INVALID_ARG;

@@ -11,6 +11,10 @@
 // cost, so the grid must cover every SM: the K dimension is split across the
 // CTAs of a thread-block cluster and the partial sums are reduced through
 // distributed shared memory (no global scratch, deterministic order).
+#include <map>
+#include <mutex>
+#include <tuple>
+
 #include "mq_device.cuh"
 
 namespace mq {
@@ -210,6 +214,45 @@ __global__ void __launch_bounds__(D_THREADS, 1)
 
 }  // namespace
 
+// CTAs of decode_bf16_kernel that can be resident at once when launched in
+// clusters of `cluster` CTAs with `smem` bytes of dynamic shared memory.
+static int max_resident_ctas(int cluster, int smem, const DeviceInfo& di)
+{
+    static std::mutex mu;
+    static std::map<std::tuple<int, int, int>, int> cache;
+    const auto key = std::make_tuple(di.device, cluster, smem);
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+    int ctas = 0;
+    if (cudaFuncSetAttribute(decode_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess) {
+        if (cluster == 1) {
+            int per_sm = 0;
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_bf16_kernel, D_THREADS, smem) ==
+                cudaSuccess)
+                ctas = per_sm * di.num_sms;
+        } else {
+            cudaLaunchConfig_t cfg{};
+            cfg.gridDim = dim3((unsigned)(cluster * di.num_sms), 1, 1);
+            cfg.blockDim = dim3(D_THREADS, 1, 1);
+            cfg.dynamicSmemBytes = (size_t)smem;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = (unsigned)cluster;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            int clusters = 0;
+            if (cudaOccupancyMaxActiveClusters(&clusters, decode_bf16_kernel, &cfg) == cudaSuccess)
+                ctas = clusters * cluster;
+        }
+    }
+    (void)cudaGetLastError();   // a failed query is not an error of the caller's stream
+    cache[key] = ctas;
+    return ctas;
+}
+
 cudaError_t launch_decode_bf16(const void* x, int64_t M, const void* w, int64_t N, int64_t K, void* y,
                                WsControl* ctrl, const DeviceInfo& di, cudaStream_t s)
 {
@@ -231,10 +274,21 @@ cudaError_t launch_decode_bf16(const void* x, int64_t M, const void* w, int64_t 
     const int red_bytes = p.MT * DBM * 4;
     p.bar_offset = std::max(p.stages * stage_bytes, red_bytes);
     const int smem = p.bar_offset + 256 + 1024;
-    // split K so that the grid fills the two CTA slots of every SM in one
-    // wave without a partial second wave (cluster size <= 8)
-    int split = (2 * di.num_sms) / n_tiles;
-    split = std::max(1, std::min(8, std::min(split, p.k_stages)));
+    // K split = cluster size, a power of two <= 8: the split that runs the
+    // grid in one wave with the most CTAs streaming W at once.  How many
+    // clusters of a size can be resident depends on how they pack into the
+    // GPCs, so it is asked of the runtime (and cached per size and smem).
+    int split = 1, best_streams = 0;
+    for (int sp = 1; sp <= 8 && sp <= p.k_stages; sp *= 2) {
+        const int active = max_resident_ctas(sp, smem, di);
+        if (active <= 0) continue;
+        const int ctas = n_tiles * sp;
+        const int streams = std::min(ctas, active);
+        if (ctas <= active && streams > best_streams) {
+            best_streams = streams;
+            split = sp;
+        }
+    }
     p.split = split;
 
     CUtensorMap tw, tx;

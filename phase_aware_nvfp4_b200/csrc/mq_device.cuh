@@ -110,14 +110,14 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity)
 // Wait until the phase with the given parity has completed.  Bounded: gives
 // up after kWaitTimeoutNs of wall time and returns false, so a lost arrival
 // turns into an error status instead of a hung GPU.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity)
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns = kWaitTimeoutNs)
 {
     const uint32_t a = smem_u32(bar);
     if (mbar_try_wait_hint(a, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
         if (mbar_try_wait_hint(a, parity)) return true;
-        if (globaltimer_ns() - t0 > kWaitTimeoutNs) return false;
+        if (globaltimer_ns() - t0 > timeout_ns) return false;
     }
 }
 
@@ -126,9 +126,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity)
 // loop under elect_one() read their operands from uniform registers).
 // Every lane observes the phase itself; the vote makes the result (and so
 // the control flow after it) identical across the warp.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* abort_flag)
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* abort_flag,
+                                          uint64_t timeout_ns = kWaitTimeoutNs)
 {
-    const bool ok = !*abort_flag && mbar_wait(bar, parity);
+    const bool ok = !*abort_flag && mbar_wait(bar, parity, timeout_ns);
     return __all_sync(0xffffffffu, ok);
 }
 

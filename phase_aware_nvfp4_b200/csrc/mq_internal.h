@@ -69,6 +69,9 @@ cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float*
 // Sweep of the E2M1 conversion instruction against the definition; adds
 // mismatch counts for positive / negative inputs into counts[0] / counts[1].
 cudaError_t launch_selftest_e2m1(unsigned long long* counts, const DeviceInfo& di, cudaStream_t s);
+// A bounded mbarrier wait that runs out (nothing arrives): posts kErrTimeout.
+cudaError_t launch_selftest_timeout(WsControl* ctrl, uint64_t timeout_ns, unsigned long long* waited_ns,
+                                    cudaStream_t s);
 
 cudaError_t launch_unswizzle(const uint8_t* scales, int64_t rows, int64_t K, uint8_t* out, cudaStream_t s);
 

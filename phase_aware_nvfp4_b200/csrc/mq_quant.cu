@@ -298,6 +298,36 @@ cudaError_t launch_selftest_e2m1(unsigned long long* counts, const DeviceInfo& d
     return cudaGetLastError();
 }
 
+// Failure-detection self-test: one warp waits, with the pipelines' own
+// warp-voted bounded wait, for a phase of an mbarrier that nothing ever
+// arrives on; when the wait gives up after timeout_ns the kernel posts
+// kErrTimeout to the workspace control block and returns normally, so the
+// context stays usable.  waited_ns receives the wall time spent waiting.
+__global__ void selftest_timeout_kernel(WsControl* ctrl, uint64_t timeout_ns, unsigned long long* waited_ns)
+{
+    __shared__ uint64_t bar;
+    __shared__ uint32_t abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_mbarrier_init();
+    }
+    __syncthreads();
+    const uint64_t t0 = globaltimer_ns();
+    const bool ok = warp_wait(&bar, 0, &abort_flag, timeout_ns);
+    if (threadIdx.x == 0) {
+        if (!ok) post_error(ctrl, kErrTimeout);
+        if (waited_ns != nullptr) *waited_ns = globaltimer_ns() - t0;
+    }
+}
+
+cudaError_t launch_selftest_timeout(WsControl* ctrl, uint64_t timeout_ns, unsigned long long* waited_ns,
+                                    cudaStream_t s)
+{
+    selftest_timeout_kernel<<<1, 32, 0, s>>>(ctrl, timeout_ns, waited_ns);
+    return cudaGetLastError();
+}
+
 // ==========================================================================
 // Scale layout -> plain row-major [rows, K/16] (test and inspection helper)
 // ==========================================================================

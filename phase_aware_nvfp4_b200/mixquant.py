@@ -32,7 +32,7 @@ STATUS_NAMES = {0: "MQ_OK", 1: "MQ_ERR_INVALID_ARG", 2: "MQ_ERR_SHAPE", 3: "MQ_E
 # Every symbol the header declares (checked by the ABI tests).
 EXPORTS = ("mq_status_string", "mq_version", "mq_nvfp4_sizes", "mq_workspace_bytes", "mq_quantize_weight",
            "mq_quantize_activation", "mq_prefill_linear", "mq_decode_linear", "mq_unswizzle_scales",
-           "mq_async_status", "mq_prefill_linear_noalloc", "mq_selftest_e2m1")
+           "mq_async_status", "mq_prefill_linear_noalloc", "mq_selftest_e2m1", "mq_selftest_timeout")
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
@@ -84,6 +84,8 @@ def load(path: str = LIB_PATH):
             lib.mq_async_status.restype = i32
             lib.mq_selftest_e2m1.argtypes = [vp, vp]
             lib.mq_selftest_e2m1.restype = i32
+            lib.mq_selftest_timeout.argtypes = [vp, sz, ctypes.c_uint64, vp, vp]
+            lib.mq_selftest_timeout.restype = i32
             lib.mq_prefill_linear_noalloc.argtypes = [vp, i64, nvp, vp, vp, vp]
             lib.mq_prefill_linear_noalloc.restype = i32
             _lib = lib
@@ -250,6 +252,16 @@ def selftest_e2m1(stream=None):
     _check(load().mq_selftest_e2m1(_ptr(counts), _stream(stream)), "mq_selftest_e2m1")
     c = counts.cpu().tolist()
     return int(c[0]), int(c[1])
+
+
+def selftest_timeout(ws, timeout_ns: int, stream=None) -> int:
+    """mq_selftest_timeout: a bounded wait that runs out; returns the nanoseconds waited.
+    Read the posted MQ_ERR_TIMEOUT with async_status(ws)."""
+    torch = _torch()
+    waited = torch.zeros(1, dtype=torch.int64, device=ws.device)
+    _check(load().mq_selftest_timeout(*_ws_args(ws), ctypes.c_uint64(int(timeout_ns)), _ptr(waited), _stream(stream)),
+           "mq_selftest_timeout")
+    return int(waited.cpu()[0])
 
 
 def async_status(ws, stream=None) -> int:

@@ -103,6 +103,11 @@ def test_argument_errors_are_synchronous(lib):
     assert lib.mq_quantize_weight(P, 200, 256, 1, ctypes.byref(out), ws, wsb, None) == 2
     assert lib.mq_quantize_weight(P, 200, 256, 0, None, ws, wsb, None) == 1
     assert lib.mq_async_status(None, None) == 1
+    # timeout self-test: timeout in (0, 2 s], a workspace, an aligned result slot
+    assert lib.mq_selftest_timeout(ws, wsb, ctypes.c_uint64(0), None, None) == 1
+    assert lib.mq_selftest_timeout(ws, wsb, ctypes.c_uint64(3 * 10 ** 9), None, None) == 1
+    assert lib.mq_selftest_timeout(None, wsb, ctypes.c_uint64(10 ** 6), None, None) == 4
+    assert lib.mq_selftest_timeout(ws, wsb, ctypes.c_uint64(10 ** 6), ctypes.c_void_p(P + 4), None) == 3
     del h
 
 
