@@ -269,27 +269,40 @@ cudaError_t launch_decode_bf16(const void* x, int64_t M, const void* w, int64_t 
     const int n_tiles = (int)((N + DBM - 1) / DBM);
     const int x_stage = p.MT * DBK * 2;
     const int stage_bytes = W_STAGE + x_stage;
-    // ~100 KB of pipeline per CTA: two CTAs share an SM and keep ~190 KB of W in flight
-    p.stages = std::max(2, std::min(8, 100 * 1024 / stage_bytes));
+    // Launch shape.  W streams from HBM, so what matters is how many bytes
+    // are in flight: about kSaturateBytes over the whole GPU keep HBM busy.
+    // Candidates: K split (= cluster size) a power of two <= 8, with either a
+    // shallow pipeline (~100 KB, two CTAs per SM) or a deep one (~200 KB, one
+    // CTA per SM).  How many clusters of a size can be resident depends on how
+    // they pack into the GPCs, so that is asked of the runtime (cached).  A
+    // candidate must run in one wave; the most bytes in flight (capped at the
+    // saturation point) wins, then the smaller split, then the shallow pipeline.
+    constexpr int64_t kSaturateBytes = 16ll << 20;
     const int red_bytes = p.MT * DBM * 4;
-    p.bar_offset = std::max(p.stages * stage_bytes, red_bytes);
-    const int smem = p.bar_offset + 256 + 1024;
-    // K split = cluster size, a power of two <= 8: the split that runs the
-    // grid in one wave with the most CTAs streaming W at once.  How many
-    // clusters of a size can be resident depends on how they pack into the
-    // GPCs, so it is asked of the runtime (and cached per size and smem).
-    int split = 1, best_streams = 0;
+    int best_split = 1, best_stages = std::max(2, std::min(8, 100 * 1024 / stage_bytes));
+    int64_t best_score = -1;
     for (int sp = 1; sp <= 8 && sp <= p.k_stages; sp *= 2) {
-        const int active = max_resident_ctas(sp, smem, di);
-        if (active <= 0) continue;
-        const int ctas = n_tiles * sp;
-        const int streams = std::min(ctas, active);
-        if (ctas <= active && streams > best_streams) {
-            best_streams = streams;
-            split = sp;
+        const int per_cta_stages = (p.k_stages + sp - 1) / sp;
+        for (int deep = 0; deep < 2; ++deep) {
+            int st = deep ? std::min(12, 200 * 1024 / stage_bytes) : std::min(8, 100 * 1024 / stage_bytes);
+            st = std::max(2, std::min(st, std::max(2, per_cta_stages)));
+            const int sm = std::max(st * stage_bytes, red_bytes) + 256 + 1024;
+            if ((size_t)sm > di.max_smem_optin) continue;
+            const int active = max_resident_ctas(sp, sm, di);
+            const int ctas = n_tiles * sp;
+            if (active <= 0 || ctas > active) continue;
+            const int64_t score = std::min<int64_t>(kSaturateBytes, (int64_t)ctas * st * stage_bytes);
+            if (score > best_score) {
+                best_score = score;
+                best_split = sp;
+                best_stages = st;
+            }
         }
     }
-    p.split = split;
+    p.split = best_split;
+    p.stages = best_stages;
+    p.bar_offset = std::max(p.stages * stage_bytes, red_bytes);
+    const int smem = p.bar_offset + 256 + 1024;
 
     CUtensorMap tw, tx;
     if (!make_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w, (uint64_t)K, (uint64_t)N, (uint64_t)K * 2, DBK, DBM,
@@ -302,13 +315,13 @@ cudaError_t launch_decode_bf16(const void* x, int64_t M, const void* w, int64_t 
     cudaError_t e = cudaFuncSetAttribute(decode_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3((unsigned)(n_tiles * split), 1, 1);
+    cfg.gridDim = dim3((unsigned)(n_tiles * p.split), 1, 1);
     cfg.blockDim = dim3(D_THREADS, 1, 1);
     cfg.dynamicSmemBytes = (size_t)smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)split;
+    attr[0].val.clusterDim.x = (unsigned)p.split;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
