@@ -59,7 +59,8 @@ struct Params {
     const float* alpha_a;
     const float* alpha_b;
     int M, N, K;
-    int num_m_blk, num_tiles, k_stages;
+    int num_m_blk, num_n_blk, num_tiles, k_stages;
+    int n_fastest;      // tile order: 1 = n-block varies fastest, 0 = m-block fastest
     int sfa_atoms, sfb_atoms, sfb_rowblks;
     void* y;
     uint8_t* h_codes;
@@ -69,6 +70,21 @@ struct Params {
     int h_atoms;
     WsControl* ctrl;
 };
+
+// Tile index -> (m block, n block).  The block index of the operand with
+// more bytes varies slowest: the CTAs resident at one time then share a few
+// of its blocks and sweep all blocks of the smaller operand, which stays in
+// L2, instead of every wave re-reading the larger one from HBM.
+__device__ __forceinline__ void tile_coords(const Params& p, int tile, int& m_blk, int& n_blk)
+{
+    if (p.n_fastest) {
+        n_blk = tile % p.num_n_blk;
+        m_blk = tile / p.num_n_blk;
+    } else {
+        m_blk = tile % p.num_m_blk;
+        n_blk = tile / p.num_m_blk;
+    }
+}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 {
@@ -253,8 +269,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int s = 0; s < STAGES; ++s) issued[s] = false, issued_parity[s] = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
-                const int m_blk = tile % p.num_m_blk;
-                const int n_blk = tile / p.num_m_blk;
+                int m_blk, n_blk;
+                tile_coords(p, tile, m_blk, n_blk);
                 const bool two_sfb = (2 * n_blk + 1) < p.sfb_rowblks;
                 const uint32_t tx = A_STAGE + B_STAGE + SFA_STAGE + (two_sfb ? SFB_STAGE : SFB_STAGE / 2);
                 for (int ks = 0; ks < p.k_stages; ++ks) {
@@ -362,8 +378,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         EpiScales es = epi_scales<EPI>(p);
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
-            const int m_blk = tile % p.num_m_blk;
-            const int n_blk = tile / p.num_m_blk;
+            int m_blk, n_blk;
+            tile_coords(p, tile, m_blk, n_blk);
             if (*abort_flag || !mbar_wait(acc_full, acc_phase)) {
                 post_error(p.ctrl, kErrTimeout);
                 *abort_flag = 1;
@@ -582,8 +598,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_NUM_THREADS, 1)
             bool ok = true;
             const uint32_t full0 = map_to_cta(smem_u32(&full_bar[0]), 0);
             for (int tile = pair; tile < p.num_tiles && ok; tile += npairs) {
-                const int m_blk = tile % p.num_m_blk;
-                const int n_blk = tile / p.num_m_blk;
+                int m_blk, n_blk;
+                tile_coords(p, tile, m_blk, n_blk);
                 const int a_row = m_blk * 2 * BM + (int)rank * BM;
                 const int b_row = n_blk * BN + (int)rank * 128;
                 const int sfa_row = (m_blk * 2 + (int)rank) * p.sfa_atoms;
@@ -693,8 +709,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_NUM_THREADS, 1)
         auto arrive = [&] { mbar_arrive_cluster(leader_acc_empty); };
         uint32_t acc_phase = 0;
         for (int tile = pair; tile < p.num_tiles; tile += npairs) {
-            const int m_blk = tile % p.num_m_blk;
-            const int n_blk = tile / p.num_m_blk;
+            int m_blk, n_blk;
+            tile_coords(p, tile, m_blk, n_blk);
             if (!warp_wait(acc_full, acc_phase, abort_flag)) {
                 if (lane == 0) {
                     post_error(p.ctrl, kErrTimeout);
@@ -779,7 +795,9 @@ cudaError_t launch_gemm_nvfp4(const GemmArgs& a, const DeviceInfo& di, cudaStrea
                           (uint64_t)a.N * 2, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B))
             return cudaErrorInvalidValue;
         p.num_m_blk = (int)((a.M + 2 * BM - 1) / (2 * BM));
+        p.num_n_blk = num_n_blk;
         p.num_tiles = p.num_m_blk * num_n_blk;
+        p.n_fastest = a.M > a.N;   // A (M rows) is the larger operand: sweep N fastest
         const int pairs = std::min(p.num_tiles, di.num_sms / 2);
         if (a.epilogue == 0) {
             auto k = gemm_nvfp4_pair_kernel<0>;
@@ -800,7 +818,9 @@ cudaError_t launch_gemm_nvfp4(const GemmArgs& a, const DeviceInfo& di, cudaStrea
                       (uint64_t)(a.K / 2), BK_BYTES, BN, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     p.num_m_blk = (int)((a.M + BM - 1) / BM);
+    p.num_n_blk = num_n_blk;
     p.num_tiles = p.num_m_blk * num_n_blk;
+    p.n_fastest = 0;   // M <= 128: a single m block
     const int grid = std::min(p.num_tiles, di.num_sms);
     if (a.epilogue == 0) {
         auto k = gemm_nvfp4_kernel<0>;
