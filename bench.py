@@ -321,7 +321,9 @@ def measure_extras(mq, torch, dev, flush, hbm_gbs, fp4_peak, reps=10):
     """Side measurements of the other workloads (the main line is the projection step):
 
     * phase-aware pair on one BF16 master weight [12288, 4096]: BF16 decode at
-      M = 1, 8, 32, 64 tokens (HBM roofline: 2NK + 2MK + 2MN bytes) and NVFP4
+      M = 1, 8, 32, 64 tokens (HBM roofline: 2NK + 2MK + 2MN bytes), the
+      uniform-NVFP4 decode on its NVFP4 copy (0.5625 NK + 2MK + 2MN bytes;
+      includes quantizing the tokens), and NVFP4
       prefill (quantize + GEMM) at M = 16384, plus the NVFP4-vs-BF16 output
       error of the two paths on the first 64 prefill tokens;
     * fused MLP at M = 32768: activation quantization, gate/up GEMM with the
@@ -342,6 +344,17 @@ def measure_extras(mq, torch, dev, flush, hbm_gbs, fp4_peak, reps=10):
         gbs = (2 * N * K + 2 * M * K + 2 * M * N) / (ms * 1e-3) / 1e9
         dec[str(M)] = {"ms": ms, "GB/s": gbs, "frac": gbs / hbm_gbs}
     Wq = mq.quantize_weight(Wm, ws=ws)
+    # uniform-NVFP4 decode on the same weight: activations quantized on the fly, NVFP4 weight
+    decq = {}
+    for M in (1, 8, 32, 64):
+        x = _to_dev(torch, wl.heavy_tailed_bf16(M, K, 4000 + M), dev)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        wsd = mq.workspace(M, K, device=dev)
+        for _ in range(3):
+            mq.decode_linear_nvfp4(x, Wq, Y=y, ws=wsd)
+        ms = _time_calls(torch, lambda: mq.decode_linear_nvfp4(x, Wq, Y=y, ws=wsd), reps, flush)
+        gbs = (0.5625 * N * K + 2 * M * K + 2 * M * N) / (ms * 1e-3) / 1e9
+        decq[str(M)] = {"ms": ms, "GB/s": gbs, "frac": gbs / hbm_gbs, "speedup_vs_bf16": dec[str(M)]["ms"] / ms}
     Mp = 16384
     X = _to_dev(torch, wl.heavy_tailed_bf16(Mp, K, 4000), dev)
     Xq = mq.nvfp4_empty(Mp, K, dev)
@@ -361,6 +374,7 @@ def measure_extras(mq, torch, dev, flush, hbm_gbs, fp4_peak, reps=10):
         "weight": [N, K], "decode_bf16": dec,
         "roofline_decode": {"bound": "hbm", "kernel": "decode_bf16_kernel", "unit": "GB/s", "peak": hbm_gbs,
                             "achieved": dec["64"]["GB/s"], "frac": dec["64"]["frac"], "M": 64},
+        "decode_nvfp4": decq,
         "prefill_nvfp4": {"M": Mp, "ms": ms, "TFLOP/s": 2 * Mp * N * K / (ms * 1e-3) / 1e12},
         "nvfp4_vs_bf16_rel_frobenius": err}
     del X, Xq, Y

@@ -188,6 +188,19 @@ MQ_API mq_status mq_decode_linear(const void* X_bf16, int64_t M, const void* W_b
 MQ_API mq_status mq_prefill_linear_noalloc(const void* X_bf16, int64_t M, const mq_nvfp4* W,
                                            const float* alpha_static, void* Y_bf16, mq_stream_t stream);
 
+/* Uniform-NVFP4 decode (the decode side of the paper's "uniform NVFP4"
+ * comparison, Section 4, whose decode also runs in NVFP4):
+ * Y[M,N] = bf16(fl(alpha_x*alpha_w) * sum_k (sigma_x q_x)(sigma_w q_w)), FP32
+ * accumulation, with X [M, K] BF16 quantized on the fly (Eq. 2 / Eq. 3, dynamic
+ * alpha_x unless alpha_static is given) into the workspace, and W the NVFP4
+ * weight from mq_quantize_weight (not gate/up interleaved).  The same weight
+ * bytes as the prefill path; 0.5625 instead of 2 bytes per weight element
+ * streamed per token batch.  M in [1, 128]; K % 64 == 0; N % 16 == 0; X and
+ * Y 16-byte aligned.  Workspace: mq_workspace_bytes(M, K), zero-filled once.
+ * Errors as mq_prefill_linear. */
+MQ_API mq_status mq_decode_linear_nvfp4(const void* X_bf16, int64_t M, const mq_nvfp4* W, const float* alpha_static,
+                                        void* Y_bf16, void* ws, size_t ws_bytes, mq_stream_t stream);
+
 /* Copy the block scales of `t` to plain row-major [rows, cols/16] bytes. */
 MQ_API mq_status mq_unswizzle_scales(const mq_nvfp4* t, uint8_t* rowmajor_out, mq_stream_t stream);
 

@@ -321,6 +321,29 @@ mq_status mq_decode_linear(const void* X_bf16, int64_t M, const void* W_bf16, in
         launch_decode_bf16(X_bf16, M, W_bf16, N, K, Y_bf16, w.ctrl, di, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+mq_status mq_decode_linear_nvfp4(const void* X_bf16, int64_t M, const mq_nvfp4* W, const float* alpha_static,
+                                 void* Y_bf16, void* ws, size_t ws_bytes, mq_stream_t stream)
+{
+    if (X_bf16 == nullptr || Y_bf16 == nullptr) return MQ_ERR_INVALID_ARG;
+    if (W == nullptr || W->codes == nullptr || W->scales == nullptr || W->alpha == nullptr) return MQ_ERR_INVALID_ARG;
+    const int64_t N = W->rows, K = W->cols;
+    if (M < 1 || M > 128 || N < 16 || N % 16 != 0 || K < 64 || K % 64 != 0) return MQ_ERR_SHAPE;
+    if (N > (int64_t)1 << 30 || K > (int64_t)1 << 30) return MQ_ERR_SHAPE;
+    mq_status st = check_nvfp4(W, N, K);
+    if (st != MQ_OK) return st;
+    if (!aligned16(X_bf16) || !aligned16(Y_bf16)) return MQ_ERR_ALIGNMENT;
+    if ((st = check_ws(ws, ws_bytes, ws_bytes_for(M, K))) != MQ_OK) return st;
+    DeviceInfo di;
+    if ((st = check_device(&di)) != MQ_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const Ws w = carve(ws, M, K);
+    const float* ax = nullptr;
+    st = quantize_into(X_bf16, M, K, alpha_static, w.xq_codes, w.xq_scales, &w.ctrl->alpha, false, 0, w, di, s, &ax);
+    if (st != MQ_OK) return st;
+    return cuda_status(launch_decode_nvfp4(w.xq_codes, w.xq_scales, ax, M, W->codes, W->scales, W->alpha, N, K, Y_bf16,
+                                           w.ctrl, di, s));
+}
+
 mq_status mq_unswizzle_scales(const mq_nvfp4* t, uint8_t* rowmajor_out, mq_stream_t stream)
 {
     if (t == nullptr || t->scales == nullptr || rowmajor_out == nullptr) return MQ_ERR_INVALID_ARG;

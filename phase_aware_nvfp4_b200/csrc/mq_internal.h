@@ -98,6 +98,12 @@ cudaError_t launch_gemm_nvfp4(const GemmArgs& a, const DeviceInfo& di, cudaStrea
 cudaError_t launch_decode_bf16(const void* x, int64_t M, const void* w, int64_t N, int64_t K, void* y,
                                WsControl* ctrl, const DeviceInfo& di, cudaStream_t s);
 
+// Uniform-NVFP4 decode: Y[M,N] = bf16(fl(alpha_w*alpha_x) * sum_k dequant)
+// with X [M <= 128, K] and W [N, K] both NVFP4 (codes, MMA-layout scales).
+cudaError_t launch_decode_nvfp4(const uint8_t* x_codes, const uint8_t* x_scales, const float* alpha_x, int64_t M,
+                                const uint8_t* w_codes, const uint8_t* w_scales, const float* alpha_w, int64_t N,
+                                int64_t K, void* y, WsControl* ctrl, const DeviceInfo& di, cudaStream_t s);
+
 // cuTensorMapEncodeTiled obtained from the driver at run time.
 bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t outer,
                   uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz);

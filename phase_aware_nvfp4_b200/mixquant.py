@@ -32,7 +32,8 @@ STATUS_NAMES = {0: "MQ_OK", 1: "MQ_ERR_INVALID_ARG", 2: "MQ_ERR_SHAPE", 3: "MQ_E
 # Every symbol the header declares (checked by the ABI tests).
 EXPORTS = ("mq_status_string", "mq_version", "mq_nvfp4_sizes", "mq_workspace_bytes", "mq_quantize_weight",
            "mq_quantize_activation", "mq_prefill_linear", "mq_decode_linear", "mq_unswizzle_scales",
-           "mq_async_status", "mq_prefill_linear_noalloc", "mq_selftest_e2m1", "mq_selftest_timeout")
+           "mq_async_status", "mq_prefill_linear_noalloc", "mq_selftest_e2m1", "mq_selftest_timeout",
+           "mq_decode_linear_nvfp4")
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
@@ -86,6 +87,8 @@ def load(path: str = LIB_PATH):
             lib.mq_selftest_e2m1.restype = i32
             lib.mq_selftest_timeout.argtypes = [vp, sz, ctypes.c_uint64, vp, vp]
             lib.mq_selftest_timeout.restype = i32
+            lib.mq_decode_linear_nvfp4.argtypes = [vp, i64, nvp, vp, vp, vp, sz, vp]
+            lib.mq_decode_linear_nvfp4.restype = i32
             lib.mq_prefill_linear_noalloc.argtypes = [vp, i64, nvp, vp, vp, vp]
             lib.mq_prefill_linear_noalloc.restype = i32
             _lib = lib
@@ -232,6 +235,18 @@ def decode_linear(X, W, Y=None, ws=None, stream=None):
     ws = ws if ws is not None else workspace(device=X.device)
     _check(load().mq_decode_linear(_ptr(X), M, _ptr(W), N, K, _ptr(Y), *_ws_args(ws), _stream(stream)),
            "mq_decode_linear")
+    return Y
+
+
+def decode_linear_nvfp4(X, W: NVFP4Tensor, alpha_static=None, Y=None, ws=None, stream=None):
+    """mq_decode_linear_nvfp4: Y[M, N] = X[M, K] W^T with X quantized on the fly and W NVFP4 (M <= 128)."""
+    torch = _torch()
+    M = X.shape[0]
+    Y = Y if Y is not None else torch.empty((M, W.rows), dtype=torch.bfloat16, device=X.device)
+    ws = ws if ws is not None else workspace(M, W.cols, X.device)
+    w_c = W.c()
+    _check(load().mq_decode_linear_nvfp4(_ptr(X), M, ctypes.byref(w_c), _ptr(alpha_static), _ptr(Y), *_ws_args(ws),
+                                         _stream(stream)), "mq_decode_linear_nvfp4")
     return Y
 
 

@@ -14,7 +14,9 @@ iteration then launches only the operation named:
   quantized;
 * ``mlp``: the gate/up GEMM with the fused SiLU-mul + NVFP4 requantization
   epilogue (N = 2 x intermediate size, interleaved gate/up rows);
-* ``decode``: the BF16 decode GEMM Y = X W^T (M <= 256).
+* ``decode``: the BF16 decode GEMM Y = X W^T (M <= 256);
+* ``decode_nvfp4``: the uniform-NVFP4 decode (tokens quantized on the fly,
+  NVFP4 weight; M <= 128).
 
 Prints the mean CUDA-event time per iteration.  The data recipe is the one the
 tests and the benchmark use (Student-t(3) activations with 1 % outlier
@@ -30,7 +32,7 @@ import numpy as np
 
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
-    ap.add_argument("op", choices=["quant", "gemm", "mlp", "decode"])
+    ap.add_argument("op", choices=["quant", "gemm", "mlp", "decode", "decode_nvfp4"])
     ap.add_argument("--M", type=int, default=8192)
     ap.add_argument("--N", type=int, default=4096)
     ap.add_argument("--K", type=int, default=4096)
@@ -64,10 +66,14 @@ def main(argv=None) -> int:
             H = mq.nvfp4_empty(a.M, a.N // 2, dev)
             ah = torch.full((1,), 0.25, dtype=torch.float32, device=dev)
             run = lambda: mq.prefill_linear(W=Wq, Xq=Xq, epilogue=mq.MQ_EPI_SILU_MUL_NVFP4, alpha_h=ah, H=H, ws=ws)
-    else:
+    elif a.op == "decode":
         W = dev_bf16(wl.normal_bf16(a.N, a.K, 0.02, 12))
         Y = torch.empty((a.M, a.N), dtype=torch.bfloat16, device=dev)
         run = lambda: mq.decode_linear(X, W, Y=Y, ws=ws)
+    else:
+        Wq = mq.quantize_weight(dev_bf16(wl.normal_bf16(a.N, a.K, 0.02, 12)), ws=ws)
+        Y = torch.empty((a.M, a.N), dtype=torch.bfloat16, device=dev)
+        run = lambda: mq.decode_linear_nvfp4(X, Wq, Y=Y, ws=ws)
     for _ in range(a.warmup):
         run()
     torch.cuda.synchronize()

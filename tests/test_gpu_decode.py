@@ -48,3 +48,68 @@ def test_decode_exact_small_integers():
     y = mq.decode_linear(to_dev(wl.f32_to_bf16_bits(xi)), to_dev(wl.f32_to_bf16_bits(wi)))
     torch.cuda.synchronize()
     assert np.array_equal(to_host_bits(y), oracle.round_bf16((xi.astype(np.float64) @ wi.T.astype(np.float64))))
+
+
+# ---------------------------------------------------------------- uniform-NVFP4 decode
+
+def _nvfp4_decode_check(x, w, y_gpu_bits, alpha_x=None):
+    """Oracle: quantize X (dynamic alpha over its M rows unless given) and W, FP64 block-scaled matmul."""
+    from gpu_helpers import gemm_check
+    ax = oracle.tensor_alpha(x)[1] if alpha_x is None else alpha_x
+    aw = oracle.tensor_alpha(w)[1]
+    y64, sabs = oracle.nvfp4_linear_rows((*oracle.quantize(x, ax), ax), (*oracle.quantize(w, aw), aw))
+    return gemm_check(y_gpu_bits, y64, sabs)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 256, 256), (7, 400, 1088), (32, 512, 1024), (64, 768, 2048),
+                                   (100, 272, 320), (128, 128, 4096), (1, 4096, 12288)])
+def test_decode_nvfp4_vs_oracle(M, N, K):
+    """Ragged tokens (MMA N padded to 32), ragged weight rows (N % 128 != 0) and a partial last
+    256-element stage (K % 256 != 0) are all covered."""
+    x = wl.heavy_tailed_bf16(M, K, 3 * M + K)
+    w = wl.normal_bf16(N, K, 0.02, 5 * N + K)
+    Wq = mq.quantize_weight(to_dev(w))
+    y = mq.decode_linear_nvfp4(to_dev(x), Wq)
+    torch.cuda.synchronize()
+    rel, mx, bmax = _nvfp4_decode_check(x, w, to_host_bits(y))
+    print(f"nvfp4 decode M={M} N={N} K={K}: rel-Frobenius {rel:.2e}")
+
+
+def test_decode_nvfp4_static_alpha_and_grid_inputs_exact():
+    """Grid-valued inputs whose blocks all hold a 6: X with a static alpha of 1 and W with a 2688
+    anchor alone in its block (alpha_w = 1) get block scales of exactly 1 (448 for the anchor), so
+    Y = bf16(X W^T) exactly (the FP32 sums stay below 2^24 quarter units)."""
+    rng = np.random.default_rng(3)
+    grid = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6], np.float32)
+    xi = (rng.choice(grid, size=(16, 512)) * rng.choice([-1, 1], size=(16, 512))).astype(np.float32)
+    wi = (rng.choice(grid, size=(256, 512)) * rng.choice([-1, 1], size=(256, 512))).astype(np.float32)
+    xi[:, ::16] = 6.0
+    wi[:, ::16] = 6.0
+    wi[0, :16] = 0.0
+    wi[0, 0] = 2688.0      # alone in its block (sigma 448 would round its neighbours to 0)
+    Wq = mq.quantize_weight(to_dev(wl.f32_to_bf16_bits(wi)))
+    assert float(Wq.alpha.cpu()[0]) == 1.0
+    y = mq.decode_linear_nvfp4(to_dev(wl.f32_to_bf16_bits(xi)), Wq, alpha_static=torch.ones(1, device="cuda"))
+    torch.cuda.synchronize()
+    exact = xi.astype(np.float64) @ wi.T.astype(np.float64)
+    assert np.array_equal(to_host_bits(y), oracle.round_bf16(exact))
+
+
+def test_decode_nvfp4_matches_prefill_on_same_weight():
+    """Uniform-NVFP4 decode and the NVFP4 prefill linear on the same tokens and the same
+    12288 x 4096 weight agree, and match the oracle on 2048 weight rows."""
+    from gpu_helpers import gemm_check
+    x = wl.heavy_tailed_bf16(64, 4096, 77)
+    w = wl.normal_bf16(12288, 4096, 0.02, 4001)
+    Wq = mq.quantize_weight(to_dev(w))
+    X = to_dev(x)
+    yd = mq.decode_linear_nvfp4(X, Wq)
+    yp = mq.prefill_linear(X, Wq)
+    torch.cuda.synchronize()
+    a, b = oracle.bf16_to_f64(to_host_bits(yd)), oracle.bf16_to_f64(to_host_bits(yp))
+    assert oracle.rel_frobenius(a, b) < 1e-3
+    ax = oracle.tensor_alpha(x)[1]
+    aw = oracle.tensor_alpha(w)[1]
+    wc, wsc = oracle.quantize(w[:2048], aw)
+    y64, sabs = oracle.nvfp4_linear_rows((*oracle.quantize(x, ax), ax), (wc, wsc, aw))
+    gemm_check(to_host_bits(yd)[:, :2048], y64, sabs)
