@@ -149,24 +149,20 @@ mq_status check_ws(void* ws, size_t ws_bytes, size_t need)
     return MQ_OK;
 }
 
-// amax (unless a static alpha is given) + quantize.  Returns the device
+// Tensor amax (unless a static alpha is given) and quantization.  Returns the device
 // pointer of the tensor scale used in *alpha_used.  With a static alpha and
 // copy_static, the value is also copied to alpha_out.
 mq_status quantize_into(const void* x, int64_t rows, int64_t K, const float* alpha_static, uint8_t* codes,
                         uint8_t* scales, float* alpha_out, bool copy_static, int64_t interleave_half,
                         const Ws& w, const DeviceInfo& di, cudaStream_t s, const float** alpha_used)
 {
-    const float* alpha = alpha_static;
-    if (alpha == nullptr) {
-        cudaError_t e = launch_amax(x, rows * K, alpha_out, w.ctrl, w.partials, di, s);
-        if (e != cudaSuccess) return MQ_ERR_CUDA;
-        alpha = alpha_out;
-    } else if (copy_static && alpha_out != alpha_static) {
+    if (alpha_static != nullptr && copy_static && alpha_out != alpha_static) {
         if (cudaMemcpyAsync(alpha_out, alpha_static, sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
             return MQ_ERR_CUDA;
     }
-    if (alpha_used != nullptr) *alpha_used = alpha;
-    return cuda_status(launch_quantize(x, rows, K, alpha, codes, scales, interleave_half, di, s));
+    if (alpha_used != nullptr) *alpha_used = (alpha_static != nullptr) ? alpha_static : alpha_out;
+    return cuda_status(launch_quantize(x, rows, K, alpha_static, alpha_out, codes, scales, interleave_half, w.ctrl,
+                                       w.partials, di, s));
 }
 
 }  // namespace

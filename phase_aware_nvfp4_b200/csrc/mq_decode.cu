@@ -128,7 +128,41 @@ __global__ void __launch_bounds__(D_THREADS, 1)
         bool ok = true;
         int last_stage = -1;
         uint32_t last_parity = 0;
-        for (int ks = ks_begin; ks < ks_end; ++ks) {
+        int ks = ks_begin;
+        if (FMT) {
+            // The tokens and alpha_x come from the quantization kernel just
+            // before this one (programmatic dependent launch): fill the first
+            // ring slots with weight tiles and scales, wait for that kernel,
+            // then add the token tiles to those slots.
+            const int pre = std::min(p.stages, ks_end - ks_begin);
+            if (elect_one()) {
+                for (int i = 0; i < pre; ++i) {
+                    uint8_t* sw = smem + i * stage_bytes;
+                    mbar_arrive_expect_tx(&full_bar[i], (uint32_t)stage_bytes);
+                    tma_load_2d(sw, &tmap_w, &full_bar[i], (ks_begin + i) * (QBK / 2), n_tile * DBM);
+                    tma_load_2d(sw + W_TILE + x_tile, &tmap_sfw, &full_bar[i], 0,
+                                n_tile * p.sfw_atoms + (ks_begin + i) * 4);
+                }
+            }
+            __syncwarp();
+            grid_dep_wait();
+            if (elect_one()) {
+                for (int i = 0; i < pre; ++i) {
+                    uint8_t* sw = smem + i * stage_bytes;
+                    tma_load_2d(sw + W_TILE, &tmap_x, &full_bar[i], (ks_begin + i) * (QBK / 2), 0);
+                    tma_load_2d(sw + W_TILE + x_tile + Q_SF, &tmap_sfx, &full_bar[i], 0, (ks_begin + i) * 4);
+                }
+            }
+            __syncwarp();
+            if (pre > 0) {
+                last_stage = pre - 1;
+                last_parity = 0;
+            }
+            ks += pre;
+            stage = pre;
+            if (stage == p.stages) stage = 0, phase = 1u;
+        }
+        for (; ks < ks_end; ++ks) {
             if (!warp_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) {
                 ok = false;
                 break;
@@ -213,7 +247,9 @@ __global__ void __launch_bounds__(D_THREADS, 1)
         const int row = 32 * lg + lane;  // W row within the tile = TMEM lane
         const int64_t n = (int64_t)n_tile * DBM + row;
         const bool have_acc = ks_end > ks_begin;
-        // FMT 1 output scale fl(alpha_w * alpha_x), applied to the FP32 sum
+        // FMT 1 output scale fl(alpha_w * alpha_x), applied to the FP32 sum;
+        // alpha_x is written by the preceding kernel
+        if (FMT) grid_dep_wait();
         const float out_scale = FMT ? __fmul_rn(*p.alpha_w, *p.alpha_x) : 1.0f;
         bool ok = mbar_wait(acc_full, 0);
         if (!ok) post_error(p.ctrl, kErrTimeout);
@@ -310,7 +346,7 @@ int max_resident_ctas(int cluster, int smem, const DeviceInfo& di)
 // SM).  How many clusters of a size can be resident depends on how they pack
 // into the GPCs, so that is asked of the runtime (cached).  A candidate must
 // run in one wave; the most bytes in flight (capped at the saturation point)
-// wins, then the smaller split, then the shallow pipeline.  Fills split,
+// wins, then the larger grid, then the smaller split and the shallow pipeline.  Fills split,
 // stages, bar_offset; returns the dynamic shared memory size.
 template <int FMT>
 int choose_shape(DParams& p, int n_tiles, const DeviceInfo& di)
@@ -330,7 +366,10 @@ int choose_shape(DParams& p, int n_tiles, const DeviceInfo& di)
             const int active = max_resident_ctas<FMT>(sp, sm, di);
             const int ctas = n_tiles * sp;
             if (active <= 0 || ctas > active) continue;
-            const int64_t score = std::min<int64_t>(kSaturateBytes, (int64_t)ctas * st * stage_bytes);
+            // a CTA streams at a bounded rate, so once the bytes in flight are
+            // saturated more CTAs still help: ties go to the larger grid
+            const int64_t score = std::min<int64_t>(kSaturateBytes, (int64_t)ctas * st * stage_bytes) * 1024 +
+                                  std::min(ctas, 1023);
             if (score > best_score) {
                 best_score = score;
                 best_split = sp;
@@ -356,13 +395,16 @@ cudaError_t launch_shape(const DParams& p, int n_tiles, int smem, const CUtensor
     cfg.blockDim = dim3(D_THREADS, 1, 1);
     cfg.dynamicSmemBytes = (size_t)smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)p.split;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    // FMT 1 follows the token quantization on the stream: let it start early
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = FMT ? 2 : 1;
     e = cudaLaunchKernelEx(&cfg, kern, tw, tx, tsfw, tsfx, p);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();

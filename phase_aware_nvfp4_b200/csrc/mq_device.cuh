@@ -150,6 +150,15 @@ __device__ __forceinline__ bool elect_one()
     return pred != 0;
 }
 
+// Programmatic dependent launch (sm_90+).  A kernel launched with
+// programmatic stream serialization may start before the previous kernel in
+// the stream has finished; grid_dep_wait() blocks the calling thread until
+// that kernel has completed and its memory operations are visible, and
+// grid_dep_launch_dependents() lets the next kernel start early.  Both are
+// no-ops when the launch has no such dependency.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
+
 // --------------------------------------------------------------------------
 // TMA / bulk copies (global -> shared, completion on an mbarrier)
 // --------------------------------------------------------------------------

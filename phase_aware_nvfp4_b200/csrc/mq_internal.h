@@ -22,7 +22,8 @@ constexpr uint32_t kErrTimeout = 2u;    // a pipeline wait gave up
 struct WsControl {
     uint32_t error_bits;   // OR of kErr* posted since the last status query
     uint32_t amax_ticket;  // blocks of the running amax pass that have finished
-    uint32_t reserved[6];
+    uint32_t epoch;        // bumped when a single-launch amax pass publishes its alpha
+    uint32_t reserved[5];
     float alpha;           // tensor scale of the activation quantized in-workspace
     uint32_t pad[55];
 };
@@ -60,11 +61,16 @@ cudaError_t device_info(DeviceInfo* out);
 cudaError_t launch_amax(const void* x, int64_t n, float* alpha_out, WsControl* ctrl, uint32_t* partials,
                         const DeviceInfo& di, cudaStream_t s);
 
-// NVFP4 quantization of X [rows, K] (ld = K) with tensor scale *alpha.
-// interleave_half: 0, or I (= rows/2) to interleave gate/up rows in 16-row
-// groups (output row 32c+t <- input row 16c+t for t<16, I+16c+t-16 else).
-cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float* alpha, uint8_t* codes,
-                            uint8_t* scales, int64_t interleave_half, const DeviceInfo& di, cudaStream_t s);
+// NVFP4 quantization of X [rows, K] (ld = K).  With alpha_static the tensor
+// scale is *alpha_static; otherwise alpha = amax/2688 (1 if amax == 0) is
+// computed first and stored at *alpha_out (kErrNonFinite on NaN/Inf): by the
+// amax kernel, or, for tensors of at most one tile per SM, inside one
+// cooperative launch of the quantization kernel.  interleave_half > 0
+// interleaves gate/up rows in 16-row groups (output row 32c+t <- input row
+// 16c+t for t<16, I+16c+t-16 else).
+cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float* alpha_static, float* alpha_out,
+                            uint8_t* codes, uint8_t* scales, int64_t interleave_half, WsControl* ctrl,
+                            uint32_t* partials, const DeviceInfo& di, cudaStream_t s);
 
 // Sweep of the E2M1 conversion instruction against the definition; adds
 // mismatch counts for positive / negative inputs into counts[0] / counts[1].

@@ -84,12 +84,10 @@ extern "C" MQ_API mq_status mq_prefill_linear_noalloc(const void* X_bf16, int64_
     uint8_t* xq_codes = base + kWsControlBytes;
     uint8_t* xq_scales = xq_codes + codes_b;
 
-    const float* alpha_x = alpha_static;
-    if (alpha_x == nullptr) {
-        if (launch_amax(X_bf16, M * K, &ctrl->alpha, ctrl, partials, di, s) != cudaSuccess) return MQ_ERR_CUDA;
-        alpha_x = &ctrl->alpha;
-    }
-    if (launch_quantize(X_bf16, M, K, alpha_x, xq_codes, xq_scales, 0, di, s) != cudaSuccess) return MQ_ERR_CUDA;
+    const float* alpha_x = (alpha_static != nullptr) ? alpha_static : &ctrl->alpha;
+    if (launch_quantize(X_bf16, M, K, alpha_static, &ctrl->alpha, xq_codes, xq_scales, 0, ctrl, partials, di, s) !=
+        cudaSuccess)
+        return MQ_ERR_CUDA;
 
     GemmArgs g{};
     g.a_codes = xq_codes;

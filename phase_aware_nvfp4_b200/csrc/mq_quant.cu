@@ -1,16 +1,17 @@
-// mq_quant.cu -- NVFP4 quantization on sm_100a: tensor amax (the tensor-level
-// scale) and the block quantizer, after "Mix-Quant: Quantized Prefilling,
-// Precise Decoding for Agentic LLMs", section 3.3, Eq. 2 and Eq. 3.
+// mq_quant.cu -- NVFP4 quantization on sm_100a: the tensor-level scale
+// (tensor amax) and the block quantizer, after "Mix-Quant: Quantized
+// Prefilling, Precise Decoding for Agentic LLMs", section 3.3, Eq. 2 and Eq. 3.
 //
-// Both kernels are HBM-bound streams: 128-bit coalesced loads, a handful of
-// FP32 operations per element, no shared-memory staging of the input.
+// Large tensors: an HBM-bound amax kernel, then the quantization kernel.
+// Tensors of at most one 128 x 256 tile per SM: one cooperative launch of the
+// quantization kernel takes the amax, hands alpha to every block through a
+// bounded grid-wide wait, and quantizes (reading X back from L2), which saves
+// a launch on the decode-sized inputs.
+#include <mutex>
+
 #include "mq_device.cuh"
 
 namespace mq {
-
-// ==========================================================================
-// Tensor amax -> alpha = amax / (q_max * 448)
-// ==========================================================================
 
 #ifndef MQ_AMAX_UNROLL
 #define MQ_AMAX_UNROLL 4
@@ -169,112 +170,341 @@ cudaError_t launch_amax(const void* x, int64_t n, float* alpha_out, WsControl* c
 constexpr int kQuantThreads = 256;
 constexpr int kQuantStepUnroll = MQ_QUANT_UNROLL;   // steps (2 rows per warp each) with loads in flight
 
-__global__ void __launch_bounds__(kQuantThreads, MQ_QUANT_MIN_BLOCKS) quantize_kernel(const uint16_t* __restrict__ x, int64_t rows,
-                                                                 int64_t K, const float* __restrict__ alpha_ptr,
-                                                                 uint8_t* __restrict__ codes,
-                                                                 uint8_t* __restrict__ scales,
-                                                                 int64_t interleave_half)
+// Per-block constants of the Eq. 2 / Eq. 3 arithmetic for one tensor scale.
+struct QuantConsts {
+    float alpha_qmax;       // fl(alpha * q_max)
+    float inv_lo, inv_hi;   // floats bracketing 1 / alpha_qmax (see e4m3_block_scale)
+};
+
+// Fills enc_tab[c] = fl(1 / fl(alpha * sigma_c)) for every E4M3 code c (0 when
+// the product is 0) and returns the block-scale constants.  Every thread of
+// the block calls it; it ends with __syncthreads().
+__device__ __forceinline__ QuantConsts quant_setup(float alpha, float* enc_tab)
 {
-    __shared__ __align__(16) uint8_t sf_stage[2048];
-    __shared__ float enc_tab[128];   // fl(1 / fl(alpha * sigma)) for every E4M3 code sigma
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int half = lane >> 4;   // which of the two rows of a step
-    const int blk = lane & 15;    // 16-element block within the 256-column chunk
-    const float alpha = *alpha_ptr;
-    const float alpha_qmax = __fmul_rn(alpha, 6.0f);
-    // 1/alpha_qmax bracketed by the floats next to fl(1/alpha_qmax) (see
-    // e4m3_block_scale).  When that reciprocal is not a normal finite float
-    // the bracket [0, inf] sends every block to the exact division.
-    const float inv_near = __frcp_rn(alpha_qmax);
+    QuantConsts q;
+    q.alpha_qmax = __fmul_rn(alpha, 6.0f);
+    // When fl(1/alpha_qmax) is not a normal finite float the bracket [0, inf]
+    // sends every block to the exact division.
+    const float inv_near = __frcp_rn(q.alpha_qmax);
     const bool inv_normal = inv_near >= 1.17549435e-38f && inv_near < 3.0e38f;
-    const float inv_lo = inv_normal ? __uint_as_float(__float_as_uint(inv_near) - 1u) : 0.0f;
-    const float inv_hi = inv_normal ? __uint_as_float(__float_as_uint(inv_near) + 1u) : __int_as_float(0x7F800000);
+    q.inv_lo = inv_normal ? __uint_as_float(__float_as_uint(inv_near) - 1u) : 0.0f;
+    q.inv_hi = inv_normal ? __uint_as_float(__float_as_uint(inv_near) + 1u) : __int_as_float(0x7F800000);
     if (threadIdx.x < 128) {
         const float d = __fmul_rn(alpha, e4m3_to_float((uint32_t)threadIdx.x));
         enc_tab[threadIdx.x] = (d == 0.0f) ? 0.0f : __frcp_rn(d);
     }
     __syncthreads();
-    const int64_t chunks = (K + 255) / 256;              // 256-column chunks per row block
-    const int64_t tiles = ((rows + 127) / 128) * chunks;
+    return q;
+}
 
+// Source row of output row r (gate/up interleave in 16-row groups when
+// interleave_half > 0: output row 32c+t <- input row 16c+t for t < 16,
+// I+16c+t-16 otherwise).
+__device__ __forceinline__ int64_t quant_src_row(int64_t r, int64_t interleave_half)
+{
+    if (interleave_half <= 0) return r;
+    const int64_t c = r >> 5, tt = r & 31;
+    return (tt < 16) ? (16 * c + tt) : (interleave_half + 16 * c + (tt - 16));
+}
+
+// The work split of one 128-row x 256-column tile: warp w owns rows 16w..16w+15,
+// taken two per step (lanes 0-15 the even row, 16-31 the odd one); lane l
+// owns the 16-element block l % 16 of the row.  The same split is used for the
+// amax pass and the quantization pass, so both read the same lines.
+__device__ __forceinline__ uint32_t amax_tile(const uint16_t* __restrict__ x, int64_t rows, int64_t K,
+                                              int64_t interleave_half, int64_t rb, int64_t kc, int warp, int half,
+                                              int blk, uint32_t mx)
+{
+    const int64_t col = kc * 256 + 16 * blk;
+    if (col >= K) return mx;
+#pragma unroll 1
+    for (int s0 = 0; s0 < 8; s0 += kQuantStepUnroll) {
+        uint4 v[kQuantStepUnroll][2];
+#pragma unroll
+        for (int u = 0; u < kQuantStepUnroll; ++u) {   // all loads of the group in flight together
+            const int64_t r = rb * 128 + 16 * warp + 2 * (s0 + u) + half;
+            v[u][0] = v[u][1] = make_uint4(0u, 0u, 0u, 0u);
+            if (r < rows) {
+                const uint4* p = reinterpret_cast<const uint4*>(x + quant_src_row(r, interleave_half) * K + col);
+                v[u][0] = __ldg(p);
+                v[u][1] = __ldg(p + 1);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kQuantStepUnroll; ++u) {
+            const uint4 a = v[u][0], b = v[u][1];
+            mx = max_u16x2(mx, max_u16x2(max_u16x2(a.x & 0x7FFF7FFFu, a.y & 0x7FFF7FFFu),
+                                         max_u16x2(a.z & 0x7FFF7FFFu, a.w & 0x7FFF7FFFu)));
+            mx = max_u16x2(mx, max_u16x2(max_u16x2(b.x & 0x7FFF7FFFu, b.y & 0x7FFF7FFFu),
+                                         max_u16x2(b.z & 0x7FFF7FFFu, b.w & 0x7FFF7FFFu)));
+        }
+    }
+    return mx;
+}
+
+// Same tile, finite values only; bad |= non-zero if a NaN/Inf was seen.
+__device__ __noinline__ uint32_t amax_tile_finite(const uint16_t* __restrict__ x, int64_t rows, int64_t K,
+                                                  int64_t interleave_half, int64_t rb, int64_t kc, int warp, int half,
+                                                  int blk, uint32_t mx, uint32_t& bad)
+{
+    const int64_t col = kc * 256 + 16 * blk;
+    if (col >= K) return mx;
+    for (int st = 0; st < 8; ++st) {
+        const int64_t r = rb * 128 + 16 * warp + 2 * st + half;
+        if (r < rows) {
+            const uint4* p = reinterpret_cast<const uint4*>(x + quant_src_row(r, interleave_half) * K + col);
+            const uint4 a = __ldg(p), b = __ldg(p + 1);
+            amax_accum(a.x, mx, bad);
+            amax_accum(a.y, mx, bad);
+            amax_accum(a.z, mx, bad);
+            amax_accum(a.w, mx, bad);
+            amax_accum(b.x, mx, bad);
+            amax_accum(b.y, mx, bad);
+            amax_accum(b.z, mx, bad);
+            amax_accum(b.w, mx, bad);
+        }
+    }
+    return mx;
+}
+
+// Eq. 3 / Eq. 2 for one tile; scales staged in shared memory and written as
+// one contiguous 2 KiB run of the MMA scale layout.
+__device__ __forceinline__ void quant_tile(const uint16_t* __restrict__ x, int64_t rows, int64_t K,
+                                           int64_t interleave_half, int64_t rb, int64_t kc, int64_t chunks,
+                                           const QuantConsts& qc, const float* enc_tab, uint8_t* sf_stage,
+                                           uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, int warp,
+                                           int half, int blk)
+{
+    const int64_t col = kc * 256 + 16 * blk;
+    const bool col_ok = col < K;
+#pragma unroll 1
+    for (int s0 = 0; s0 < 8; s0 += kQuantStepUnroll) {
+        uint4 v[kQuantStepUnroll][2];
+#pragma unroll
+        for (int u = 0; u < kQuantStepUnroll; ++u) {
+            const int64_t r = rb * 128 + 16 * warp + 2 * (s0 + u) + half;
+            v[u][0] = v[u][1] = make_uint4(0u, 0u, 0u, 0u);
+            if (r < rows && col_ok) {
+                const uint4* p = reinterpret_cast<const uint4*>(x + quant_src_row(r, interleave_half) * K + col);
+                v[u][0] = __ldcs(p);
+                v[u][1] = __ldcs(p + 1);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kQuantStepUnroll; ++u) {
+            const int rl = 16 * warp + 2 * (s0 + u) + half;   // row within the 128-row block
+            const int64_t r = rb * 128 + rl;
+            const uint32_t w[8] = {v[u][0].x, v[u][0].y, v[u][0].z, v[u][0].w,
+                                   v[u][1].x, v[u][1].y, v[u][1].z, v[u][1].w};
+            // Eq. 3: sigma_b = Pi_E4M3(amax_b / (alpha * q_max))
+            const float amax = bf16x16_absmax(w);
+            const uint32_t sc = e4m3_block_scale(amax, qc.alpha_qmax, qc.inv_lo, qc.inv_hi);
+            // Eq. 2: q_i = Pi_FP4(x_i / (alpha * sigma_b)), as x * fl(1/fl(alpha*sigma))
+            const float enc = enc_tab[sc];
+            float f0[8], f1[8];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                f0[2 * j] = bf16_lo(w[j]);
+                f0[2 * j + 1] = bf16_hi(w[j]);
+                f1[2 * j] = bf16_lo(w[4 + j]);
+                f1[2 * j + 1] = bf16_hi(w[4 + j]);
+            }
+            const uint32_t c0 = e2m1x8_encode(f0, enc);
+            const uint32_t c1 = e2m1x8_encode(f1, enc);
+            const bool ok = (r < rows) && col_ok;
+            if (ok) *reinterpret_cast<uint2*>(codes + r * (K / 2) + col / 2) = make_uint2(c0, c1);
+            sf_stage[(blk >> 2) * 512 + (rl & 31) * 16 + (rl >> 5) * 4 + (blk & 3)] = ok ? (uint8_t)sc : 0;
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x < 128) {
+        uint4* dst = reinterpret_cast<uint4*>(scales + (rb * chunks + kc) * 2048);
+        dst[threadIdx.x] = reinterpret_cast<const uint4*>(sf_stage)[threadIdx.x];
+    }
+    __syncthreads();
+}
+
+__device__ __forceinline__ uint32_t fold_max_flag(uint32_t a, uint32_t b)
+{
+    return max(a & 0x7FFFFFFFu, b & 0x7FFFFFFFu) | ((a | b) & 0x80000000u);
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p)
+{
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v)
+{
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Quantization of X [rows, K] in one launch.  Tiles of 128 rows x 256
+// columns are dealt to the blocks round robin.
+//   * alpha_static != nullptr: Eq. 2 / Eq. 3 with that tensor scale.
+//   * otherwise (launched cooperatively, every block resident): the blocks
+//     first take the |x| maximum of their tiles; the last block to finish
+//     folds the per-block maxima into alpha = amax / (q_max * 448) (1 for an
+//     all-zero tensor), stores it at alpha_out and publishes it with a
+//     release store of a new epoch number, which the other blocks wait for
+//     (bounded; a wait that runs out posts kErrTimeout and the block stops).
+//     The quantization pass then walks the tiles in the opposite order, so
+//     the lines read last by the amax pass, still in L2, are read first.
+__global__ void __launch_bounds__(kQuantThreads, MQ_QUANT_MIN_BLOCKS)
+    quantize_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t K, const float* __restrict__ alpha_static,
+                    float* __restrict__ alpha_out, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                    int64_t interleave_half, WsControl* ctrl, uint32_t* __restrict__ partials)
+{
+    __shared__ __align__(16) uint8_t sf_stage[2048];
+    __shared__ float enc_tab[128];
+    __shared__ uint32_t s_red[kQuantThreads / 32];
+    __shared__ uint32_t s_epoch, s_last, s_ok;
+    __shared__ float s_alpha;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int half = lane >> 4;
+    const int blk = lane & 15;
+    const int64_t chunks = (K + 255) / 256;
+    const int64_t tiles = ((rows + 127) / 128) * chunks;
+    // a consumer launched with programmatic serialization (the uniform-NVFP4
+    // decode) may start now: it streams its weights and waits for this grid
+    // before it reads the quantized tokens
+    grid_dep_launch_dependents();
+
+    float alpha;
+    if (alpha_static != nullptr) {
+        alpha = *alpha_static;
+    } else {
+        uint32_t* epoch = &ctrl->epoch;
+        if (threadIdx.x == 0) s_epoch = ld_acquire_u32(epoch);
+        // ---- pass 1: |x| maximum of this block's tiles
+        uint32_t mx = 0;
+        for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x)
+            mx = amax_tile(x, rows, K, interleave_half, t / chunks, t % chunks, warp, half, blk, mx);
+        uint32_t m = max(mx & 0xFFFFu, mx >> 16);
+        if (m >= 0x7F80u) {
+            // a NaN/Inf in this thread's share: its finite maximum, and the flag
+            uint32_t bad = 0;
+            mx = 0;
+            for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x)
+                mx = amax_tile_finite(x, rows, K, interleave_half, t / chunks, t % chunks, warp, half, blk, mx, bad);
+            m = max(mx & 0xFFFFu, mx >> 16) | (bad ? 0x80000000u : 0u);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fold_max_flag(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+        if (lane == 0) s_red[warp] = m;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            uint32_t b = 0;
+            for (int w = 0; w < kQuantThreads / 32; ++w) b = fold_max_flag(b, s_red[w]);
+            partials[blockIdx.x] = b;
+            __threadfence();
+            const uint32_t ticket = atomicAdd(&ctrl->amax_ticket, 1u);
+            s_last = (ticket == gridDim.x - 1);
+        }
+        __syncthreads();
+        if (s_last) {
+            // every block's maximum is in `partials`: fold them, publish alpha
+            __threadfence();
+            uint32_t b = 0;
+            for (int j = threadIdx.x; j < (int)gridDim.x; j += blockDim.x) b = fold_max_flag(b, __ldcg(partials + j));
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) b = fold_max_flag(b, __shfl_xor_sync(0xFFFFFFFFu, b, o));
+            __syncthreads();
+            if (lane == 0) s_red[warp] = b;
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                uint32_t r = 0;
+                for (int w = 0; w < kQuantThreads / 32; ++w) r = fold_max_flag(r, s_red[w]);
+                const float amax = __uint_as_float((r & 0x7FFFu) << 16);
+                *alpha_out = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
+                if (r & 0x80000000u) post_error(ctrl, kErrNonFinite);
+                ctrl->amax_ticket = 0;   // ready for the next pass on this workspace
+                __threadfence();
+                st_release_u32(epoch, s_epoch + 1u);
+            }
+        }
+        // ---- every block: wait for the published alpha
+        if (threadIdx.x == 0) {
+            bool ok = ld_acquire_u32(epoch) != s_epoch;
+            if (!ok) {
+                const uint64_t t0 = globaltimer_ns();
+                while (!(ok = (ld_acquire_u32(epoch) != s_epoch))) {
+                    if (globaltimer_ns() - t0 > kWaitTimeoutNs) break;
+                    __nanosleep(64);
+                }
+            }
+            s_ok = ok;
+            s_alpha = ok ? __ldcg(alpha_out) : 0.0f;
+            if (!ok) post_error(ctrl, kErrTimeout);
+        }
+        __syncthreads();
+        if (!s_ok) return;
+        alpha = s_alpha;
+    }
+    const QuantConsts qc = quant_setup(alpha, enc_tab);
+    // ---- pass 2: quantize, tiles in reverse order of pass 1
     for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
         const int64_t tile = tiles - 1 - t;
-        const int64_t rb = tile / chunks, kc = tile % chunks;
-        const int64_t col = kc * 256 + 16 * blk;
-        const bool col_ok = col < K;
-#pragma unroll 1
-        for (int s0 = 0; s0 < 8; s0 += kQuantStepUnroll) {
-            uint4 v[kQuantStepUnroll][2];
-#pragma unroll
-            for (int u = 0; u < kQuantStepUnroll; ++u) {
-                const int64_t r = rb * 128 + 16 * warp + 2 * (s0 + u) + half;
-                v[u][0] = v[u][1] = make_uint4(0u, 0u, 0u, 0u);
-                if (r < rows && col_ok) {
-                    int64_t src = r;
-                    if (interleave_half > 0) {
-                        const int64_t c = r >> 5, tt = r & 31;
-                        src = (tt < 16) ? (16 * c + tt) : (interleave_half + 16 * c + (tt - 16));
-                    }
-                    const uint4* p = reinterpret_cast<const uint4*>(x + src * K + col);
-                    v[u][0] = __ldcs(p);
-                    v[u][1] = __ldcs(p + 1);
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < kQuantStepUnroll; ++u) {
-                const int rl = 16 * warp + 2 * (s0 + u) + half;   // row within the 128-row block
-                const int64_t r = rb * 128 + rl;
-                const uint32_t w[8] = {v[u][0].x, v[u][0].y, v[u][0].z, v[u][0].w,
-                                       v[u][1].x, v[u][1].y, v[u][1].z, v[u][1].w};
-                // Eq. 3: sigma_b = Pi_E4M3(amax_b / (alpha * q_max))
-                const float amax = bf16x16_absmax(w);
-                const uint32_t sc = e4m3_block_scale(amax, alpha_qmax, inv_lo, inv_hi);
-                // Eq. 2: q_i = Pi_FP4(x_i / (alpha * sigma_b)), as x * fl(1/fl(alpha*sigma))
-                const float enc = enc_tab[sc];
-                float f0[8], f1[8];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    f0[2 * j] = bf16_lo(w[j]);
-                    f0[2 * j + 1] = bf16_hi(w[j]);
-                    f1[2 * j] = bf16_lo(w[4 + j]);
-                    f1[2 * j + 1] = bf16_hi(w[4 + j]);
-                }
-                const uint32_t c0 = e2m1x8_encode(f0, enc);
-                const uint32_t c1 = e2m1x8_encode(f1, enc);
-                const bool ok = (r < rows) && col_ok;
-                if (ok) *reinterpret_cast<uint2*>(codes + r * (K / 2) + col / 2) = make_uint2(c0, c1);
-                sf_stage[(blk >> 2) * 512 + (rl & 31) * 16 + (rl >> 5) * 4 + (blk & 3)] = ok ? (uint8_t)sc : 0;
-            }
-        }
-        __syncthreads();
-        if (threadIdx.x < 128) {
-            uint4* dst = reinterpret_cast<uint4*>(scales + (rb * chunks + kc) * 2048);
-            dst[threadIdx.x] = reinterpret_cast<const uint4*>(sf_stage)[threadIdx.x];
-        }
-        __syncthreads();
+        quant_tile(x, rows, K, interleave_half, tile / chunks, tile % chunks, chunks, qc, enc_tab, sf_stage, codes,
+                   scales, warp, half, blk);
     }
 }
 
-cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float* alpha, uint8_t* codes,
-                            uint8_t* scales, int64_t interleave_half, const DeviceInfo& di, cudaStream_t s)
+// Resident blocks per SM of quantize_kernel (cached per device).
+static int quantize_blocks_per_sm(const DeviceInfo& di)
 {
-    const int64_t tiles = ((rows + 127) / 128) * ((K + 255) / 256);
-    int64_t blocks = (int64_t)di.num_sms * (MQ_QUANT_MIN_BLOCKS > 4 ? MQ_QUANT_MIN_BLOCKS : 4);
-    if (blocks > tiles) blocks = tiles;
-    if (blocks < 1) blocks = 1;
-    quantize_kernel<<<(unsigned)blocks, kQuantThreads, 0, s>>>(static_cast<const uint16_t*>(x), rows, K, alpha,
-                                                               codes, scales, interleave_half);
-    return cudaGetLastError();
+    static std::mutex mu;
+    static int per_sm[64] = {};
+    std::lock_guard<std::mutex> lock(mu);
+    if (di.device >= 0 && di.device < 64 && per_sm[di.device] > 0) return per_sm[di.device];
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quantize_kernel, kQuantThreads, 0) != cudaSuccess) {
+        (void)cudaGetLastError();
+        occ = 0;
+    }
+    if (di.device >= 0 && di.device < 64 && occ > 0) per_sm[di.device] = occ;
+    return occ;
 }
 
-// ==========================================================================
-// Self-test of the E2M1 conversion instruction against the definition
-// ==========================================================================
-//
-// For every FP32 bit pattern p in [0, 0x41000000] (0 .. 8.0) and its
-// negative, compare the conversion instruction with the comparison-chain
-// rounding of the definition (nearest E2M1 magnitude, ties to even, clip at
-// 6, sign kept).  Counts mismatches into counts[0] (positive) / counts[1].
+cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float* alpha_static, float* alpha_out,
+                            uint8_t* codes, uint8_t* scales, int64_t interleave_half, WsControl* ctrl,
+                            uint32_t* partials, const DeviceInfo& di, cudaStream_t s)
+{
+    const int64_t tiles = ((rows + 127) / 128) * ((K + 255) / 256);
+    const int occ = quantize_blocks_per_sm(di);
+    const int64_t resident = (int64_t)di.num_sms * std::max(1, occ);
+    // Small tensors (at most one tile per SM): one cooperative launch takes
+    // the amax, hands alpha to every block and quantizes; the two-kernel path
+    // would pay a second launch and its ramp for a few microseconds of work.
+    // Larger tensors: the amax kernel (full occupancy) and then the
+    // quantization kernel with that alpha.
+    const bool single = (alpha_static == nullptr) && tiles <= di.num_sms && occ > 0;
+    const float* alpha_in = alpha_static;
+    if (alpha_static == nullptr && !single) {
+        cudaError_t e = launch_amax(x, rows * K, alpha_out, ctrl, partials, di, s);
+        if (e != cudaSuccess) return e;
+        alpha_in = alpha_out;
+    }
+    int64_t blocks = std::min(tiles, resident);
+    if (blocks > kAmaxMaxBlocks) blocks = kAmaxMaxBlocks;
+    if (blocks < 1) blocks = 1;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)blocks, 1, 1);
+    cfg.blockDim = dim3(kQuantThreads, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = single ? 1 : 0;   // blocks wait on one another only in the single-launch amax
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, quantize_kernel, static_cast<const uint16_t*>(x), rows, K, alpha_in,
+                                       alpha_out, codes, scales, interleave_half, ctrl, partials);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
 
 __global__ void selftest_e2m1_kernel(unsigned long long* counts)
 {
