@@ -317,13 +317,31 @@ def _time_calls(torch, fn, reps, flush):
     return float(np.mean([a.elapsed_time(b) for a, b in evs]))
 
 
+def _time_rotating(torch, calls, reps):
+    """Mean device time (ms) of one call, cycling through `calls` (each on its
+    own copy of the weights, together larger than L2, so every call streams
+    its weights from HBM while the kernels' code and descriptors stay warm).
+    A spin kernel before each call keeps the GPU busy while the host enqueues."""
+    evs = []
+    for i in range(reps):
+        torch.cuda._sleep(200_000)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        calls[i % len(calls)]()
+        b.record()
+        evs.append((a, b))
+    torch.cuda.synchronize()
+    return float(np.mean([a.elapsed_time(b) for a, b in evs]))
+
+
 def measure_extras(mq, torch, dev, flush, hbm_gbs, fp4_peak, reps=10):
     """Side measurements of the other workloads (the main line is the projection step):
 
     * phase-aware pair on one BF16 master weight [12288, 4096]: BF16 decode at
       M = 1, 8, 32, 64 tokens (HBM roofline: 2NK + 2MK + 2MN bytes), the
       uniform-NVFP4 decode on its NVFP4 copy (0.5625 NK + 2MK + 2MN bytes;
-      includes quantizing the tokens), and NVFP4
+      includes quantizing the tokens) -- both timed on rotating weight copies
+      larger than L2 (weights cold, code warm) -- and NVFP4
       prefill (quantize + GEMM) at M = 16384, plus the NVFP4-vs-BF16 output
       error of the two paths on the first 64 prefill tokens;
     * fused MLP at M = 32768: activation quantization, gate/up GEMM with the
@@ -334,27 +352,27 @@ def measure_extras(mq, torch, dev, flush, hbm_gbs, fp4_peak, reps=10):
     N, K = 12288, 4096
     Wm = _to_dev(torch, wl.normal_bf16(N, K, 0.02, 4001), dev)
     ws = mq.workspace(16384, K, device=dev)
-    dec = {}
-    for M in (1, 8, 32, 64):
-        x = _to_dev(torch, wl.heavy_tailed_bf16(M, K, 4000 + M), dev)
-        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-        for _ in range(3):
-            mq.decode_linear(x, Wm, Y=y, ws=ws)
-        ms = _time_calls(torch, lambda: mq.decode_linear(x, Wm, Y=y, ws=ws), reps, flush)
-        gbs = (2 * N * K + 2 * M * K + 2 * M * N) / (ms * 1e-3) / 1e9
-        dec[str(M)] = {"ms": ms, "GB/s": gbs, "frac": gbs / hbm_gbs}
     Wq = mq.quantize_weight(Wm, ws=ws)
-    # uniform-NVFP4 decode on the same weight: activations quantized on the fly, NVFP4 weight
-    decq = {}
+    # decode: weights cold (copies cycled, 4 x 100 MB BF16 / 12 x 28 MB NVFP4 > L2), code warm
+    Wm_copies = [Wm] + [Wm.clone() for _ in range(3)]
+    Wq_copies = [Wq] + [mq.NVFP4Tensor(Wq.codes.clone(), Wq.scales.clone(), Wq.alpha.clone(), Wq.rows, Wq.cols)
+                        for _ in range(11)]
+    dec, decq = {}, {}
     for M in (1, 8, 32, 64):
         x = _to_dev(torch, wl.heavy_tailed_bf16(M, K, 4000 + M), dev)
         y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
         wsd = mq.workspace(M, K, device=dev)
-        for _ in range(3):
-            mq.decode_linear_nvfp4(x, Wq, Y=y, ws=wsd)
-        ms = _time_calls(torch, lambda: mq.decode_linear_nvfp4(x, Wq, Y=y, ws=wsd), reps, flush)
-        gbs = (0.5625 * N * K + 2 * M * K + 2 * M * N) / (ms * 1e-3) / 1e9
-        decq[str(M)] = {"ms": ms, "GB/s": gbs, "frac": gbs / hbm_gbs, "speedup_vs_bf16": dec[str(M)]["ms"] / ms}
+        bf = [lambda W=W: mq.decode_linear(x, W, Y=y, ws=wsd) for W in Wm_copies]
+        q4 = [lambda W=W: mq.decode_linear_nvfp4(x, W, Y=y, ws=wsd) for W in Wq_copies]
+        for f in bf + q4:
+            f()
+        ms = _time_rotating(torch, bf, 4 * reps)
+        gbs = (2 * N * K + 2 * M * K + 2 * M * N) / (ms * 1e-3) / 1e9
+        dec[str(M)] = {"ms": ms, "GB/s": gbs, "frac": gbs / hbm_gbs}
+        msq = _time_rotating(torch, q4, 4 * reps)
+        gbs = (0.5625 * N * K + 2 * M * K + 2 * M * N) / (msq * 1e-3) / 1e9
+        decq[str(M)] = {"ms": msq, "GB/s": gbs, "frac": gbs / hbm_gbs, "speedup_vs_bf16": ms / msq}
+    del Wm_copies, Wq_copies
     Mp = 16384
     X = _to_dev(torch, wl.heavy_tailed_bf16(Mp, K, 4000), dev)
     Xq = mq.nvfp4_empty(Mp, K, dev)
