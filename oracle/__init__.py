@@ -81,6 +81,8 @@ def _L():
             lib.orc_tensor_alpha.restype = ctypes.c_int
             lib.orc_quantize_rows.argtypes = [u16p, i64, i64, ctypes.c_float, u8p, u8p]
             lib.orc_quantize_rows.restype = None
+            lib.orc_quantize_rows_search.argtypes = [u16p, i64, i64, ctypes.c_float, u8p, u8p]
+            lib.orc_quantize_rows_search.restype = None
             lib.orc_dequantize_rows.argtypes = [u8p, u8p, i64, i64, ctypes.c_float, f64p]
             lib.orc_dequantize_rows.restype = None
             lib.orc_round_bf16.argtypes = [f64p, i64, u16p]
@@ -149,20 +151,25 @@ def tensor_alpha(x_bf16: np.ndarray):
     return float(amax.value), float(np.float32(alpha.value)), bool(bad)
 
 
-def quantize(x_bf16: np.ndarray, alpha: float):
+def quantize(x_bf16: np.ndarray, alpha: float, search: bool = False):
     """NVFP4-quantize BF16 rows [rows, K] with tensor scale ``alpha``.
 
     Returns (codes [rows, K/2] uint8, scales [rows, K/16] uint8 E4M3 codes),
     the plain row-major layout: element k of a row sits in byte k/2, even k
     in the low nibble; scale b covers elements 16b..16b+15.
+
+    ``search``: per block, the Eq. 3 scale code and its two E4M3 neighbours
+    are tried and the one with the smallest binary32 squared error is kept
+    (the opt-in "scale optimization" reading; ties keep the Eq. 3 scale).
     """
     x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
     assert x.ndim == 2 and x.shape[1] % BLOCK == 0
     rows, K = x.shape
     codes = np.empty((rows, K // 2), dtype=np.uint8)
     scales = np.empty((rows, K // BLOCK), dtype=np.uint8)
-    _L().orc_quantize_rows(_ptr(x, ctypes.c_uint16), rows, K, ctypes.c_float(alpha),
-                           _ptr(codes, ctypes.c_uint8), _ptr(scales, ctypes.c_uint8))
+    fn = _L().orc_quantize_rows_search if search else _L().orc_quantize_rows
+    fn(_ptr(x, ctypes.c_uint16), rows, K, ctypes.c_float(alpha), _ptr(codes, ctypes.c_uint8),
+       _ptr(scales, ctypes.c_uint8))
     return codes, scales
 
 

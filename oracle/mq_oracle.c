@@ -33,6 +33,10 @@
  *     |x| * fl(1 / fl(alpha * sigma)); a block with alpha * sigma == 0 gets
  *     all-zero magnitudes.  Eq. 3's quotient is fl(amax_b / fl(alpha * 6)).
  *   - Packing: element k of a row goes to byte k/2, even k in the low nibble.
+ *   - Scale optimization (mentioned once, never defined): an opt-in search
+ *     per block over the Eq. 3 scale code and its two E4M3 neighbours,
+ *     keeping the one with the smallest binary32 squared error (ties keep
+ *     the Eq. 3 scale); off by default.
  *
  * Floating point: IEEE binary32 / binary64 with no contraction (compile with
  * -ffp-contract=off) and no fast-math.  Dequantization and every matmul are
@@ -213,6 +217,67 @@ static unsigned quantize_block(const uint16_t* xb, float alpha, unsigned char co
     return sigma_code;
 }
 
+/* ------------------------------------------------------------------------ */
+/* Optional scale search (the paper's "scale optimization", read as a       */
+/* per-block choice among the E4M3 neighbours of the Eq. 3 scale)          */
+/* ------------------------------------------------------------------------ */
+
+/* Eq. 2 codes of one block for a given block-scale code. */
+static void encode_block(const uint16_t* xb, float alpha, unsigned sigma_code, unsigned char codes16[16])
+{
+    float d = alpha * (float)orc_e4m3_value(sigma_code);
+    float enc = (d == 0.0f) ? 0.0f : 1.0f / d;
+    for (int i = 0; i < 16; ++i) {
+        float v = orc_bf16_to_float(xb[i]);
+        unsigned sign = signbit(v) ? 8u : 0u;
+        float a = fabsf(v);
+        unsigned mag = (a == 0.0f) ? 0u : orc_e2m1_round(a * enc);
+        codes16[i] = (unsigned char)(sign | mag);
+    }
+}
+
+/* Squared error of a coded block, in binary32 and in element order:
+ * y_i = fl(d * v_i) with d = fl(alpha * sigma) and v_i the signed E2M1
+ * value; r_i = fl(x_i - y_i); e = fl(e + fl(r_i * r_i)). */
+static float block_sq_error(const uint16_t* xb, float alpha, unsigned sigma_code, const unsigned char codes16[16])
+{
+    float d = alpha * (float)orc_e4m3_value(sigma_code);
+    float e = 0.0f;
+    for (int i = 0; i < 16; ++i) {
+        float v = (float)orc_e2m1_value(codes16[i]);
+        float y = d * v;
+        float r = orc_bf16_to_float(xb[i]) - y;
+        float rr = r * r;
+        e = e + rr;
+    }
+    return e;
+}
+
+/* Block quantization with scale search: candidates are the Eq. 3 code c0
+ * and its E4M3 neighbours c0 - 1 and c0 + 1 (within 0 .. 0x7E), tried in the
+ * order c0, c0 - 1, c0 + 1; the first candidate with the smallest squared
+ * error (block_sq_error) wins, so ties keep the Eq. 3 scale. */
+static unsigned quantize_block_search(const uint16_t* xb, float alpha, unsigned char codes16[16])
+{
+    unsigned c0 = quantize_block(xb, alpha, codes16);
+    float best = block_sq_error(xb, alpha, c0, codes16);
+    unsigned best_c = c0;
+    unsigned cand[2] = {c0 - 1u, c0 + 1u};
+    int valid[2] = {c0 >= 1u, c0 <= 0x7Du};
+    for (int j = 0; j < 2; ++j) {
+        if (!valid[j]) continue;
+        unsigned char q[16];
+        encode_block(xb, alpha, cand[j], q);
+        float e = block_sq_error(xb, alpha, cand[j], q);
+        if (e < best) {
+            best = e;
+            best_c = cand[j];
+            memcpy(codes16, q, 16);
+        }
+    }
+    return best_c;
+}
+
 /* Quantize rows x[rows][K] (BF16, row-major; K a multiple of 16).
  * codes: [rows][K/2] bytes, element k in byte k/2, even k in the low nibble.
  * scales: [rows][K/16] E4M3 codes, row-major (the plain layout). */
@@ -225,6 +290,23 @@ void orc_quantize_rows(const uint16_t* x, int64_t rows, int64_t K, float alpha,
         for (int64_t b = 0; b < nb; ++b) {
             unsigned char q[16];
             unsigned sc = quantize_block(x + r * K + b * 16, alpha, q);
+            scales[r * nb + b] = (uint8_t)sc;
+            for (int i = 0; i < 16; i += 2)
+                codes[r * (K / 2) + b * 8 + i / 2] = (uint8_t)(q[i] | (q[i + 1] << 4));
+        }
+    }
+}
+
+/* As orc_quantize_rows, with the per-block scale search. */
+void orc_quantize_rows_search(const uint16_t* x, int64_t rows, int64_t K, float alpha,
+                              uint8_t* codes, uint8_t* scales)
+{
+    const int64_t nb = K / 16;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t b = 0; b < nb; ++b) {
+            unsigned char q[16];
+            unsigned sc = quantize_block_search(x + r * K + b * 16, alpha, q);
             scales[r * nb + b] = (uint8_t)sc;
             for (int i = 0; i < 16; i += 2)
                 codes[r * (K / 2) + b * 8 + i / 2] = (uint8_t)(q[i] | (q[i + 1] << 4));

@@ -399,3 +399,58 @@ def test_pins_catch_planted_mistakes(mutation):
         for i, v in enumerate(xf[16:32]):   # block B has alpha = sigma = 1
             planted[16 + i] = (got[16 + i] & 8) | int(np.argmin([abs(p - v) - 1e-9 * p for p in E2M1_POS]))
     assert not np.array_equal(planted, want)
+
+
+# ------------------------------------------------------------------ opt-in scale search
+
+def test_scale_search_handworked_blocks():
+    g = json.load(open(os.path.join(GOLDEN, "scale_search_blocks.json")))
+    for b in g["blocks"]:
+        x = bf16(b["x"]).reshape(1, 16)
+        assert np.array_equal(wl.bf16_bits_to_f32(x).ravel(), np.asarray(b["x"], np.float32)), b["name"]
+        c0, s0 = oracle.quantize(x, g["alpha"])
+        c1, s1 = oracle.quantize(x, g["alpha"], search=True)
+        assert int(s0[0, 0]) == b["sigma_code_rne"], b["name"]
+        assert int(s1[0, 0]) == b["sigma_code_search"], b["name"]
+        got = [(int(c1[0, j // 2]) >> (4 * (j % 2))) & 15 for j in range(16)]
+        assert got == b["codes"], b["name"]
+
+
+def test_scale_search_never_worse_than_eq3_and_stays_next_to_it():
+    """Exact (FP64) block error of the searched scale <= that of the Eq. 3 scale, up to the
+    binary32 rounding of the search metric; the chosen code is c0 - 1, c0 or c0 + 1."""
+    for seed in range(3):
+        x = wl.heavy_tailed_bf16(96, 512, 40 + seed)
+        _, alpha, _ = oracle.tensor_alpha(x)
+        c0, s0 = oracle.quantize(x, alpha)
+        c1, s1 = oracle.quantize(x, alpha, search=True)
+        assert np.all(np.abs(s1.astype(np.int64) - s0.astype(np.int64)) <= 1)
+        xf = wl.bf16_bits_to_f32(x).astype(np.float64)
+        e0 = ((oracle.dequantize(c0, s0, alpha) - xf) ** 2).reshape(96, -1, 16).sum(axis=2)
+        e1 = ((oracle.dequantize(c1, s1, alpha) - xf) ** 2).reshape(96, -1, 16).sum(axis=2)
+        assert np.all(e1 <= e0 * (1 + 2.0 ** -18) + 1e-30)
+        assert e1.sum() < e0.sum()                     # the search does help on heavy-tailed data
+        changed = s1 != s0
+        assert changed.any() and np.all(e1[changed] < e0[changed] * (1 + 2.0 ** -18))
+
+
+def test_scale_search_output_is_on_the_grid_of_its_scale():
+    """With the searched scale the codes are still Eq. 2's nearest grid points (the same invariant
+    as the Eq. 3 path: |x - xhat| <= half the local step unless clipped)."""
+    x = wl.heavy_tailed_bf16(64, 512, 7)
+    _, alpha, _ = oracle.tensor_alpha(x)
+    codes, scales = oracle.quantize(x, alpha, search=True)
+    xhat = oracle.dequantize(codes, scales, alpha)
+    xf = wl.bf16_bits_to_f32(x).astype(np.float64)
+    sig = np.vectorize(oracle.e4m3_value)(scales.astype(np.int64)).repeat(16, axis=1)
+    d = (np.float32(alpha) * sig.astype(np.float32)).astype(np.float64)
+    d_exact = np.float64(np.float32(alpha)) * sig
+    with np.errstate(divide="ignore", invalid="ignore"):
+        v = np.where(d_exact > 0, xhat / np.where(d_exact > 0, d_exact, 1.0), 0.0)
+    assert np.all(np.isin(np.abs(v), E2M1_POS))
+    m = np.where(d > 0, np.abs(xf) / d, 0.0)
+    half = np.where(m <= 2.0, 0.25, np.where(m <= 4.0, 0.5, 1.0))
+    normal = sig >= 2.0 ** -6
+    err = np.abs(xf - xhat)
+    bound = d * half * (1 + 2.0 ** -20) + np.abs(xf) * 2.0 ** -22
+    assert np.all((err <= bound) | ~normal | (m > 6.0))
