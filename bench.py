@@ -388,6 +388,25 @@ def measure_extras(mq, torch, dev, flush, hbm_gbs, fp4_peak, reps=10):
     torch.cuda.synchronize()
     yq, yr = Y[:64].double(), yb.double()
     err = float(torch.linalg.norm(yq - yr) / torch.linalg.norm(yr))
+    # opt-in per-block scale search on the same weight: cost and quantization error
+    def dequant(t):
+        rs = mq.unswizzle_scales(t).to(torch.float32)          # E4M3 codes, row-major [N, K/16]
+        sig = rs.to(torch.uint8).view(torch.float8_e4m3fn).to(torch.float32)
+        c = t.codes.to(torch.int32)
+        nib = torch.stack([c & 15, c >> 4], dim=-1).reshape(t.rows, t.cols)
+        lut = torch.tensor([0, .5, 1, 1.5, 2, 3, 4, 6, -0., -.5, -1, -1.5, -2, -3, -4, -6], device=dev)
+        return lut[nib] * sig.repeat_interleave(16, dim=1) * t.alpha
+    wref = Wm.to(torch.float32)
+    tp = mq.quantize(Wm, ws=ws)
+    tsr = mq.quantize(Wm, scale_search=True, ws=ws)
+    ms_p = _time_calls(torch, lambda: mq.quantize(Wm, out=tp, ws=ws), reps, flush)
+    ms_s = _time_calls(torch, lambda: mq.quantize(Wm, scale_search=True, out=tsr, ws=ws), reps, flush)
+    err_p = float(torch.linalg.norm(dequant(tp) - wref) / torch.linalg.norm(wref))
+    err_s = float(torch.linalg.norm(dequant(tsr) - wref) / torch.linalg.norm(wref))
+    moved = float((mq.unswizzle_scales(tp) != mq.unswizzle_scales(tsr)).float().mean())
+    out["scale_search"] = {"weight": [N, K], "ms_eq3": ms_p, "ms_search": ms_s,
+                           "GB/s_search": (2 + 0.5625) * N * K / (ms_s * 1e-3) / 1e9,
+                           "rel_err_eq3": err_p, "rel_err_search": err_s, "blocks_moved": moved}
     out["phase_aware_pair"] = {
         "weight": [N, K], "decode_bf16": dec,
         "roofline_decode": {"bound": "hbm", "kernel": "decode_bf16_kernel", "unit": "GB/s", "peak": hbm_gbs,

@@ -188,6 +188,26 @@ MQ_API mq_status mq_decode_linear(const void* X_bf16, int64_t M, const void* W_b
 MQ_API mq_status mq_prefill_linear_noalloc(const void* X_bf16, int64_t M, const mq_nvfp4* W,
                                            const float* alpha_static, void* Y_bf16, mq_stream_t stream);
 
+/* Flags of mq_quantize. */
+#define MQ_QUANT_GATE_UP_INTERLEAVE 1u  /* rows = [gate; up], interleaved in 16-row groups (as mq_quantize_weight) */
+#define MQ_QUANT_SCALE_SEARCH 2u        /* per-block scale search (below) */
+
+/* General quantization entry: BF16 [rows, K] -> NVFP4 `out` (Eq. 2, Eq. 3),
+ * tensor scale dynamic (amax/2688, 1 for an all-zero tensor) unless
+ * alpha_static is given (then copied to out->alpha).
+ * MQ_QUANT_SCALE_SEARCH: the paper mentions "scale optimization" once without
+ * defining it; read here as an opt-in per-block search: besides the Eq. 3
+ * scale code c0, its E4M3 neighbours c0 - 1 and c0 + 1 are tried (each with
+ * its Eq. 2 codes) and the one with the smallest squared error
+ * sum_i (x_i - fl(fl(alpha*sigma) * v_i))^2, accumulated in binary32 in
+ * element order, is kept; ties keep c0.  Costs about three times the
+ * quantization arithmetic; meant for the offline weights.
+ * MQ_QUANT_GATE_UP_INTERLEAVE needs rows % 128 == 0.  Other flag bits:
+ * MQ_ERR_INVALID_ARG.  Shapes, alignment, workspace and errors as
+ * mq_quantize_weight. */
+MQ_API mq_status mq_quantize(const void* X_bf16, int64_t rows, int64_t K, const float* alpha_static, unsigned flags,
+                             const mq_nvfp4* out, void* ws, size_t ws_bytes, mq_stream_t stream);
+
 /* Uniform-NVFP4 decode (the decode side of the paper's "uniform NVFP4"
  * comparison, Section 4, whose decode also runs in NVFP4):
  * Y[M,N] = bf16(fl(alpha_x*alpha_w) * sum_k (sigma_x q_x)(sigma_w q_w)), FP32

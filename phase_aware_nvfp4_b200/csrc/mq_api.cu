@@ -154,7 +154,8 @@ mq_status check_ws(void* ws, size_t ws_bytes, size_t need)
 // copy_static, the value is also copied to alpha_out.
 mq_status quantize_into(const void* x, int64_t rows, int64_t K, const float* alpha_static, uint8_t* codes,
                         uint8_t* scales, float* alpha_out, bool copy_static, int64_t interleave_half,
-                        const Ws& w, const DeviceInfo& di, cudaStream_t s, const float** alpha_used)
+                        const Ws& w, const DeviceInfo& di, cudaStream_t s, const float** alpha_used,
+                        bool scale_search = false)
 {
     if (alpha_static != nullptr && copy_static && alpha_out != alpha_static) {
         if (cudaMemcpyAsync(alpha_out, alpha_static, sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
@@ -162,7 +163,7 @@ mq_status quantize_into(const void* x, int64_t rows, int64_t K, const float* alp
     }
     if (alpha_used != nullptr) *alpha_used = (alpha_static != nullptr) ? alpha_static : alpha_out;
     return cuda_status(launch_quantize(x, rows, K, alpha_static, alpha_out, codes, scales, interleave_half, w.ctrl,
-                                       w.partials, di, s));
+                                       w.partials, di, s, scale_search));
 }
 
 }  // namespace
@@ -232,6 +233,26 @@ mq_status mq_quantize_activation(const void* X_bf16, int64_t M, int64_t K, const
     const Ws w = carve(ws, 0, 0);
     return quantize_into(X_bf16, M, K, alpha_static, out->codes, out->scales, out->alpha, true, 0, w, di,
                          reinterpret_cast<cudaStream_t>(stream), nullptr);
+}
+
+mq_status mq_quantize(const void* X_bf16, int64_t rows, int64_t K, const float* alpha_static, unsigned flags,
+                      const mq_nvfp4* out, void* ws, size_t ws_bytes, mq_stream_t stream)
+{
+    if (X_bf16 == nullptr) return MQ_ERR_INVALID_ARG;
+    if ((flags & ~(unsigned)(MQ_QUANT_GATE_UP_INTERLEAVE | MQ_QUANT_SCALE_SEARCH)) != 0) return MQ_ERR_INVALID_ARG;
+    if (rows < 1 || K < 64 || K % 64 != 0) return MQ_ERR_SHAPE;
+    const bool interleave = (flags & MQ_QUANT_GATE_UP_INTERLEAVE) != 0;
+    if (interleave && rows % 128 != 0) return MQ_ERR_SHAPE;
+    if (!aligned16(X_bf16)) return MQ_ERR_ALIGNMENT;
+    mq_status st = check_nvfp4(out, rows, K);
+    if (st != MQ_OK) return st;
+    if ((st = check_ws(ws, ws_bytes, kWsControlBytes)) != MQ_OK) return st;
+    DeviceInfo di;
+    if ((st = check_device(&di)) != MQ_OK) return st;
+    const Ws w = carve(ws, 0, 0);
+    return quantize_into(X_bf16, rows, K, alpha_static, out->codes, out->scales, out->alpha, true,
+                         interleave ? rows / 2 : 0, w, di, reinterpret_cast<cudaStream_t>(stream), nullptr,
+                         (flags & MQ_QUANT_SCALE_SEARCH) != 0);
 }
 
 mq_status mq_prefill_linear(const void* X_bf16, const mq_nvfp4* X_q, int64_t M, const mq_nvfp4* W, mq_epilogue epi,

@@ -68,9 +68,11 @@ cudaError_t launch_amax(const void* x, int64_t n, float* alpha_out, WsControl* c
 // cooperative launch of the quantization kernel.  interleave_half > 0
 // interleaves gate/up rows in 16-row groups (output row 32c+t <- input row
 // 16c+t for t<16, I+16c+t-16 else).
+// scale_search: per block, also try the E4M3 neighbours of the Eq. 3 scale
+// and keep the smallest binary32 squared error (ties keep the Eq. 3 scale).
 cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float* alpha_static, float* alpha_out,
                             uint8_t* codes, uint8_t* scales, int64_t interleave_half, WsControl* ctrl,
-                            uint32_t* partials, const DeviceInfo& di, cudaStream_t s);
+                            uint32_t* partials, const DeviceInfo& di, cudaStream_t s, bool scale_search = false);
 
 // Sweep of the E2M1 conversion instruction against the definition; adds
 // mismatch counts for positive / negative inputs into counts[0] / counts[1].

@@ -179,7 +179,7 @@ struct QuantConsts {
 // Fills enc_tab[c] = fl(1 / fl(alpha * sigma_c)) for every E4M3 code c (0 when
 // the product is 0) and returns the block-scale constants.  Every thread of
 // the block calls it; it ends with __syncthreads().
-__device__ __forceinline__ QuantConsts quant_setup(float alpha, float* enc_tab)
+__device__ __forceinline__ QuantConsts quant_setup(float alpha, float* enc_tab, float* dec_tab)
 {
     QuantConsts q;
     q.alpha_qmax = __fmul_rn(alpha, 6.0f);
@@ -192,6 +192,7 @@ __device__ __forceinline__ QuantConsts quant_setup(float alpha, float* enc_tab)
     if (threadIdx.x < 128) {
         const float d = __fmul_rn(alpha, e4m3_to_float((uint32_t)threadIdx.x));
         enc_tab[threadIdx.x] = (d == 0.0f) ? 0.0f : __frcp_rn(d);
+        dec_tab[threadIdx.x] = d;
     }
     __syncthreads();
     return q;
@@ -267,13 +268,42 @@ __device__ __noinline__ uint32_t amax_tile_finite(const uint16_t* __restrict__ x
     return mx;
 }
 
+// Squared error of one coded 16-element block in binary32, element order
+// 0..15: y = fl(d * v) with v the signed E2M1 value of the code, r = fl(x - y),
+// e = fl(e + fl(r * r)).  Codes: nibble j of c0 / c1 is element j / 8 + j.
+__device__ __forceinline__ float block_sq_error(const float (&f0)[8], const float (&f1)[8], uint32_t c0, uint32_t c1,
+                                                float d)
+{
+    // E2M1 magnitude index -> 2 x value {0, 1, 2, 3, 4, 6, 8, 12}, one nibble each
+    constexpr uint32_t kTwiceValue = 0xC8643210u;
+    float e = 0.0f;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const uint32_t c = h ? c1 : c0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const uint32_t nib = (c >> (4 * j)) & 15u;
+            const float mag = (float)((kTwiceValue >> (4 * (nib & 7u))) & 15u) * 0.5f;   // exact
+            const float v = (nib & 8u) ? -mag : mag;
+            const float y = __fmul_rn(d, v);
+            const float r = __fsub_rn(h ? f1[j] : f0[j], y);
+            e = __fadd_rn(e, __fmul_rn(r, r));
+        }
+    }
+    return e;
+}
+
 // Eq. 3 / Eq. 2 for one tile; scales staged in shared memory and written as
 // one contiguous 2 KiB run of the MMA scale layout.
+// With `search`, each block also tries the E4M3 neighbours of its Eq. 3 scale
+// code (c0 - 1, then c0 + 1) and keeps the first with the smallest squared
+// error, so ties keep the Eq. 3 scale.
+template <bool SEARCH>
 __device__ __forceinline__ void quant_tile(const uint16_t* __restrict__ x, int64_t rows, int64_t K,
                                            int64_t interleave_half, int64_t rb, int64_t kc, int64_t chunks,
-                                           const QuantConsts& qc, const float* enc_tab, uint8_t* sf_stage,
-                                           uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, int warp,
-                                           int half, int blk)
+                                           const QuantConsts& qc, const float* enc_tab, const float* dec_tab,
+                                           uint8_t* sf_stage, uint8_t* __restrict__ codes,
+                                           uint8_t* __restrict__ scales, int warp, int half, int blk)
 {
     const int64_t col = kc * 256 + 16 * blk;
     const bool col_ok = col < K;
@@ -298,7 +328,7 @@ __device__ __forceinline__ void quant_tile(const uint16_t* __restrict__ x, int64
                                    v[u][1].x, v[u][1].y, v[u][1].z, v[u][1].w};
             // Eq. 3: sigma_b = Pi_E4M3(amax_b / (alpha * q_max))
             const float amax = bf16x16_absmax(w);
-            const uint32_t sc = e4m3_block_scale(amax, qc.alpha_qmax, qc.inv_lo, qc.inv_hi);
+            uint32_t sc = e4m3_block_scale(amax, qc.alpha_qmax, qc.inv_lo, qc.inv_hi);
             // Eq. 2: q_i = Pi_FP4(x_i / (alpha * sigma_b)), as x * fl(1/fl(alpha*sigma))
             const float enc = enc_tab[sc];
             float f0[8], f1[8];
@@ -309,8 +339,27 @@ __device__ __forceinline__ void quant_tile(const uint16_t* __restrict__ x, int64
                 f1[2 * j] = bf16_lo(w[4 + j]);
                 f1[2 * j + 1] = bf16_hi(w[4 + j]);
             }
-            const uint32_t c0 = e2m1x8_encode(f0, enc);
-            const uint32_t c1 = e2m1x8_encode(f1, enc);
+            uint32_t c0 = e2m1x8_encode(f0, enc);
+            uint32_t c1 = e2m1x8_encode(f1, enc);
+            if (SEARCH) {
+                float best = block_sq_error(f0, f1, c0, c1, dec_tab[sc]);
+                const uint32_t base = sc;
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    if (t == 0 ? base < 1u : base > 0x7Du) continue;
+                    const uint32_t cand = t == 0 ? base - 1u : base + 1u;
+                    const float ec = enc_tab[cand];
+                    const uint32_t q0 = e2m1x8_encode(f0, ec);
+                    const uint32_t q1 = e2m1x8_encode(f1, ec);
+                    const float err = block_sq_error(f0, f1, q0, q1, dec_tab[cand]);
+                    if (err < best) {
+                        best = err;
+                        sc = cand;
+                        c0 = q0;
+                        c1 = q1;
+                    }
+                }
+            }
             const bool ok = (r < rows) && col_ok;
             if (ok) *reinterpret_cast<uint2*>(codes + r * (K / 2) + col / 2) = make_uint2(c0, c1);
             sf_stage[(blk >> 2) * 512 + (rl & 31) * 16 + (rl >> 5) * 4 + (blk & 3)] = ok ? (uint8_t)sc : 0;
@@ -352,6 +401,7 @@ __device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v)
 //     (bounded; a wait that runs out posts kErrTimeout and the block stops).
 //     The quantization pass then walks the tiles in the opposite order, so
 //     the lines read last by the amax pass, still in L2, are read first.
+template <bool SEARCH>
 __global__ void __launch_bounds__(kQuantThreads, MQ_QUANT_MIN_BLOCKS)
     quantize_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t K, const float* __restrict__ alpha_static,
                     float* __restrict__ alpha_out, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
@@ -359,6 +409,7 @@ __global__ void __launch_bounds__(kQuantThreads, MQ_QUANT_MIN_BLOCKS)
 {
     __shared__ __align__(16) uint8_t sf_stage[2048];
     __shared__ float enc_tab[128];
+    __shared__ float dec_tab[128];   // fl(alpha * sigma) for every E4M3 code sigma
     __shared__ uint32_t s_red[kQuantThreads / 32];
     __shared__ uint32_t s_epoch, s_last, s_ok;
     __shared__ float s_alpha;
@@ -443,24 +494,26 @@ __global__ void __launch_bounds__(kQuantThreads, MQ_QUANT_MIN_BLOCKS)
         if (!s_ok) return;
         alpha = s_alpha;
     }
-    const QuantConsts qc = quant_setup(alpha, enc_tab);
+    const QuantConsts qc = quant_setup(alpha, enc_tab, dec_tab);
     // ---- pass 2: quantize, tiles in reverse order of pass 1
     for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
         const int64_t tile = tiles - 1 - t;
-        quant_tile(x, rows, K, interleave_half, tile / chunks, tile % chunks, chunks, qc, enc_tab, sf_stage, codes,
-                   scales, warp, half, blk);
+        quant_tile<SEARCH>(x, rows, K, interleave_half, tile / chunks, tile % chunks, chunks, qc, enc_tab, dec_tab,
+                           sf_stage, codes, scales, warp, half, blk);
     }
 }
 
-// Resident blocks per SM of quantize_kernel (cached per device).
-static int quantize_blocks_per_sm(const DeviceInfo& di)
+// Resident blocks per SM of quantize_kernel<SEARCH> (cached per device).
+template <bool SEARCH>
+int quantize_blocks_per_sm(const DeviceInfo& di)
 {
     static std::mutex mu;
     static int per_sm[64] = {};
     std::lock_guard<std::mutex> lock(mu);
     if (di.device >= 0 && di.device < 64 && per_sm[di.device] > 0) return per_sm[di.device];
     int occ = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quantize_kernel, kQuantThreads, 0) != cudaSuccess) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quantize_kernel<SEARCH>, kQuantThreads, 0) !=
+        cudaSuccess) {
         (void)cudaGetLastError();
         occ = 0;
     }
@@ -470,10 +523,10 @@ static int quantize_blocks_per_sm(const DeviceInfo& di)
 
 cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float* alpha_static, float* alpha_out,
                             uint8_t* codes, uint8_t* scales, int64_t interleave_half, WsControl* ctrl,
-                            uint32_t* partials, const DeviceInfo& di, cudaStream_t s)
+                            uint32_t* partials, const DeviceInfo& di, cudaStream_t s, bool scale_search)
 {
     const int64_t tiles = ((rows + 127) / 128) * ((K + 255) / 256);
-    const int occ = quantize_blocks_per_sm(di);
+    const int occ = scale_search ? quantize_blocks_per_sm<true>(di) : quantize_blocks_per_sm<false>(di);
     const int64_t resident = (int64_t)di.num_sms * std::max(1, occ);
     // Small tensors (at most one tile per SM): one cooperative launch takes
     // the amax, hands alpha to every block and quantizes; the two-kernel path
@@ -500,8 +553,9 @@ cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float*
     attr[0].val.cooperative = single ? 1 : 0;   // blocks wait on one another only in the single-launch amax
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, quantize_kernel, static_cast<const uint16_t*>(x), rows, K, alpha_in,
-                                       alpha_out, codes, scales, interleave_half, ctrl, partials);
+    auto kern = scale_search ? quantize_kernel<true> : quantize_kernel<false>;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, static_cast<const uint16_t*>(x), rows, K, alpha_in, alpha_out,
+                                       codes, scales, interleave_half, ctrl, partials);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

@@ -33,7 +33,7 @@ STATUS_NAMES = {0: "MQ_OK", 1: "MQ_ERR_INVALID_ARG", 2: "MQ_ERR_SHAPE", 3: "MQ_E
 EXPORTS = ("mq_status_string", "mq_version", "mq_nvfp4_sizes", "mq_workspace_bytes", "mq_quantize_weight",
            "mq_quantize_activation", "mq_prefill_linear", "mq_decode_linear", "mq_unswizzle_scales",
            "mq_async_status", "mq_prefill_linear_noalloc", "mq_selftest_e2m1", "mq_selftest_timeout",
-           "mq_decode_linear_nvfp4")
+           "mq_decode_linear_nvfp4", "mq_quantize")
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
@@ -89,6 +89,8 @@ def load(path: str = LIB_PATH):
             lib.mq_selftest_timeout.restype = i32
             lib.mq_decode_linear_nvfp4.argtypes = [vp, i64, nvp, vp, vp, vp, sz, vp]
             lib.mq_decode_linear_nvfp4.restype = i32
+            lib.mq_quantize.argtypes = [vp, i64, i64, vp, ctypes.c_uint, nvp, vp, sz, vp]
+            lib.mq_quantize.restype = i32
             lib.mq_prefill_linear_noalloc.argtypes = [vp, i64, nvp, vp, vp, vp]
             lib.mq_prefill_linear_noalloc.restype = i32
             _lib = lib
@@ -171,6 +173,23 @@ def quantize_weight(W, gate_up_interleave: bool = False, out: NVFP4Tensor | None
     cs = out.c()
     _check(load().mq_quantize_weight(_ptr(W), N, K, int(bool(gate_up_interleave)), ctypes.byref(cs),
                                      *_ws_args(ws), _stream(stream)), "mq_quantize_weight")
+    return out
+
+
+MQ_QUANT_GATE_UP_INTERLEAVE = 1
+MQ_QUANT_SCALE_SEARCH = 2
+
+
+def quantize(X, alpha_static=None, gate_up_interleave: bool = False, scale_search: bool = False,
+             out: NVFP4Tensor | None = None, ws=None, stream=None) -> NVFP4Tensor:
+    """mq_quantize: BF16 [rows, K] -> NVFP4, optionally with the per-block scale search."""
+    rows, K = X.shape
+    out = out or nvfp4_empty(rows, K, X.device)
+    ws = ws if ws is not None else workspace(device=X.device)
+    flags = (MQ_QUANT_GATE_UP_INTERLEAVE if gate_up_interleave else 0) | (MQ_QUANT_SCALE_SEARCH if scale_search else 0)
+    oc = out.c()
+    _check(load().mq_quantize(_ptr(X), rows, K, _ptr(alpha_static), flags, ctypes.byref(oc), *_ws_args(ws),
+                              _stream(stream)), "mq_quantize")
     return out
 
 

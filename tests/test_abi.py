@@ -103,6 +103,11 @@ def test_argument_errors_are_synchronous(lib):
     assert lib.mq_quantize_weight(P, 200, 256, 1, ctypes.byref(out), ws, wsb, None) == 2
     assert lib.mq_quantize_weight(P, 200, 256, 0, None, ws, wsb, None) == 1
     assert lib.mq_async_status(None, None) == 1
+    # general quantization entry: unknown flag bits, interleave needs rows % 128
+    q = _nv(200, 256)
+    assert lib.mq_quantize(P, 200, 256, None, ctypes.c_uint(4), ctypes.byref(q), ws, wsb, None) == 1
+    assert lib.mq_quantize(P, 200, 256, None, ctypes.c_uint(1), ctypes.byref(q), ws, wsb, None) == 2
+    assert lib.mq_quantize(P + 2, 200, 256, None, ctypes.c_uint(2), ctypes.byref(q), ws, wsb, None) == 3
     # timeout self-test: timeout in (0, 2 s], a workspace, an aligned result slot
     assert lib.mq_selftest_timeout(ws, wsb, ctypes.c_uint64(0), None, None) == 1
     assert lib.mq_selftest_timeout(ws, wsb, ctypes.c_uint64(3 * 10 ** 9), None, None) == 1

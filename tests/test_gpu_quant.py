@@ -152,6 +152,67 @@ def test_weight_quantization_and_gate_up_interleave():
     assert np.array_equal(codes, rc[perm]) and np.array_equal(scales, rs[perm])
 
 
+@pytest.mark.parametrize("rows,K,kind", [(128, 256, "heavy"), (200, 1088, "heavy"), (1, 64, "heavy"),
+                                         (512, 4096, "weights"), (2048, 12288, "heavy")])
+def test_scale_search_bit_exact(rows, K, kind):
+    """Opt-in per-block scale search: codes, scales and alpha bit-exact against the oracle's
+    search (same binary32 error arithmetic, same tie rule); small inputs take the single-launch
+    path, the largest the amax-kernel path."""
+    x = wl.normal_bf16(rows, K, 0.02, 91) if kind == "weights" else wl.heavy_tailed_bf16(rows, K, 93)
+    t = mq.quantize(to_dev(x), scale_search=True)
+    torch.cuda.synchronize()
+    codes, scales, alpha = nvfp4_host(t)
+    _, a_ref, _ = oracle.tensor_alpha(x)
+    assert np.float32(alpha) == np.float32(a_ref)
+    rc, rs = oracle.quantize(x, a_ref, search=True)
+    assert np.array_equal(scales, rs), f"{int((scales != rs).sum())} scale mismatches"
+    assert np.array_equal(codes, rc), f"{int((codes != rc).sum())} code byte mismatches"
+    plain_c, plain_s = oracle.quantize(x, a_ref)
+    print(f"scale search {rows}x{K}: {100.0 * float((rs != plain_s).mean()):.1f} % of blocks moved")
+
+
+def test_scale_search_golden_blocks_static_alpha_and_interleave():
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "scale_search_blocks.json")))
+    x = np.concatenate([wl.f32_to_bf16_bits(np.asarray(b["x"], np.float32)) for b in g["blocks"]])[None, :]
+    x = np.concatenate([x, np.zeros((1, 64 - x.shape[1] % 64 if x.shape[1] % 64 else 0), np.uint16)], axis=1)
+    t = mq.quantize(to_dev(x), alpha_static=torch.ones(1, device="cuda"), scale_search=True)
+    torch.cuda.synchronize()
+    codes, scales, alpha = nvfp4_host(t)
+    assert alpha == 1.0
+    for i, b in enumerate(g["blocks"]):
+        assert scales[0, i] == b["sigma_code_search"], b["name"]
+        got = [(int(codes[0, 8 * i + j // 2]) >> (4 * (j % 2))) & 15 for j in range(16)]
+        assert got == b["codes"], b["name"]
+    # gate/up interleave with the search
+    I, K = 128, 512
+    w = wl.normal_bf16(2 * I, K, 0.02, 78)
+    inter = mq.quantize(to_dev(w), gate_up_interleave=True, scale_search=True)
+    perm = np.empty(2 * I, np.int64)
+    for r in range(2 * I):
+        c, t_ = divmod(r, 32)
+        perm[r] = 16 * c + t_ if t_ < 16 else I + 16 * c + (t_ - 16)
+    codes, scales, alpha = nvfp4_host(inter)
+    _, a_ref, _ = oracle.tensor_alpha(w)
+    rc, rs = oracle.quantize(w, a_ref, search=True)
+    assert np.array_equal(codes, rc[perm]) and np.array_equal(scales, rs[perm])
+
+
+def test_gemm_with_searched_weights_matches_oracle():
+    """The GEMM consumes searched scales like any others: parity against the oracle's
+    block-scaled matmul on the searched weight."""
+    from gpu_helpers import gemm_check
+    x = wl.heavy_tailed_bf16(256, 1024, 95)
+    w = wl.normal_bf16(512, 1024, 0.02, 96)
+    Wq = mq.quantize(to_dev(w), scale_search=True)
+    y = mq.prefill_linear(to_dev(x), Wq)
+    torch.cuda.synchronize()
+    ax = oracle.tensor_alpha(x)[1]
+    aw = oracle.tensor_alpha(w)[1]
+    y64, sabs = oracle.nvfp4_linear_rows((*oracle.quantize(x, ax), ax), (*oracle.quantize(w, aw, search=True), aw))
+    from gpu_helpers import to_host_bits
+    gemm_check(to_host_bits(y), y64, sabs)
+
+
 def test_unswizzle_matches_layout_mapping_and_padding_is_zero():
     x = wl.heavy_tailed_bf16(200, 320, 9)
     t = mq.quantize_activation(to_dev(x))
