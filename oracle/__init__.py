@@ -83,6 +83,9 @@ def _L():
             lib.orc_quantize_rows.restype = None
             lib.orc_quantize_rows_search.argtypes = [u16p, i64, i64, ctypes.c_float, u8p, u8p]
             lib.orc_quantize_rows_search.restype = None
+            lib.orc_rmsnorm_rows.argtypes = [u16p, i64, i64, u16p, ctypes.c_float, u16p,
+                                             ctypes.POINTER(ctypes.c_float)]
+            lib.orc_rmsnorm_rows.restype = None
             lib.orc_dequantize_rows.argtypes = [u8p, u8p, i64, i64, ctypes.c_float, f64p]
             lib.orc_dequantize_rows.restype = None
             lib.orc_round_bf16.argtypes = [f64p, i64, u16p]
@@ -171,6 +174,24 @@ def quantize(x_bf16: np.ndarray, alpha: float, search: bool = False):
     fn(_ptr(x, ctypes.c_uint16), rows, K, ctypes.c_float(alpha), _ptr(codes, ctypes.c_uint8),
        _ptr(scales, ctypes.c_uint8))
     return codes, scales
+
+
+def rmsnorm(x_bf16: np.ndarray, gamma_bf16: np.ndarray, eps: float):
+    """RMSNorm rows of BF16 x with BF16 weight gamma -> (h BF16 bits [rows, K], rstd float32 [rows]).
+
+    ms = fl32(sum x^2 (binary64) / K), rstd = fl32(1 / sqrt(ms + eps)) (binary64, one rounding),
+    h = bf16(fl32(fl32(x * rstd) * gamma)): the BF16 tensor an unfused norm would hand to the
+    quantizer of the next linear layer.
+    """
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    g = np.ascontiguousarray(gamma_bf16, dtype=np.uint16).ravel()
+    rows, K = x.shape
+    assert g.shape == (K,)
+    h = np.empty_like(x)
+    r = np.empty(rows, dtype=np.float32)
+    _L().orc_rmsnorm_rows(_ptr(x, ctypes.c_uint16), rows, K, _ptr(g, ctypes.c_uint16), ctypes.c_float(eps),
+                          _ptr(h, ctypes.c_uint16), r.ctypes.data_as(ctypes.POINTER(ctypes.c_float)))
+    return h, r
 
 
 def dequantize(codes: np.ndarray, scales: np.ndarray, alpha: float) -> np.ndarray:

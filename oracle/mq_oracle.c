@@ -314,6 +314,36 @@ void orc_quantize_rows_search(const uint16_t* x, int64_t rows, int64_t K, float 
     }
 }
 
+/* ------------------------------------------------------------------------ */
+/* RMSNorm producing the tensor that the prefill linear quantizes           */
+/* ------------------------------------------------------------------------ */
+
+/* h[r][k] = bf16( fl32( fl32(x[r][k] * rstd_r) * gamma[k] ) ) with
+ *   ms_r   = fl32( (sum_k x^2, in binary64, k ascending) / K ),
+ *   rstd_r = fl32( 1 / sqrt( (double)ms_r + (double)eps ) )  (binary64, one rounding).
+ * x, gamma, h: BF16 bit patterns; rstd (optional): the per-row FP32 factors. */
+void orc_rmsnorm_rows(const uint16_t* x, int64_t rows, int64_t K, const uint16_t* gamma, float eps,
+                      uint16_t* h, float* rstd)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        const uint16_t* xr = x + r * K;
+        double ss = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            double v = (double)orc_bf16_to_float(xr[k]);
+            ss += v * v;
+        }
+        float ms = (float)(ss / (double)K);
+        float rs = (float)(1.0 / sqrt((double)ms + (double)eps));
+        if (rstd) rstd[r] = rs;
+        for (int64_t k = 0; k < K; ++k) {
+            float t = orc_bf16_to_float(xr[k]) * rs;
+            float u = t * orc_bf16_to_float(gamma[k]);
+            h[r * K + k] = orc_double_to_bf16((double)u);
+        }
+    }
+}
+
 /* Dequantize (Eq. 2 right-hand side): xhat = alpha * sigma_b * q_i, in
  * binary64.  With alpha = 1 this gives sigma_b * q_i, the operand the
  * block-scaled matmul multiplies before the tensor scales are applied. */

@@ -454,3 +454,35 @@ def test_scale_search_output_is_on_the_grid_of_its_scale():
     err = np.abs(xf - xhat)
     bound = d * half * (1 + 2.0 ** -20) + np.abs(xf) * 2.0 ** -22
     assert np.all((err <= bound) | ~normal | (m > 6.0))
+
+
+# ------------------------------------------------------------------ RMSNorm feeding the quantizer
+
+def test_rmsnorm_matches_torch_within_one_bf16_ulp():
+    x = wl.heavy_tailed_bf16(64, 1024, 51)
+    g = wl.normal_bf16(1, 1024, 1.0, 52)[0]
+    h, rstd = oracle.rmsnorm(x, g, 1e-6)
+    xf = torch.from_numpy(wl.bf16_bits_to_f32(x).astype(np.float64))
+    gf = torch.from_numpy(wl.bf16_bits_to_f32(g).astype(np.float64))
+    ref = torch.nn.functional.rms_norm(xf, (1024,), weight=gf, eps=1e-6).numpy()
+    ref_bf = oracle.bf16_to_f64(oracle.round_bf16(ref))
+    mine = oracle.bf16_to_f64(h)
+    ulp = oracle.bf16_ulp(ref_bf)
+    assert np.all(np.abs(mine - ref_bf) <= ulp)
+    assert np.mean(mine == ref_bf) > 0.99
+    r64 = 1.0 / np.sqrt((xf.numpy() ** 2).mean(axis=1) + 1e-6)
+    assert np.allclose(rstd, r64, rtol=2.0 ** -22, atol=0)
+
+
+def test_rmsnorm_closed_forms():
+    g = wl.normal_bf16(1, 256, 1.0, 53)[0]
+    # constant rows of 2 (eps 0): ms = 4, rstd = 0.5 exactly, h = gamma exactly
+    x = wl.f32_to_bf16_bits(np.full((2, 256), 2.0, np.float32))
+    h, r = oracle.rmsnorm(x, g, 0.0)
+    assert np.all(r == 0.5) and np.array_equal(h[0], g) and np.array_equal(h[1], g)
+    # +-3 rows: ms = 9, rstd = fl32(1/3), fl32(3 * fl32(1/3)) = 1, so h = +-gamma exactly
+    x = wl.f32_to_bf16_bits(np.tile(np.array([3.0, -3.0], np.float32), 128)[None, :])
+    h, r = oracle.rmsnorm(x, g, 0.0)
+    assert r[0] == np.float32(1.0 / 3.0)
+    sign = np.tile(np.array([0, 0x8000], np.uint16), 128)
+    assert np.array_equal(h[0], g ^ sign)
