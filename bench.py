@@ -407,6 +407,23 @@ def measure_extras(mq, torch, dev, flush, hbm_gbs, fp4_peak, reps=10):
     out["scale_search"] = {"weight": [N, K], "ms_eq3": ms_p, "ms_search": ms_s,
                            "GB/s_search": (2 + 0.5625) * N * K / (ms_s * 1e-3) / 1e9,
                            "rel_err_eq3": err_p, "rel_err_search": err_s, "blocks_moved": moved}
+    # RMSNorm -> NVFP4 fused (the producer of the q/k/v input) vs the unfused pair
+    Mr = 8192
+    Xr = _to_dev(torch, wl.heavy_tailed_bf16(Mr, K, 61), dev)
+    gam = _to_dev(torch, wl.normal_bf16(1, K, 1.0, 62)[0], dev)
+    wsr = mq.workspace(Mr, K, device=dev)
+    tr = mq.rmsnorm_quantize(Xr, gam, 1e-6, ws=wsr)
+    tu = mq.nvfp4_empty(Mr, K, dev)
+
+    def unfused():   # torch's norm writes BF16 h, then the quantizer reads it (amax + quantize)
+        h = torch.nn.functional.rms_norm(Xr, (K,), weight=gam, eps=1e-6)
+        mq.quantize_activation(h, out=tu, ws=wsr)
+    ms_f = _time_calls(torch, lambda: mq.rmsnorm_quantize(Xr, gam, 1e-6, out=tr, ws=wsr), reps, flush)
+    ms_u = _time_calls(torch, unfused, reps, flush)
+    gbs_f = (2 + 2 + 0.5625) * Mr * K / (ms_f * 1e-3) / 1e9
+    out["rmsnorm_quantize"] = {"M": Mr, "K": K, "ms_fused": ms_f, "ms_unfused_torch_norm": ms_u,
+                               "GB/s_fused": gbs_f, "frac_fused": gbs_f / hbm_gbs, "speedup": ms_u / ms_f}
+    del Xr
     out["phase_aware_pair"] = {
         "weight": [N, K], "decode_bf16": dec,
         "roofline_decode": {"bound": "hbm", "kernel": "decode_bf16_kernel", "unit": "GB/s", "peak": hbm_gbs,

@@ -208,6 +208,24 @@ MQ_API mq_status mq_prefill_linear_noalloc(const void* X_bf16, int64_t M, const 
 MQ_API mq_status mq_quantize(const void* X_bf16, int64_t rows, int64_t K, const float* alpha_static, unsigned flags,
                              const mq_nvfp4* out, void* ws, size_t ws_bytes, mq_stream_t stream);
 
+/* RMSNorm fused with the quantization of its output: the NVFP4 copy of
+ *   h[m][k] = bf16( fl32( fl32(x[m][k] * rstd_m) * gamma[k] ) ),
+ *   ms_m = fl32( sum_k x^2 (binary64) / K ), rstd_m = fl32( 1/sqrt(ms_m + eps) ),
+ * with a dynamic tensor scale over h (alpha_h = amax|h| / 2688, 1 if 0) and
+ * Eq. 2 / Eq. 3 as mq_quantize_activation -- the same codes and scales as an
+ * unfused RMSNorm writing BF16 h followed by mq_quantize_activation(h), with
+ * h never written to memory (two reads of X instead of a write and three
+ * reads of h).  This puts the activation quantization inside the producer of
+ * the prefill linear's input (the pages give no fused design; RMSNorm is the
+ * pre-projection norm of the Qwen3 layers they evaluate).
+ * X [M, K] BF16, gamma [K] BF16, both 16-byte aligned; eps finite >= 0;
+ * K % 64 == 0.  h_debug: optional BF16 [M, K] output of h (testing).
+ * Workspace: mq_workspace_bytes(M, K) (it also holds the M per-row factors).
+ * Errors as mq_quantize_activation (NaN/Inf in h -> MQ_ERR_NONFINITE). */
+MQ_API mq_status mq_rmsnorm_quantize(const void* X_bf16, int64_t M, int64_t K, const void* gamma_bf16, float eps,
+                                     const mq_nvfp4* out, void* h_debug, void* ws, size_t ws_bytes,
+                                     mq_stream_t stream);
+
 /* Uniform-NVFP4 decode (the decode side of the paper's "uniform NVFP4"
  * comparison, Section 4, whose decode also runs in NVFP4):
  * Y[M,N] = bf16(fl(alpha_x*alpha_w) * sum_k (sigma_x q_x)(sigma_w q_w)), FP32

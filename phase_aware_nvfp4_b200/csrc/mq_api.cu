@@ -255,6 +255,26 @@ mq_status mq_quantize(const void* X_bf16, int64_t rows, int64_t K, const float* 
                          (flags & MQ_QUANT_SCALE_SEARCH) != 0);
 }
 
+mq_status mq_rmsnorm_quantize(const void* X_bf16, int64_t M, int64_t K, const void* gamma_bf16, float eps,
+                              const mq_nvfp4* out, void* h_debug, void* ws, size_t ws_bytes, mq_stream_t stream)
+{
+    if (X_bf16 == nullptr || gamma_bf16 == nullptr) return MQ_ERR_INVALID_ARG;
+    if (!(eps >= 0.0f) || eps > 3.0e38f) return MQ_ERR_INVALID_ARG;
+    if (M < 1 || M > (int64_t)1 << 30 || K < 64 || K % 64 != 0 || K > (int64_t)1 << 30) return MQ_ERR_SHAPE;
+    if (!aligned16(X_bf16) || !aligned16(gamma_bf16) || (h_debug != nullptr && !aligned16(h_debug)))
+        return MQ_ERR_ALIGNMENT;
+    mq_status st = check_nvfp4(out, M, K);
+    if (st != MQ_OK) return st;
+    if ((st = check_ws(ws, ws_bytes, ws_bytes_for(M, K))) != MQ_OK) return st;
+    DeviceInfo di;
+    if ((st = check_device(&di)) != MQ_OK) return st;
+    const Ws w = carve(ws, M, K);
+    float* rstd = reinterpret_cast<float*>(w.xq_codes);   // M floats; the NVFP4 scratch is not used here
+    return cuda_status(launch_rmsnorm_quantize(X_bf16, M, K, gamma_bf16, eps, rstd, out->codes, out->scales,
+                                               out->alpha, h_debug, w.ctrl, w.partials, di,
+                                               reinterpret_cast<cudaStream_t>(stream)));
+}
+
 mq_status mq_prefill_linear(const void* X_bf16, const mq_nvfp4* X_q, int64_t M, const mq_nvfp4* W, mq_epilogue epi,
                             const float* alpha_static, const float* alpha_h, void* Y, const mq_nvfp4* H_out,
                             void* h_debug, void* ws, size_t ws_bytes, mq_stream_t stream)

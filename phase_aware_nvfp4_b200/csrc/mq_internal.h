@@ -74,6 +74,13 @@ cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float*
                             uint8_t* codes, uint8_t* scales, int64_t interleave_half, WsControl* ctrl,
                             uint32_t* partials, const DeviceInfo& di, cudaStream_t s, bool scale_search = false);
 
+// RMSNorm of X [rows, K] (gamma [K], eps) fused with the NVFP4 quantization of
+// its BF16 output h: rstd per row to `rstd`, alpha_h to *alpha_out, codes and
+// scales of h; h itself to h_out when not null.
+cudaError_t launch_rmsnorm_quantize(const void* x, int64_t rows, int64_t K, const void* gamma, float eps,
+                                    float* rstd, uint8_t* codes, uint8_t* scales, float* alpha_out, void* h_out,
+                                    WsControl* ctrl, uint32_t* partials, const DeviceInfo& di, cudaStream_t s);
+
 // Sweep of the E2M1 conversion instruction against the definition; adds
 // mismatch counts for positive / negative inputs into counts[0] / counts[1].
 cudaError_t launch_selftest_e2m1(unsigned long long* counts, const DeviceInfo& di, cudaStream_t s);

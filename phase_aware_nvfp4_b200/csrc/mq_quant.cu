@@ -298,12 +298,30 @@ __device__ __forceinline__ float block_sq_error(const float (&f0)[8], const floa
 // With `search`, each block also tries the E4M3 neighbours of its Eq. 3 scale
 // code (c0 - 1, then c0 + 1) and keeps the first with the smallest squared
 // error, so ties keep the Eq. 3 scale.
-template <bool SEARCH>
+// With NORM the loaded x are first replaced by h = bf16(fl(fl(x * rstd_row) *
+// gamma_k)) (RMSNorm; rstd from rmsnorm_amax_kernel), optionally written to
+// h_out, and h is quantized.
+struct NormArgs {
+    const uint16_t* gamma;   // [K] BF16
+    const float* rstd;       // [rows]
+    uint16_t* h_out;         // optional [rows, K] BF16
+};
+
+__device__ __forceinline__ uint32_t norm_pair(uint32_t xw, uint32_t gw, float r)
+{
+    const float lo = __fmul_rn(__fmul_rn(bf16_lo(xw), r), bf16_lo(gw));
+    const float hi = __fmul_rn(__fmul_rn(bf16_hi(xw), r), bf16_hi(gw));
+    const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&p);
+}
+
+template <bool SEARCH, bool NORM>
 __device__ __forceinline__ void quant_tile(const uint16_t* __restrict__ x, int64_t rows, int64_t K,
                                            int64_t interleave_half, int64_t rb, int64_t kc, int64_t chunks,
                                            const QuantConsts& qc, const float* enc_tab, const float* dec_tab,
                                            uint8_t* sf_stage, uint8_t* __restrict__ codes,
-                                           uint8_t* __restrict__ scales, int warp, int half, int blk)
+                                           uint8_t* __restrict__ scales, int warp, int half, int blk,
+                                           const NormArgs& na)
 {
     const int64_t col = kc * 256 + 16 * blk;
     const bool col_ok = col < K;
@@ -324,8 +342,21 @@ __device__ __forceinline__ void quant_tile(const uint16_t* __restrict__ x, int64
         for (int u = 0; u < kQuantStepUnroll; ++u) {
             const int rl = 16 * warp + 2 * (s0 + u) + half;   // row within the 128-row block
             const int64_t r = rb * 128 + rl;
-            const uint32_t w[8] = {v[u][0].x, v[u][0].y, v[u][0].z, v[u][0].w,
-                                   v[u][1].x, v[u][1].y, v[u][1].z, v[u][1].w};
+            uint32_t w[8] = {v[u][0].x, v[u][0].y, v[u][0].z, v[u][0].w,
+                             v[u][1].x, v[u][1].y, v[u][1].z, v[u][1].w};
+            if (NORM && r < rows && col_ok) {
+                const float rs = __ldg(na.rstd + r);
+                const uint4 g0 = __ldg(reinterpret_cast<const uint4*>(na.gamma + col));
+                const uint4 g1 = __ldg(reinterpret_cast<const uint4*>(na.gamma + col) + 1);
+                const uint32_t g[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+#pragma unroll
+                for (int j = 0; j < 8; ++j) w[j] = norm_pair(w[j], g[j], rs);
+                if (na.h_out != nullptr) {
+                    uint4* hp = reinterpret_cast<uint4*>(na.h_out + r * K + col);
+                    hp[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                    hp[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                }
+            }
             // Eq. 3: sigma_b = Pi_E4M3(amax_b / (alpha * q_max))
             const float amax = bf16x16_absmax(w);
             uint32_t sc = e4m3_block_scale(amax, qc.alpha_qmax, qc.inv_lo, qc.inv_hi);
@@ -401,11 +432,11 @@ __device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v)
 //     (bounded; a wait that runs out posts kErrTimeout and the block stops).
 //     The quantization pass then walks the tiles in the opposite order, so
 //     the lines read last by the amax pass, still in L2, are read first.
-template <bool SEARCH>
+template <bool SEARCH, bool NORM>
 __global__ void __launch_bounds__(kQuantThreads, MQ_QUANT_MIN_BLOCKS)
     quantize_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t K, const float* __restrict__ alpha_static,
                     float* __restrict__ alpha_out, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
-                    int64_t interleave_half, WsControl* ctrl, uint32_t* __restrict__ partials)
+                    int64_t interleave_half, WsControl* ctrl, uint32_t* __restrict__ partials, NormArgs na)
 {
     __shared__ __align__(16) uint8_t sf_stage[2048];
     __shared__ float enc_tab[128];
@@ -498,13 +529,13 @@ __global__ void __launch_bounds__(kQuantThreads, MQ_QUANT_MIN_BLOCKS)
     // ---- pass 2: quantize, tiles in reverse order of pass 1
     for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
         const int64_t tile = tiles - 1 - t;
-        quant_tile<SEARCH>(x, rows, K, interleave_half, tile / chunks, tile % chunks, chunks, qc, enc_tab, dec_tab,
-                           sf_stage, codes, scales, warp, half, blk);
+        quant_tile<SEARCH, NORM>(x, rows, K, interleave_half, tile / chunks, tile % chunks, chunks, qc, enc_tab,
+                                 dec_tab, sf_stage, codes, scales, warp, half, blk, na);
     }
 }
 
 // Resident blocks per SM of quantize_kernel<SEARCH> (cached per device).
-template <bool SEARCH>
+template <bool SEARCH, bool NORM>
 int quantize_blocks_per_sm(const DeviceInfo& di)
 {
     static std::mutex mu;
@@ -512,7 +543,7 @@ int quantize_blocks_per_sm(const DeviceInfo& di)
     std::lock_guard<std::mutex> lock(mu);
     if (di.device >= 0 && di.device < 64 && per_sm[di.device] > 0) return per_sm[di.device];
     int occ = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quantize_kernel<SEARCH>, kQuantThreads, 0) !=
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quantize_kernel<SEARCH, NORM>, kQuantThreads, 0) !=
         cudaSuccess) {
         (void)cudaGetLastError();
         occ = 0;
@@ -526,7 +557,7 @@ cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float*
                             uint32_t* partials, const DeviceInfo& di, cudaStream_t s, bool scale_search)
 {
     const int64_t tiles = ((rows + 127) / 128) * ((K + 255) / 256);
-    const int occ = scale_search ? quantize_blocks_per_sm<true>(di) : quantize_blocks_per_sm<false>(di);
+    const int occ = scale_search ? quantize_blocks_per_sm<true, false>(di) : quantize_blocks_per_sm<false, false>(di);
     const int64_t resident = (int64_t)di.num_sms * std::max(1, occ);
     // Small tensors (at most one tile per SM): one cooperative launch takes
     // the amax, hands alpha to every block and quantizes; the two-kernel path
@@ -553,10 +584,112 @@ cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float*
     attr[0].val.cooperative = single ? 1 : 0;   // blocks wait on one another only in the single-launch amax
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    auto kern = scale_search ? quantize_kernel<true> : quantize_kernel<false>;
+    auto kern = scale_search ? quantize_kernel<true, false> : quantize_kernel<false, false>;
     cudaError_t e = cudaLaunchKernelEx(&cfg, kern, static_cast<const uint16_t*>(x), rows, K, alpha_in, alpha_out,
-                                       codes, scales, interleave_half, ctrl, partials);
+                                       codes, scales, interleave_half, ctrl, partials, NormArgs{});
     if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+// ==========================================================================
+// RMSNorm fused with the quantization of its output
+// ==========================================================================
+//
+// Pass 1 (this kernel): one warp per row computes ms = fl32(sum x^2 / K) with
+// the sum in binary64, rstd = fl32(1 / sqrt(ms + eps)) (binary64, one
+// rounding), stores rstd and takes the |h| maximum of the row's
+// h = bf16(fl(fl(x * rstd) * gamma)); the last block folds the per-block
+// maxima into alpha_h = amax/2688 (1 if 0; NaN/Inf excluded and reported).
+// Pass 2 is quantize_kernel<false, true>, which forms h again on load.
+constexpr int kNormThreads = 256;
+
+__global__ void __launch_bounds__(kNormThreads) rmsnorm_amax_kernel(const uint16_t* __restrict__ x, int64_t rows,
+                                                                    int64_t K, const uint16_t* __restrict__ gamma,
+                                                                    float eps, float* __restrict__ rstd,
+                                                                    float* __restrict__ alpha_out, WsControl* ctrl,
+                                                                    uint32_t* __restrict__ partials)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t wstride = (int64_t)gridDim.x * (kNormThreads / 32);
+    uint32_t mx = 0, bad = 0;
+    for (int64_t r = (int64_t)blockIdx.x * (kNormThreads / 32) + warp; r < rows; r += wstride) {
+        const uint4* xr = reinterpret_cast<const uint4*>(x + r * K);
+        const int64_t nv = K / 8;
+        double ss = 0.0;
+        for (int64_t i = lane; i < nv; i += 32) {
+            const uint4 v = __ldg(xr + i);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const double a = (double)bf16_lo(w[j]), b = (double)bf16_hi(w[j]);
+                ss = __dadd_rn(ss, __dmul_rn(a, a));
+                ss = __dadd_rn(ss, __dmul_rn(b, b));
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
+        const float ms = __double2float_rn(__ddiv_rn(ss, (double)K));
+        const float rs = __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(__dadd_rn((double)ms, (double)eps))));
+        if (lane == 0) rstd[r] = rs;
+        const uint4* gr = reinterpret_cast<const uint4*>(gamma);
+        for (int64_t i = lane; i < nv; i += 32) {
+            const uint4 v = __ldg(xr + i);
+            const uint4 g = __ldg(gr + i);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            const uint32_t gw[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) amax_accum(norm_pair(w[j], gw[j], rs), mx, bad);
+        }
+    }
+    uint32_t m = max(mx & 0xFFFFu, mx >> 16) | (bad ? 0x80000000u : 0u);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fold_max_flag(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    __shared__ uint32_t s_red[kNormThreads / 32];
+    __shared__ bool is_last;
+    if (lane == 0) s_red[warp] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t b = 0;
+        for (int w = 0; w < kNormThreads / 32; ++w) b = fold_max_flag(b, s_red[w]);
+        partials[blockIdx.x] = b;
+        __threadfence();
+        is_last = (atomicAdd(&ctrl->amax_ticket, 1u) == gridDim.x - 1);
+    }
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+    if (threadIdx.x == 0) {
+        uint32_t b = 0;
+        for (int j = 0; j < (int)gridDim.x; ++j) b = fold_max_flag(b, __ldcg(partials + j));
+        const float amax = __uint_as_float((b & 0x7FFFu) << 16);
+        *alpha_out = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
+        if (b & 0x80000000u) post_error(ctrl, kErrNonFinite);
+        ctrl->amax_ticket = 0;
+        __threadfence();
+    }
+}
+
+cudaError_t launch_rmsnorm_quantize(const void* x, int64_t rows, int64_t K, const void* gamma, float eps,
+                                    float* rstd, uint8_t* codes, uint8_t* scales, float* alpha_out, void* h_out,
+                                    WsControl* ctrl, uint32_t* partials, const DeviceInfo& di, cudaStream_t s)
+{
+    int64_t blocks = (rows + kNormThreads / 32 - 1) / (kNormThreads / 32);
+    blocks = std::min<int64_t>(blocks, (int64_t)di.num_sms * 8);
+    blocks = std::min<int64_t>(blocks, kAmaxMaxBlocks);
+    blocks = std::max<int64_t>(blocks, 1);
+    rmsnorm_amax_kernel<<<(unsigned)blocks, kNormThreads, 0, s>>>(static_cast<const uint16_t*>(x), rows, K,
+                                                                  static_cast<const uint16_t*>(gamma), eps, rstd,
+                                                                  alpha_out, ctrl, partials);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const int64_t tiles = ((rows + 127) / 128) * ((K + 255) / 256);
+    const int occ = quantize_blocks_per_sm<false, true>(di);
+    int64_t qb = std::min(tiles, (int64_t)di.num_sms * std::max(1, occ));
+    qb = std::max<int64_t>(qb, 1);
+    NormArgs na{static_cast<const uint16_t*>(gamma), rstd, static_cast<uint16_t*>(h_out)};
+    quantize_kernel<false, true><<<(unsigned)qb, kQuantThreads, 0, s>>>(static_cast<const uint16_t*>(x), rows, K,
+                                                                         alpha_out, alpha_out, codes, scales, 0, ctrl,
+                                                                         partials, na);
     return cudaGetLastError();
 }
 

@@ -33,7 +33,7 @@ STATUS_NAMES = {0: "MQ_OK", 1: "MQ_ERR_INVALID_ARG", 2: "MQ_ERR_SHAPE", 3: "MQ_E
 EXPORTS = ("mq_status_string", "mq_version", "mq_nvfp4_sizes", "mq_workspace_bytes", "mq_quantize_weight",
            "mq_quantize_activation", "mq_prefill_linear", "mq_decode_linear", "mq_unswizzle_scales",
            "mq_async_status", "mq_prefill_linear_noalloc", "mq_selftest_e2m1", "mq_selftest_timeout",
-           "mq_decode_linear_nvfp4", "mq_quantize")
+           "mq_decode_linear_nvfp4", "mq_quantize", "mq_rmsnorm_quantize")
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
@@ -91,6 +91,8 @@ def load(path: str = LIB_PATH):
             lib.mq_decode_linear_nvfp4.restype = i32
             lib.mq_quantize.argtypes = [vp, i64, i64, vp, ctypes.c_uint, nvp, vp, sz, vp]
             lib.mq_quantize.restype = i32
+            lib.mq_rmsnorm_quantize.argtypes = [vp, i64, i64, vp, ctypes.c_float, nvp, vp, vp, sz, vp]
+            lib.mq_rmsnorm_quantize.restype = i32
             lib.mq_prefill_linear_noalloc.argtypes = [vp, i64, nvp, vp, vp, vp]
             lib.mq_prefill_linear_noalloc.restype = i32
             _lib = lib
@@ -190,6 +192,18 @@ def quantize(X, alpha_static=None, gate_up_interleave: bool = False, scale_searc
     oc = out.c()
     _check(load().mq_quantize(_ptr(X), rows, K, _ptr(alpha_static), flags, ctypes.byref(oc), *_ws_args(ws),
                               _stream(stream)), "mq_quantize")
+    return out
+
+
+def rmsnorm_quantize(X, gamma, eps: float = 1e-6, out: NVFP4Tensor | None = None, h_debug=None, ws=None,
+                     stream=None) -> NVFP4Tensor:
+    """mq_rmsnorm_quantize: NVFP4 copy of RMSNorm(X) * gamma without writing the BF16 norm output."""
+    M, K = X.shape
+    out = out or nvfp4_empty(M, K, X.device)
+    ws = ws if ws is not None else workspace(M, K, X.device)
+    oc = out.c()
+    _check(load().mq_rmsnorm_quantize(_ptr(X), M, K, _ptr(gamma), ctypes.c_float(eps), ctypes.byref(oc),
+                                      _ptr(h_debug), *_ws_args(ws), _stream(stream)), "mq_rmsnorm_quantize")
     return out
 
 

@@ -16,7 +16,8 @@ iteration then launches only the operation named:
   epilogue (N = 2 x intermediate size, interleaved gate/up rows);
 * ``decode``: the BF16 decode GEMM Y = X W^T (M <= 256);
 * ``decode_nvfp4``: the uniform-NVFP4 decode (tokens quantized on the fly,
-  NVFP4 weight; M <= 128).
+  NVFP4 weight; M <= 128);
+* ``rmsnorm_quant``: RMSNorm fused with the NVFP4 quantization of its output.
 
 Prints the mean CUDA-event time per iteration.  The data recipe is the one the
 tests and the benchmark use (Student-t(3) activations with 1 % outlier
@@ -32,7 +33,7 @@ import numpy as np
 
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
-    ap.add_argument("op", choices=["quant", "gemm", "mlp", "decode", "decode_nvfp4"])
+    ap.add_argument("op", choices=["quant", "gemm", "mlp", "decode", "decode_nvfp4", "rmsnorm_quant"])
     ap.add_argument("--M", type=int, default=8192)
     ap.add_argument("--N", type=int, default=4096)
     ap.add_argument("--K", type=int, default=4096)
@@ -51,7 +52,11 @@ def main(argv=None) -> int:
 
     X = dev_bf16(wl.heavy_tailed_bf16(a.M, a.K, 11))
     ws = mq.workspace(a.M, a.K, device=dev)
-    if a.op == "quant":
+    if a.op == "rmsnorm_quant":
+        gam = dev_bf16(wl.normal_bf16(1, a.K, 1.0, 13)[0])
+        Xq = mq.nvfp4_empty(a.M, a.K, dev)
+        run = lambda: mq.rmsnorm_quantize(X, gam, 1e-6, out=Xq, ws=ws)
+    elif a.op == "quant":
         Xq = mq.nvfp4_empty(a.M, a.K, dev)
         run = lambda: mq.quantize_activation(X, out=Xq, ws=ws)
     elif a.op in ("gemm", "mlp"):

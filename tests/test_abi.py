@@ -108,6 +108,14 @@ def test_argument_errors_are_synchronous(lib):
     assert lib.mq_quantize(P, 200, 256, None, ctypes.c_uint(4), ctypes.byref(q), ws, wsb, None) == 1
     assert lib.mq_quantize(P, 200, 256, None, ctypes.c_uint(1), ctypes.byref(q), ws, wsb, None) == 2
     assert lib.mq_quantize(P + 2, 200, 256, None, ctypes.c_uint(2), ctypes.byref(q), ws, wsb, None) == 3
+    # fused RMSNorm + quantization: gamma required, eps finite >= 0, K % 64
+    rq = _nv(128, 256)
+    assert lib.mq_rmsnorm_quantize(P, 128, 256, None, ctypes.c_float(1e-6), ctypes.byref(rq), None, ws, wsb,
+                                   None) == 1
+    assert lib.mq_rmsnorm_quantize(P, 128, 256, P, ctypes.c_float(-1.0), ctypes.byref(rq), None, ws, wsb, None) == 1
+    assert lib.mq_rmsnorm_quantize(P, 128, 200, P, ctypes.c_float(1e-6), ctypes.byref(rq), None, ws, wsb, None) == 2
+    assert lib.mq_rmsnorm_quantize(P, 128, 256, P + 8, ctypes.c_float(1e-6), ctypes.byref(rq), None, ws, wsb,
+                                   None) == 3
     # timeout self-test: timeout in (0, 2 s], a workspace, an aligned result slot
     assert lib.mq_selftest_timeout(ws, wsb, ctypes.c_uint64(0), None, None) == 1
     assert lib.mq_selftest_timeout(ws, wsb, ctypes.c_uint64(3 * 10 ** 9), None, None) == 1
