@@ -603,6 +603,16 @@ cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float*
 // Pass 2 is quantize_kernel<false, true>, which forms h again on load.
 constexpr int kNormThreads = 256;
 
+// (hi, lo) += b with Knuth's TwoSum: hi + lo keeps the sum to about 48 bits.
+__device__ __forceinline__ void ff_add(float& hi, float& lo, float b)
+{
+    const float s = __fadd_rn(hi, b);
+    const float bp = __fsub_rn(s, hi);
+    const float e = __fadd_rn(__fsub_rn(hi, __fsub_rn(s, bp)), __fsub_rn(b, bp));
+    hi = s;
+    lo = __fadd_rn(lo, e);
+}
+
 __global__ void __launch_bounds__(kNormThreads) rmsnorm_amax_kernel(const uint16_t* __restrict__ x, int64_t rows,
                                                                     int64_t K, const uint16_t* __restrict__ gamma,
                                                                     float eps, float* __restrict__ rstd,
@@ -612,33 +622,72 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_amax_kernel(const uint16
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t wstride = (int64_t)gridDim.x * (kNormThreads / 32);
     uint32_t mx = 0, bad = 0;
+    // A row is read in chunks of kNormChunk 16-byte vectors per lane, all in
+    // flight at once; a row of at most one chunk (K <= 4096) stays in
+    // registers for the |h| pass, longer rows are read again (from L2).
+    constexpr int kNormChunk = 16;
+    const uint4* gr = reinterpret_cast<const uint4*>(gamma);
+    const int64_t nv = K / 8;
+    const int64_t chunk = 32 * kNormChunk;
     for (int64_t r = (int64_t)blockIdx.x * (kNormThreads / 32) + warp; r < rows; r += wstride) {
         const uint4* xr = reinterpret_cast<const uint4*>(x + r * K);
-        const int64_t nv = K / 8;
-        double ss = 0.0;
-        for (int64_t i = lane; i < nv; i += 32) {
-            const uint4 v = __ldg(xr + i);
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        uint4 v[kNormChunk];
+        // sum of squares: each square of a BF16 value is exact in binary32
+        // (8 significant bits, for |x| in [2^-63, 2^63]); the running sum is an
+        // unevaluated pair (about 48 bits), converted to binary64 once per row,
+        // which stands for the binary64 sum of the definition (the two agree
+        // unless the sum lies within ~2^-45 relative of an FP32 rounding
+        // boundary of ms).  FP64 conversions per element would be the slow path.
+        float hi0 = 0.0f, lo0 = 0.0f, hi1 = 0.0f, lo1 = 0.0f;
+        for (int64_t c0 = 0; c0 < nv; c0 += chunk) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const double a = (double)bf16_lo(w[j]), b = (double)bf16_hi(w[j]);
-                ss = __dadd_rn(ss, __dmul_rn(a, a));
-                ss = __dadd_rn(ss, __dmul_rn(b, b));
+            for (int u = 0; u < kNormChunk; ++u) {
+                const int64_t i = c0 + lane + 32 * u;
+                v[u] = (i < nv) ? __ldg(xr + i) : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int u = 0; u < kNormChunk; ++u) {
+                const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float a = bf16_lo(w[j]), b = bf16_hi(w[j]);
+                    ff_add(hi0, lo0, __fmul_rn(a, a));
+                    ff_add(hi1, lo1, __fmul_rn(b, b));
+                }
             }
         }
+        ff_add(hi0, lo0, hi1);
+        lo0 = __fadd_rn(lo0, lo1);
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
+        for (int o = 16; o > 0; o >>= 1) {
+            const float oh = __shfl_xor_sync(0xFFFFFFFFu, hi0, o);
+            const float ol = __shfl_xor_sync(0xFFFFFFFFu, lo0, o);
+            ff_add(hi0, lo0, oh);
+            lo0 = __fadd_rn(lo0, ol);
+        }
+        const double ss = __dadd_rn((double)hi0, (double)lo0);
         const float ms = __double2float_rn(__ddiv_rn(ss, (double)K));
         const float rs = __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(__dadd_rn((double)ms, (double)eps))));
         if (lane == 0) rstd[r] = rs;
-        const uint4* gr = reinterpret_cast<const uint4*>(gamma);
-        for (int64_t i = lane; i < nv; i += 32) {
-            const uint4 v = __ldg(xr + i);
-            const uint4 g = __ldg(gr + i);
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-            const uint32_t gw[4] = {g.x, g.y, g.z, g.w};
+        for (int64_t c0 = 0; c0 < nv; c0 += chunk) {
+            if (nv > chunk) {   // the chunk is no longer in registers
 #pragma unroll
-            for (int j = 0; j < 4; ++j) amax_accum(norm_pair(w[j], gw[j], rs), mx, bad);
+                for (int u = 0; u < kNormChunk; ++u) {
+                    const int64_t i = c0 + lane + 32 * u;
+                    v[u] = (i < nv) ? __ldg(xr + i) : make_uint4(0u, 0u, 0u, 0u);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kNormChunk; ++u) {
+                const int64_t i = c0 + lane + 32 * u;
+                if (i < nv) {
+                    const uint4 g = __ldg(gr + i);
+                    amax_accum(norm_pair(v[u].x, g.x, rs), mx, bad);
+                    amax_accum(norm_pair(v[u].y, g.y, rs), mx, bad);
+                    amax_accum(norm_pair(v[u].z, g.z, rs), mx, bad);
+                    amax_accum(norm_pair(v[u].w, g.w, rs), mx, bad);
+                }
+            }
         }
     }
     uint32_t m = max(mx & 0xFFFFu, mx >> 16) | (bad ? 0x80000000u : 0u);
@@ -657,10 +706,18 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_amax_kernel(const uint16
     }
     __syncthreads();
     if (!is_last) return;
+    // the last block folds every block's maximum, all threads at once
     __threadfence();
+    uint32_t b = 0;
+    for (int j = threadIdx.x; j < (int)gridDim.x; j += kNormThreads) b = fold_max_flag(b, __ldcg(partials + j));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) b = fold_max_flag(b, __shfl_xor_sync(0xFFFFFFFFu, b, o));
+    __syncthreads();
+    if (lane == 0) s_red[warp] = b;
+    __syncthreads();
     if (threadIdx.x == 0) {
-        uint32_t b = 0;
-        for (int j = 0; j < (int)gridDim.x; ++j) b = fold_max_flag(b, __ldcg(partials + j));
+        b = 0;
+        for (int w = 0; w < kNormThreads / 32; ++w) b = fold_max_flag(b, s_red[w]);
         const float amax = __uint_as_float((b & 0x7FFFu) << 16);
         *alpha_out = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
         if (b & 0x80000000u) post_error(ctrl, kErrNonFinite);
