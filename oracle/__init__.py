@@ -231,6 +231,25 @@ def nvfp4_linear_rows(xq, wq, rows=None):
     return y, sabs
 
 
+def kv_rope_rows(yk: np.ndarray, yv: np.ndarray, positions: np.ndarray, cos_sin: np.ndarray, head_dim: int = 128):
+    """RoPE on the K projection output and the KV-cache values in BF16 (the decode precision).
+
+    yk, yv: float64 [M, H*head_dim] projection outputs (before BF16 rounding).  For every head
+    and i < head_dim/2, with c = cos_sin[pos, i], s = cos_sin[pos, head_dim/2 + i]:
+    k'_i = k_i c - k_{i+d/2} s and k'_{i+d/2} = k_{i+d/2} c + k_i s (rotate-half form), in float64.
+    Returns (K', V) as BF16 bit patterns [M, H*head_dim].
+    """
+    yk = np.asarray(yk, dtype=np.float64)
+    M, n = yk.shape
+    H, d2 = n // head_dim, head_dim // 2
+    cs = np.asarray(cos_sin, dtype=np.float64)[np.asarray(positions, dtype=np.int64)]   # [M, head_dim]
+    c, s = cs[:, None, :d2], cs[:, None, d2:]
+    k = yk.reshape(M, H, head_dim)
+    a, b = k[:, :, :d2], k[:, :, d2:]
+    kr = np.concatenate([a * c - b * s, b * c + a * s], axis=2).reshape(M, n)
+    return round_bf16(kr), round_bf16(np.asarray(yv, dtype=np.float64))
+
+
 def bf16_linear_rows(x_bf16: np.ndarray, w_bf16: np.ndarray, rows=None) -> np.ndarray:
     """y = x @ w^T in float64 on BF16 inputs (the precise decode path)."""
     x = x_bf16 if rows is None else x_bf16[np.asarray(rows, dtype=np.int64)]

@@ -175,3 +175,14 @@ def mlp_weights(seed: int, hidden: int = QWEN3_8B_HIDDEN, inter: int = QWEN3_8B_
     w_gu = normal_bf16(2 * inter, hidden, WEIGHT_STD, seed + 1)
     w_dn = normal_bf16(hidden, inter, WEIGHT_STD, seed + 2)
     return w_gu, w_dn
+
+
+def rope_cos_sin(max_pos: int, head_dim: int = 128, theta: float = 1.0e6) -> np.ndarray:
+    """Rotary-embedding table input [max_pos, head_dim] float32: row p holds
+    cos(p * f_i) for i < head_dim/2 followed by sin(p * f_i), f_i =
+    theta^(-2i/head_dim) (theta = 1e6 as in the Qwen3 models).  Evaluated in
+    float64 and rounded once; an input of the K/V projection, like the weights."""
+    half = head_dim // 2
+    f = theta ** (-2.0 * np.arange(half, dtype=np.float64) / head_dim)
+    ang = np.arange(max_pos, dtype=np.float64)[:, None] * f[None, :]
+    return np.concatenate([np.cos(ang), np.sin(ang)], axis=1).astype(np.float32)

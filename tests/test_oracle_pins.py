@@ -486,3 +486,63 @@ def test_rmsnorm_closed_forms():
     assert r[0] == np.float32(1.0 / 3.0)
     sign = np.tile(np.array([0, 0x8000], np.uint16), 128)
     assert np.array_equal(h[0], g ^ sign)
+
+
+# ------------------------------------------------------------------ RoPE on the K projection
+
+def _rope_f64(yk, pos, cs):
+    k, _ = oracle.kv_rope_rows(yk, np.zeros_like(yk), pos, cs)
+    return oracle.bf16_to_f64(k)
+
+
+def test_rope_identity_at_position_zero_and_norm_preserved():
+    rng = np.random.default_rng(71)
+    cs = wl.rope_cos_sin(64)
+    yk = rng.standard_normal((4, 256))
+    k0 = _rope_f64(yk, np.zeros(4, np.int64), cs)
+    assert np.array_equal(k0, oracle.bf16_to_f64(oracle.round_bf16(yk)))
+    # each (i, i+64) pair is rotated: its norm is kept (up to the BF16 rounding of the output)
+    kr = _rope_f64(yk, np.array([1, 7, 33, 63]), cs).reshape(4, 2, 2, 64)
+    y = yk.reshape(4, 2, 2, 64)
+    n_in = y[:, :, 0] ** 2 + y[:, :, 1] ** 2
+    n_out = kr[:, :, 0] ** 2 + kr[:, :, 1] ** 2
+    assert np.allclose(n_out, n_in, rtol=2 ** -6, atol=1e-3)
+
+
+def test_rope_scores_depend_only_on_relative_position():
+    """The defining property of rotary embeddings: <R(p) q, R(p') k> depends on p - p' only
+    (checked on the un-rounded rotation; the oracle's output differs from it by BF16 rounding)."""
+    rng = np.random.default_rng(72)
+    cs = wl.rope_cos_sin(512).astype(np.float64)
+    q, k = rng.standard_normal(128), rng.standard_normal(128)
+
+    def rot(v, p):
+        c, s = cs[p, :64], cs[p, 64:]
+        return np.concatenate([v[:64] * c - v[64:] * s, v[64:] * c + v[:64] * s])
+    for p, pp, delta in [(10, 3, 100), (200, 50, 7), (5, 5, 300)]:
+        a = rot(q, p) @ rot(k, pp)
+        b = rot(q, p + delta) @ rot(k, pp + delta)
+        assert abs(a - b) < 2e-5 * (1 + abs(a))
+    # the oracle computes exactly that rotation before rounding to BF16
+    yk = rng.standard_normal((3, 128))
+    pos = np.array([3, 100, 511])
+    mine = _rope_f64(yk, pos, cs.astype(np.float32))
+    ref = np.stack([rot(yk[i], pos[i]) for i in range(3)])
+    cs32 = cs.astype(np.float32).astype(np.float64)
+    ref32 = np.stack([np.concatenate([yk[i, :64] * cs32[p, :64] - yk[i, 64:] * cs32[p, 64:],
+                                      yk[i, 64:] * cs32[p, :64] + yk[i, :64] * cs32[p, 64:]])
+                      for i, p in enumerate(pos)])
+    assert np.array_equal(mine, oracle.bf16_to_f64(oracle.round_bf16(ref32)))
+    assert np.allclose(mine, ref, rtol=2 ** -7, atol=1e-6)
+    # and the property holds for the oracle's own (BF16) outputs, which a sign or index slip
+    # in its rotation would break
+    cs32 = cs.astype(np.float32)
+    qs = rng.standard_normal((1, 128)) * 4
+    ks = rng.standard_normal((1, 128)) * 4
+    for p, pp, delta in [(10, 3, 100), (200, 50, 7), (30, 400, 60)]:
+        a = _rope_f64(qs, np.array([p]), cs32)[0] @ _rope_f64(ks, np.array([pp]), cs32)[0]
+        b = _rope_f64(qs, np.array([p + delta]), cs32)[0] @ _rope_f64(ks, np.array([pp + delta]), cs32)[0]
+        assert abs(a - b) < 0.02 * np.linalg.norm(qs) * np.linalg.norm(ks) ** 1, (p, pp, a, b)
+        if delta >= 60:   # shifting only one side does change the score, well beyond the rounding noise
+            c = _rope_f64(qs, np.array([p]), cs32)[0] @ _rope_f64(ks, np.array([pp + delta]), cs32)[0]
+            assert abs(a - c) > 10 * abs(a - b)
