@@ -407,6 +407,25 @@ def measure_extras(mq, torch, dev, flush, hbm_gbs, fp4_peak, reps=10):
     out["scale_search"] = {"weight": [N, K], "ms_eq3": ms_p, "ms_search": ms_s,
                            "GB/s_search": (2 + 0.5625) * N * K / (ms_s * 1e-3) / 1e9,
                            "rel_err_eq3": err_p, "rel_err_search": err_s, "blocks_moved": moved}
+    # K/V projection with RoPE + KV-cache write in the epilogue vs the same GEMM with a plain BF16 output
+    Hk, Mk = 8, 8192
+    Xk = _to_dev(torch, wl.heavy_tailed_bf16(Mk, K, 70), dev)
+    wsk = mq.workspace(Mk, K, device=dev)
+    Xkq = mq.quantize_activation(Xk, ws=wsk)
+    Wkv = mq.quantize_weight(_to_dev(torch, wl.normal_bf16(2 * Hk * 128, K, 0.02, 71), dev), ws=wsk)
+    csk = torch.from_numpy(wl.rope_cos_sin(40960)).to(dev)
+    posk = torch.randint(0, 40960, (Mk,), dtype=torch.int32, device=dev)
+    slk = torch.randperm(Mk, device=dev)
+    kck = torch.empty((Mk, Hk, 128), dtype=torch.bfloat16, device=dev)
+    vck = torch.empty_like(kck)
+    Yk = torch.empty((Mk, 2 * Hk * 128), dtype=torch.bfloat16, device=dev)
+    ms_kv = _time_calls(torch, lambda: mq.prefill_kv_rope(W=Wkv, Xq=Xkq, n_kv_heads=Hk, positions=posk, cos_sin=csk,
+                                                           slots=slk, k_cache=kck, v_cache=vck, ws=wsk), reps, flush)
+    ms_plain = _time_calls(torch, lambda: mq.prefill_linear(W=Wkv, Xq=Xkq, Y=Yk, ws=wsk), reps, flush)
+    fl_kv = 2 * Mk * 2 * Hk * 128 * K
+    out["kv_rope"] = {"M": Mk, "K": K, "n_kv_heads": Hk, "ms_fused": ms_kv, "ms_plain_gemm": ms_plain,
+                      "TFLOP/s_fused": fl_kv / (ms_kv * 1e-3) / 1e12, "TFLOP/s_plain": fl_kv / (ms_plain * 1e-3) / 1e12}
+    del Xk, Xkq, kck, vck, Yk
     # RMSNorm -> NVFP4 fused (the producer of the q/k/v input) vs the unfused pair
     Mr = 8192
     Xr = _to_dev(torch, wl.heavy_tailed_bf16(Mr, K, 61), dev)

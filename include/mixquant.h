@@ -66,7 +66,8 @@ typedef enum mq_status {
     MQ_ERR_NONFINITE = 5,   /* (async) NaN or Inf in a tensor that was quantized */
     MQ_ERR_TIMEOUT = 6,     /* (async) a device-side pipeline wait gave up */
     MQ_ERR_CUDA = 7,        /* a CUDA runtime/driver call failed */
-    MQ_ERR_DEVICE = 8       /* current device is not compute capability 10.0 (B200) */
+    MQ_ERR_DEVICE = 8,      /* current device is not compute capability 10.0 (B200) */
+    MQ_ERR_INDEX = 9        /* (async) a token position or cache slot out of range */
 } mq_status;
 
 typedef enum mq_epilogue {
@@ -208,6 +209,30 @@ MQ_API mq_status mq_prefill_linear_noalloc(const void* X_bf16, int64_t M, const 
 MQ_API mq_status mq_quantize(const void* X_bf16, int64_t rows, int64_t K, const float* alpha_static, unsigned flags,
                              const mq_nvfp4* out, void* ws, size_t ws_bytes, mq_stream_t stream);
 
+/* K/V projection of the prefill with its outputs in the decode precision
+ * ("Prefill-Decode Disaggregation Deployment": the prefill writes the KV cache
+ * in the precision the high-precision decode engine expects): one NVFP4 GEMM
+ * against W_kv = [K-projection rows; V-projection rows], 2 * n_kv_heads * 128
+ * rows of head dimension 128, whose epilogue
+ *   - scales the FP32 sums by fl(alpha_x * alpha_w),
+ *   - applies rotary position embedding to the K heads (rotate-half form:
+ *     pairs i, i + 64 with c = cos_sin[pos][i], s = cos_sin[pos][64 + i]:
+ *     k'_i = fl(fl(k_i c) - fl(k_{i+64} s)), k'_{i+64} = fl(fl(k_{i+64} c) +
+ *     fl(k_i s)), binary32),
+ *   - rounds to BF16 and writes token m's heads to k_cache[slots[m]][h][:] and
+ *     v_cache[slots[m]][h][:] ([num_slots, n_kv_heads, 128] BF16 each).
+ * positions: int32 [M] (4-byte aligned), slots: int64 [M] (8-byte aligned),
+ * cos_sin: FP32 [max_pos, 128] (cos of the 64 frequencies, then sin; 16-byte
+ * aligned), caches 16-byte aligned.  X as in mq_prefill_linear (BF16 quantized
+ * on the fly with a dynamic alpha, or an NVFP4 X_q).  A position outside
+ * [0, max_pos) or a slot outside [0, num_slots) skips that token and posts
+ * MQ_ERR_INDEX (read with mq_async_status).  Slots must be distinct.
+ * The method has no fused form of this; RoPE is the Qwen3 attention's. */
+MQ_API mq_status mq_prefill_kv_rope(const void* X_bf16, const mq_nvfp4* X_q, int64_t M, const mq_nvfp4* W_kv,
+                                    int64_t n_kv_heads, const int32_t* positions, const float* cos_sin,
+                                    int64_t max_pos, const int64_t* slots, void* k_cache, void* v_cache,
+                                    int64_t num_slots, void* ws, size_t ws_bytes, mq_stream_t stream);
+
 /* RMSNorm fused with the quantization of its output: the NVFP4 copy of
  *   h[m][k] = bf16( fl32( fl32(x[m][k] * rstd_m) * gamma[k] ) ),
  *   ms_m = fl32( sum_k x^2 (binary64) / K ), rstd_m = fl32( 1/sqrt(ms_m + eps) ),
@@ -265,7 +290,7 @@ MQ_API mq_status mq_selftest_timeout(void* ws, size_t ws_bytes, uint64_t timeout
                                      mq_stream_t stream);
 
 /* Synchronize `stream`, then read and clear the asynchronous error bits of
- * workspace `ws`: MQ_OK, MQ_ERR_NONFINITE, MQ_ERR_TIMEOUT (or MQ_ERR_CUDA if
+ * workspace `ws`: MQ_OK, MQ_ERR_NONFINITE, MQ_ERR_TIMEOUT, MQ_ERR_INDEX (or MQ_ERR_CUDA if
  * the synchronization itself failed). */
 MQ_API mq_status mq_async_status(void* ws, mq_stream_t stream);
 

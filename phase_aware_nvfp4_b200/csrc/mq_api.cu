@@ -185,6 +185,7 @@ const char* mq_status_string(mq_status s)
         case MQ_ERR_TIMEOUT: return "MQ_ERR_TIMEOUT";
         case MQ_ERR_CUDA: return "MQ_ERR_CUDA";
         case MQ_ERR_DEVICE: return "MQ_ERR_DEVICE";
+        case MQ_ERR_INDEX: return "MQ_ERR_INDEX";
     }
     return "MQ_ERR_UNKNOWN";
 }
@@ -253,6 +254,68 @@ mq_status mq_quantize(const void* X_bf16, int64_t rows, int64_t K, const float* 
     return quantize_into(X_bf16, rows, K, alpha_static, out->codes, out->scales, out->alpha, true,
                          interleave ? rows / 2 : 0, w, di, reinterpret_cast<cudaStream_t>(stream), nullptr,
                          (flags & MQ_QUANT_SCALE_SEARCH) != 0);
+}
+
+mq_status mq_prefill_kv_rope(const void* X_bf16, const mq_nvfp4* X_q, int64_t M, const mq_nvfp4* W_kv,
+                             int64_t n_kv_heads, const int32_t* positions, const float* cos_sin, int64_t max_pos,
+                             const int64_t* slots, void* k_cache, void* v_cache, int64_t num_slots, void* ws,
+                             size_t ws_bytes, mq_stream_t stream)
+{
+    if ((X_bf16 == nullptr) == (X_q == nullptr)) return MQ_ERR_INVALID_ARG;
+    if (W_kv == nullptr || W_kv->codes == nullptr || W_kv->scales == nullptr || W_kv->alpha == nullptr)
+        return MQ_ERR_INVALID_ARG;
+    if (positions == nullptr || cos_sin == nullptr || slots == nullptr || k_cache == nullptr || v_cache == nullptr)
+        return MQ_ERR_INVALID_ARG;
+    const int64_t N = W_kv->rows, K = W_kv->cols;
+    if (n_kv_heads < 1 || n_kv_heads > 4096 || N != 2 * n_kv_heads * 128) return MQ_ERR_SHAPE;
+    if (M < 1 || M > (int64_t)1 << 30 || K < 64 || K % 64 != 0 || K > (int64_t)1 << 30) return MQ_ERR_SHAPE;
+    if (max_pos < 1 || num_slots < 1) return MQ_ERR_SHAPE;
+    if (!aligned16(cos_sin) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        (reinterpret_cast<uintptr_t>(positions) & 3u) || (reinterpret_cast<uintptr_t>(slots) & 7u))
+        return MQ_ERR_ALIGNMENT;
+    mq_status st = check_nvfp4(W_kv, N, K);
+    if (st != MQ_OK) return st;
+    const bool quantize_x = X_bf16 != nullptr;
+    if (quantize_x) {
+        if (!aligned16(X_bf16)) return MQ_ERR_ALIGNMENT;
+    } else if ((st = check_nvfp4(X_q, M, K)) != MQ_OK) {
+        return st;
+    }
+    if ((st = check_ws(ws, ws_bytes, quantize_x ? ws_bytes_for(M, K) : kWsControlBytes)) != MQ_OK) return st;
+    DeviceInfo di;
+    if ((st = check_device(&di)) != MQ_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const Ws w = carve(ws, quantize_x ? M : 0, quantize_x ? K : 0);
+    GemmArgs g{};
+    if (quantize_x) {
+        const float* ax = nullptr;
+        st = quantize_into(X_bf16, M, K, nullptr, w.xq_codes, w.xq_scales, &w.ctrl->alpha, false, 0, w, di, s, &ax);
+        if (st != MQ_OK) return st;
+        g.a_codes = w.xq_codes;
+        g.a_scales = w.xq_scales;
+        g.a_alpha = ax;
+    } else {
+        g.a_codes = X_q->codes;
+        g.a_scales = X_q->scales;
+        g.a_alpha = X_q->alpha;
+    }
+    g.b_codes = W_kv->codes;
+    g.b_scales = W_kv->scales;
+    g.b_alpha = W_kv->alpha;
+    g.M = M;
+    g.N = N;
+    g.K = K;
+    g.epilogue = 2;
+    g.positions = positions;
+    g.cos_sin = cos_sin;
+    g.max_pos = max_pos;
+    g.slots = slots;
+    g.k_cache = static_cast<uint16_t*>(k_cache);
+    g.v_cache = static_cast<uint16_t*>(v_cache);
+    g.num_slots = num_slots;
+    g.n_heads = (int)n_kv_heads;
+    g.ctrl = w.ctrl;
+    return cuda_status(launch_gemm_nvfp4(g, di, s));
 }
 
 mq_status mq_rmsnorm_quantize(const void* X_bf16, int64_t M, int64_t K, const void* gamma_bf16, float eps,
@@ -430,6 +493,7 @@ mq_status mq_async_status(void* ws, mq_stream_t stream)
         if (cudaStreamSynchronize(s) != cudaSuccess) return MQ_ERR_CUDA;
     }
     if (bits & kErrTimeout) return MQ_ERR_TIMEOUT;
+    if (bits & kErrIndex) return MQ_ERR_INDEX;
     if (bits & kErrNonFinite) return MQ_ERR_NONFINITE;
     return MQ_OK;
 }

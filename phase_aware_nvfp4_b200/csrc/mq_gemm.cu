@@ -68,6 +68,14 @@ struct Params {
     const float* h_alpha;
     uint16_t* h_debug;
     int h_atoms;
+    const int32_t* positions;
+    const float* cos_sin;
+    int64_t max_pos;
+    const int64_t* slots;
+    uint16_t* k_cache;
+    uint16_t* v_cache;
+    int64_t num_slots;
+    int n_heads;
     WsControl* ctrl;
 };
 
@@ -147,10 +155,85 @@ __device__ __forceinline__ EpiScales epi_scales(const Params& p)
 // registers, calls release() (the accumulator may then be overwritten by the
 // next tile's MMAs), and only then stores BF16 Y, or (EPI 1) SiLU-mul ->
 // NVFP4 h codes + scales (+ optional BF16 h).
+// KV epilogue (EPI 2) for one token and one 128-column head: the projection
+// columns are K heads 0..H-1 then V heads 0..H-1.  Values are
+// fl(acc * fl(alpha_x*alpha_w)); K heads are rotated (rotate-half RoPE: pairs i,
+// i+64 with c = cos_sin[pos][i], s = cos_sin[pos][64+i], k'_i = fl(fl(k_i c) -
+// fl(k_{i+64} s)), k'_{i+64} = fl(fl(k_{i+64} c) + fl(k_i s))), then rounded to
+// BF16 and stored at cache[slot][head][0..127].  A position or slot out of
+// range posts kErrIndex and the row is not written.  acc[c][j] = column 32c + j.
+__device__ __forceinline__ void kv_rope_store(const Params& p, float alpha_ab, int64_t m, int hh,
+                                              uint32_t (&acc)[4][32])
+{
+    if (m >= p.M) return;
+    const int32_t pos = __ldg(p.positions + m);
+    const int64_t slot = __ldg(p.slots + m);
+    if (pos < 0 || pos >= p.max_pos || slot < 0 || slot >= p.num_slots) {
+        post_error(p.ctrl, kErrIndex);
+        return;
+    }
+    const bool is_k = hh < p.n_heads;
+    const int head = is_k ? hh : hh - p.n_heads;
+    if (is_k) {
+        const float4* cs = reinterpret_cast<const float4*>(p.cos_sin + (int64_t)pos * 128);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const float4 cv = __ldg(cs + 8 * c + q);        // cos of frequencies 32c + 4q .. + 3
+                const float4 sv = __ldg(cs + 16 + 8 * c + q);   // sin of the same
+                const float cc[4] = {cv.x, cv.y, cv.z, cv.w};
+                const float ss[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    const int j = 4 * q + t;
+                    const float a = __fmul_rn(__uint_as_float(acc[c][j]), alpha_ab);
+                    const float b = __fmul_rn(__uint_as_float(acc[c + 2][j]), alpha_ab);
+                    acc[c][j] = __float_as_uint(__fsub_rn(__fmul_rn(a, cc[t]), __fmul_rn(b, ss[t])));
+                    acc[c + 2][j] = __float_as_uint(__fadd_rn(__fmul_rn(b, cc[t]), __fmul_rn(a, ss[t])));
+                }
+            }
+        }
+    } else {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int j = 0; j < 32; ++j) acc[c][j] = __float_as_uint(__fmul_rn(__uint_as_float(acc[c][j]), alpha_ab));
+    }
+    uint4* dst = reinterpret_cast<uint4*>((is_k ? p.k_cache : p.v_cache) + (slot * p.n_heads + head) * 128);
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int j = 8 * q;
+            dst[4 * c + q] = make_uint4(pack_bf16x2(__uint_as_float(acc[c][j]), __uint_as_float(acc[c][j + 1])),
+                                        pack_bf16x2(__uint_as_float(acc[c][j + 2]), __uint_as_float(acc[c][j + 3])),
+                                        pack_bf16x2(__uint_as_float(acc[c][j + 4]), __uint_as_float(acc[c][j + 5])),
+                                        pack_bf16x2(__uint_as_float(acc[c][j + 6]), __uint_as_float(acc[c][j + 7])));
+        }
+}
+
 template <int EPI, class Release>
 __device__ __forceinline__ void epilogue_tile(const Params& p, const EpiScales& es, uint32_t t_row, int64_t row,
                                               int n_blk, Release release)
 {
+    if (EPI == 2) {
+        // two heads per 256-column tile; TMEM is released after the second head's loads
+        uint32_t acc[4][32];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(t_row + 128 * h + 32 * c, acc[c]);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_wait_ld(acc[c]);
+            if (h == 1) {
+                tc_fence_before();
+                release();
+            }
+            kv_rope_store(p, es.alpha_ab, row, 2 * n_blk + h, acc);
+        }
+        return;
+    }
     const int lane_ok = row < p.M;
     if (EPI == 0) {
         uint32_t out[128];
@@ -723,8 +806,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_NUM_THREADS, 1)
             const int64_t row0 = (int64_t)m_blk * 2 * BM + (int64_t)rank * BM + 32 * lg;
             if (EPI == 0) {
                 epilogue_half_bf16_tma(es, t_col, lane, stg, &tmap_y, n_blk * BN + 128 * half, (int32_t)row0, arrive);
-            } else {
+            } else if (EPI == 1) {
                 epilogue_half_mlp(p, es, t_col, half, row0 + lane, n_blk, lane, arrive);
+            } else {
+                uint32_t acc[4][32];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(t_col + 32 * c, acc[c]);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) tmem_wait_ld(acc[c]);
+                release_acc_warp(lane, arrive);
+                kv_rope_store(p, es.alpha_ab, row0 + lane, 2 * n_blk + half, acc);
             }
         }
         // every output store has finished before the CTA may leave
@@ -763,6 +854,14 @@ cudaError_t launch_gemm_nvfp4(const GemmArgs& a, const DeviceInfo& di, cudaStrea
     p.h_alpha = a.h_alpha;
     p.h_debug = a.h_debug;
     p.h_atoms = (int)sf_atoms_per_rowblk(a.N / 2);
+    p.positions = a.positions;
+    p.cos_sin = a.cos_sin;
+    p.max_pos = a.max_pos;
+    p.slots = a.slots;
+    p.k_cache = a.k_cache;
+    p.v_cache = a.v_cache;
+    p.num_slots = a.num_slots;
+    p.n_heads = a.n_heads;
     p.ctrl = a.ctrl;
 
     CUtensorMap ta, tb;
@@ -804,6 +903,11 @@ cudaError_t launch_gemm_nvfp4(const GemmArgs& a, const DeviceInfo& di, cudaStrea
             cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM_BYTES);
             if (e != cudaSuccess) return e;
             k<<<2 * pairs, P_NUM_THREADS, P_SMEM_BYTES, s>>>(ta, tb, tsfa, tsfb, ty, p);
+        } else if (a.epilogue == 2) {
+            auto k = gemm_nvfp4_pair_kernel<2>;
+            cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM_BYTES);
+            if (e != cudaSuccess) return e;
+            k<<<2 * pairs, P_NUM_THREADS, P_SMEM_BYTES, s>>>(ta, tb, tsfa, tsfb, ty, p);
         } else {
             auto k = gemm_nvfp4_pair_kernel<1>;
             cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM_BYTES);
@@ -824,6 +928,11 @@ cudaError_t launch_gemm_nvfp4(const GemmArgs& a, const DeviceInfo& di, cudaStrea
     const int grid = std::min(p.num_tiles, di.num_sms);
     if (a.epilogue == 0) {
         auto k = gemm_nvfp4_kernel<0>;
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        k<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, tb, p);
+    } else if (a.epilogue == 2) {
+        auto k = gemm_nvfp4_kernel<2>;
         cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
         if (e != cudaSuccess) return e;
         k<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, tb, p);

@@ -16,6 +16,7 @@ constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s
 // Asynchronous error bits posted by kernels into the workspace control block.
 constexpr uint32_t kErrNonFinite = 1u;  // NaN / Inf in a tensor being quantized
 constexpr uint32_t kErrTimeout = 2u;    // a pipeline wait gave up
+constexpr uint32_t kErrIndex = 4u;      // a position or cache slot out of range (KV epilogue)
 
 // Control block at the start of every workspace (zero-filled by the caller
 // once, before first use; kernels keep the counters consistent afterwards).
@@ -99,12 +100,21 @@ struct GemmArgs {
     const uint8_t* b_scales;
     const float* b_alpha;
     int64_t M, N, K;
-    int epilogue;          // 0: BF16 Y; 1: SiLU-mul + NVFP4 requantize
+    int epilogue;          // 0: BF16 Y; 1: SiLU-mul + NVFP4 requantize; 2: RoPE + KV-cache write
     void* y;               // epilogue 0: BF16 [M, N]
     uint8_t* h_codes;      // epilogue 1: [M, N/4] bytes (h has N/2 columns)
     uint8_t* h_scales;     // epilogue 1: scale layout for [M, N/2]
     const float* h_alpha;  // epilogue 1: static tensor scale of h
     uint16_t* h_debug;     // epilogue 1, optional: BF16 h [M, N/2]
+    // epilogue 2: N = 2 * n_heads * 128 columns = K heads then V heads
+    const int32_t* positions;   // [M]
+    const float* cos_sin;       // [max_pos, 128]: cos of the 64 frequencies, then sin
+    int64_t max_pos;
+    const int64_t* slots;       // [M] cache slot of each token
+    uint16_t* k_cache;          // [num_slots, n_heads, 128] BF16
+    uint16_t* v_cache;
+    int64_t num_slots;
+    int n_heads;
     WsControl* ctrl;
 };
 cudaError_t launch_gemm_nvfp4(const GemmArgs& a, const DeviceInfo& di, cudaStream_t s);

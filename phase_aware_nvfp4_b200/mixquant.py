@@ -27,13 +27,13 @@ WS_CONTROL_BYTES = 16384
 
 STATUS_NAMES = {0: "MQ_OK", 1: "MQ_ERR_INVALID_ARG", 2: "MQ_ERR_SHAPE", 3: "MQ_ERR_ALIGNMENT",
                 4: "MQ_ERR_WORKSPACE", 5: "MQ_ERR_NONFINITE", 6: "MQ_ERR_TIMEOUT", 7: "MQ_ERR_CUDA",
-                8: "MQ_ERR_DEVICE"}
+                8: "MQ_ERR_DEVICE", 9: "MQ_ERR_INDEX"}
 
 # Every symbol the header declares (checked by the ABI tests).
 EXPORTS = ("mq_status_string", "mq_version", "mq_nvfp4_sizes", "mq_workspace_bytes", "mq_quantize_weight",
            "mq_quantize_activation", "mq_prefill_linear", "mq_decode_linear", "mq_unswizzle_scales",
            "mq_async_status", "mq_prefill_linear_noalloc", "mq_selftest_e2m1", "mq_selftest_timeout",
-           "mq_decode_linear_nvfp4", "mq_quantize", "mq_rmsnorm_quantize")
+           "mq_decode_linear_nvfp4", "mq_quantize", "mq_rmsnorm_quantize", "mq_prefill_kv_rope")
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
@@ -93,6 +93,8 @@ def load(path: str = LIB_PATH):
             lib.mq_quantize.restype = i32
             lib.mq_rmsnorm_quantize.argtypes = [vp, i64, i64, vp, ctypes.c_float, nvp, vp, vp, sz, vp]
             lib.mq_rmsnorm_quantize.restype = i32
+            lib.mq_prefill_kv_rope.argtypes = [vp, nvp, i64, nvp, i64, vp, vp, i64, vp, vp, vp, i64, vp, sz, vp]
+            lib.mq_prefill_kv_rope.restype = i32
             lib.mq_prefill_linear_noalloc.argtypes = [vp, i64, nvp, vp, vp, vp]
             lib.mq_prefill_linear_noalloc.restype = i32
             _lib = lib
@@ -193,6 +195,23 @@ def quantize(X, alpha_static=None, gate_up_interleave: bool = False, scale_searc
     _check(load().mq_quantize(_ptr(X), rows, K, _ptr(alpha_static), flags, ctypes.byref(oc), *_ws_args(ws),
                               _stream(stream)), "mq_quantize")
     return out
+
+
+def prefill_kv_rope(X=None, W: NVFP4Tensor = None, *, Xq: NVFP4Tensor | None = None, n_kv_heads: int,
+                    positions, cos_sin, slots, k_cache, v_cache, ws=None, stream=None):
+    """mq_prefill_kv_rope: K/V projection with RoPE on K, BF16 K/V written to cache slots."""
+    if (X is None) == (Xq is None):
+        raise ValueError("give exactly one of X (BF16) and Xq (NVFP4)")
+    M = X.shape[0] if X is not None else Xq.rows
+    dev = W.codes.device
+    if ws is None:
+        ws = workspace(M, W.cols, dev) if X is not None else workspace(device=dev)
+    xq_c = Xq.c() if Xq is not None else None
+    w_c = W.c()
+    _check(load().mq_prefill_kv_rope(_ptr(X), ctypes.byref(xq_c) if xq_c is not None else None, M,
+                                     ctypes.byref(w_c), n_kv_heads, _ptr(positions), _ptr(cos_sin),
+                                     cos_sin.shape[0], _ptr(slots), _ptr(k_cache), _ptr(v_cache), k_cache.shape[0],
+                                     *_ws_args(ws), _stream(stream)), "mq_prefill_kv_rope")
 
 
 def rmsnorm_quantize(X, gamma, eps: float = 1e-6, out: NVFP4Tensor | None = None, h_debug=None, ws=None,

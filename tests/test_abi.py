@@ -116,6 +116,16 @@ def test_argument_errors_are_synchronous(lib):
     assert lib.mq_rmsnorm_quantize(P, 128, 200, P, ctypes.c_float(1e-6), ctypes.byref(rq), None, ws, wsb, None) == 2
     assert lib.mq_rmsnorm_quantize(P, 128, 256, P + 8, ctypes.c_float(1e-6), ctypes.byref(rq), None, ws, wsb,
                                    None) == 3
+    # K/V projection with RoPE: W rows = 2 * heads * 128, index arrays and caches required/aligned
+    wkv = _nv(512, 256)
+    args = lambda X, heads, pos, cs, sl, kc: (X, None, 128, ctypes.byref(wkv), heads, pos, cs, 1024, sl, kc, P,
+                                               4096, ws, wsb, None)
+    assert lib.mq_prefill_kv_rope(*args(P, 3, P, P, P, P)) == 2             # 2 * 3 * 128 != 512
+    assert lib.mq_prefill_kv_rope(*args(P, 2, None, P, P, P)) == 1
+    assert lib.mq_prefill_kv_rope(*args(P, 2, P + 2, P, P, P)) == 3          # positions 4-byte aligned
+    assert lib.mq_prefill_kv_rope(*args(P, 2, P, P, P + 4, P)) == 3          # slots 8-byte aligned
+    assert lib.mq_prefill_kv_rope(*args(P, 2, P, P + 4, P, P)) == 3          # cos/sin 16-byte aligned
+    assert lib.mq_prefill_kv_rope(*args(None, 2, P, P, P, P)) == 1           # neither X nor X_q
     # timeout self-test: timeout in (0, 2 s], a workspace, an aligned result slot
     assert lib.mq_selftest_timeout(ws, wsb, ctypes.c_uint64(0), None, None) == 1
     assert lib.mq_selftest_timeout(ws, wsb, ctypes.c_uint64(3 * 10 ** 9), None, None) == 1
