@@ -506,6 +506,50 @@ def measure_extras(mq, torch, dev, flush, hbm_gbs, fp4_peak, reps=10):
     return out
 
 
+def measure_library_gemm(torch, w, Wq, Xq, Y, flush, fp4_peak, reps=10):
+    """Same-box context number: torch's block-scaled NVFP4 matmul (a library
+    kernel) on the very operands the projection step quantized -- codes, E4M3
+    block scales in the MMA scale layout (the "32_4_4" swizzle), and the FP32
+    tensor scales -- timed like the step's GEMMs (L2 flushed before each call),
+    with its output compared to the step's BF16 output as a cross-check."""
+    import torch.nn.functional as F
+    if not hasattr(torch, "float4_e2m1fn_x2") or not hasattr(F, "scaled_mm"):
+        return {"unavailable": "this torch build has no NVFP4 scaled_mm"}
+    ST, SW = F.ScalingType, F.SwizzleType
+
+    def operands(t):
+        rows, k16 = -(-t.rows // 128) * 128, -(-(t.cols // 16) // 4) * 4
+        if t.scales.numel() != rows * k16:
+            raise ValueError(f"scale buffer of {t.scales.numel()} bytes is not the library's {rows} x {k16}")
+        return t.codes.view(torch.float4_e2m1fn_x2), t.scales.view(torch.float8_e4m3fn)
+
+    out = {}
+    for p in w.projections:
+        xq, wq = Xq[p.x_group], Wq[p.name]
+        try:
+            a, sa = operands(xq)
+            b, sb = operands(wq)
+
+            def call(a=a, b=b, sa=sa, sb=sb, xq=xq, wq=wq):
+                return F.scaled_mm(a, b.t(), [sa, xq.alpha], [ST.BlockWise1x16, ST.TensorWise],
+                                   [sb, wq.alpha], [ST.BlockWise1x16, ST.TensorWise],
+                                   swizzle_a=[SW.SWIZZLE_32_4_4, SW.NO_SWIZZLE],
+                                   swizzle_b=[SW.SWIZZLE_32_4_4, SW.NO_SWIZZLE], output_dtype=torch.bfloat16)
+            yl = call()
+            torch.cuda.synchronize()
+            yo = Y[p.name].double()
+            rel = float(torch.linalg.norm(yl.double() - yo) / torch.linalg.norm(yo))
+            del yl
+            for _ in range(3):
+                call()
+            ms = _time_calls(torch, call, reps, flush)
+            tf = p.flops / (ms * 1e-3) / 1e12
+            out[p.name] = {"ms": ms, "TFLOP/s": tf, "frac": tf / fp4_peak, "rel_frobenius_vs_ours": rel}
+        except Exception as e:     # the library's own argument checks; reported, not fatal
+            out[p.name] = {"unavailable": f"{type(e).__name__}: {str(e).splitlines()[0][:200]}"}
+    return out
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -671,6 +715,7 @@ def run_gpu(args):
 
     if not args.no_extras:
         line["extras"] = measure_extras(mq, torch, dev, flush, hbm_gbs, fp4_peak)
+        line["extras"]["library_nvfp4_gemm"] = measure_library_gemm(torch, w, Wq, Xq, Y, flush, fp4_peak)
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res = time_oracle(w, xs_h, ws_h, args.cpu_baseline_seconds, steps=1)
