@@ -108,20 +108,38 @@ class ClockSampler:
                0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
                0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
 
-    def __init__(self, index: int, period_s: float = 0.005):
+    def __init__(self, index: int, period_s: float = 0.005, pci=None, nvml=None):
+        """index: NVML index to use when no NVML device matches `pci`, the
+        (domain, bus, device) PCI address of the CUDA device being timed (NVML
+        enumerates every GPU of the node, CUDA only the visible ones)."""
         self.period = period_s
         self.samples, self.reasons = [], set()
         self.max_mhz = None
+        self.match = None
         self._stop = threading.Event()
         self._t = None
         try:
-            import pynvml
-            pynvml.nvmlInit()
-            self.nv = pynvml
-            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
-            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            if nvml is None:
+                import pynvml as nvml
+            nvml.nvmlInit()
+            self.nv = nvml
+            self.h, self.match = self._handle(nvml, index, pci)
+            self.max_mhz = nvml.nvmlDeviceGetMaxClockInfo(self.h, nvml.NVML_CLOCK_SM)
         except Exception:
             self.nv = None
+
+    @staticmethod
+    def _handle(nv, index, pci):
+        if pci is not None:
+            try:
+                for i in range(nv.nvmlDeviceGetCount()):
+                    h = nv.nvmlDeviceGetHandleByIndex(i)
+                    info = nv.nvmlDeviceGetPciInfo(h)
+                    if (int(info.domain), int(info.bus), int(info.device)) == tuple(int(v) for v in pci):
+                        return h, "pci"
+            except Exception:
+                pass
+        return nv.nvmlDeviceGetHandleByIndex(index), "index"
 
     def _run(self):
         nv = self.nv
@@ -151,7 +169,8 @@ class ClockSampler:
         if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
         return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples),
+                "nvml_device": self.match}
 
 
 # ---------------------------------------------------------------- multi-rank aggregation
@@ -623,7 +642,9 @@ def run_gpu(args):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else local) as clk:
+    props = torch.cuda.get_device_properties(dev)
+    with ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else local,
+                      pci=(props.pci_domain_id, props.pci_bus_id, props.pci_device_id)) as clk:
         for i in range(K):
             flush()
             step_ev[i][0].record()

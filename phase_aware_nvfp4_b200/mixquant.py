@@ -7,8 +7,12 @@ computes anything itself and has no fallback: if ``libmixquant.so`` is
 missing or a call returns an error, it raises.
 
 Names mirror the C ABI: ``quantize_weight``, ``quantize_activation``,
-``prefill_linear``, ``decode_linear``, ``unswizzle_scales``,
-``async_status``, ``nvfp4_sizes``, ``workspace_bytes``.
+``quantize`` (general entry: gate/up interleave, opt-in scale search),
+``prefill_linear`` (BF16 or fused SiLU-mul + NVFP4 epilogue),
+``prefill_linear_noalloc``, ``prefill_kv_rope``, ``rmsnorm_quantize``,
+``decode_linear`` (BF16), ``decode_linear_nvfp4``, ``unswizzle_scales``,
+``async_status``, ``selftest_e2m1``, ``selftest_timeout``, ``nvfp4_sizes``,
+``workspace_bytes``.
 """
 from __future__ import annotations
 
