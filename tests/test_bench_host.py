@@ -68,3 +68,21 @@ def test_sampler_without_nvml_reports_no_samples():
     with bench.ClockSampler(0, pci=(0, 0x1B, 0), nvml=Broken([], [], [])) as clk:
         pass
     assert clk.summary()["samples"] == 0 and clk.summary()["sm_mhz"] is None
+
+
+def test_reference_arm_prints_one_contract_line(capsys, monkeypatch):
+    """`bench.py --impl reference` (the oracle on the host cores) on rank 0: one JSON line with the
+    contract's keys, the same metric and workload as the GPU arm, and zero host-device bytes."""
+    import json
+    monkeypatch.setenv("RANK", "0")
+    args = bench.parse_args(["--impl", "reference", "--steps", "1", "--warmup", "0", "--M", "256"])
+    assert bench.run_reference(args) == 0
+    lines = [l for l in capsys.readouterr().out.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == bench.UNIT
+    assert d["higher_is_better"] is True and d["value"] > 0 and d["steps"] == 1
+    assert d["config"]["workload"].startswith("qwen3_8b_projections") and d["config"]["M"] == 256
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
