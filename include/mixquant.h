@@ -25,7 +25,8 @@
  *     mq_async_status().
  *   - BF16 tensors are row-major with a 16-byte aligned base.
  *   - Shapes: K (the reduction dimension) is a multiple of 64; N is a
- *     multiple of 16 (128 for the fused MLP epilogue); M >= 1.
+ *     multiple of 16 (128 for the fused MLP epilogue); M >= 1; M, N and K
+ *     are at most 2^30 (MQ_ERR_SHAPE beyond).
  *
  * NVFP4 tensor storage (mq_nvfp4), for a logical [rows, cols] matrix:
  *   codes   rows x cols/2 bytes, row-major; element k of a row is in byte

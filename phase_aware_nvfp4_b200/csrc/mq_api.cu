@@ -121,6 +121,10 @@ Ws carve(void* ws, int64_t M, int64_t K)
     return w;
 }
 
+// Largest M, N or K any call accepts: keeps every byte offset and element count
+// far inside 64 bits and every tensor-map coordinate inside 32 bits.
+constexpr int64_t kMaxDim = (int64_t)1 << 30;
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 mq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MQ_OK : MQ_ERR_CUDA; }
@@ -207,7 +211,7 @@ mq_status mq_quantize_weight(const void* W_bf16, int64_t N, int64_t K, int gate_
                              void* ws, size_t ws_bytes, mq_stream_t stream)
 {
     if (W_bf16 == nullptr) return MQ_ERR_INVALID_ARG;
-    if (N < 1 || K < 64 || K % 64 != 0) return MQ_ERR_SHAPE;
+    if (N < 1 || K < 64 || K % 64 != 0 || N > kMaxDim || K > kMaxDim) return MQ_ERR_SHAPE;
     if (gate_up_interleave && (N % 128 != 0)) return MQ_ERR_SHAPE;
     if (!aligned16(W_bf16)) return MQ_ERR_ALIGNMENT;
     mq_status st = check_nvfp4(out, N, K);
@@ -224,7 +228,7 @@ mq_status mq_quantize_activation(const void* X_bf16, int64_t M, int64_t K, const
                                  const mq_nvfp4* out, void* ws, size_t ws_bytes, mq_stream_t stream)
 {
     if (X_bf16 == nullptr) return MQ_ERR_INVALID_ARG;
-    if (M < 1 || K < 64 || K % 64 != 0) return MQ_ERR_SHAPE;
+    if (M < 1 || K < 64 || K % 64 != 0 || M > kMaxDim || K > kMaxDim) return MQ_ERR_SHAPE;
     if (!aligned16(X_bf16)) return MQ_ERR_ALIGNMENT;
     mq_status st = check_nvfp4(out, M, K);
     if (st != MQ_OK) return st;
@@ -241,7 +245,7 @@ mq_status mq_quantize(const void* X_bf16, int64_t rows, int64_t K, const float* 
 {
     if (X_bf16 == nullptr) return MQ_ERR_INVALID_ARG;
     if ((flags & ~(unsigned)(MQ_QUANT_GATE_UP_INTERLEAVE | MQ_QUANT_SCALE_SEARCH)) != 0) return MQ_ERR_INVALID_ARG;
-    if (rows < 1 || K < 64 || K % 64 != 0) return MQ_ERR_SHAPE;
+    if (rows < 1 || K < 64 || K % 64 != 0 || rows > kMaxDim || K > kMaxDim) return MQ_ERR_SHAPE;
     const bool interleave = (flags & MQ_QUANT_GATE_UP_INTERLEAVE) != 0;
     if (interleave && rows % 128 != 0) return MQ_ERR_SHAPE;
     if (!aligned16(X_bf16)) return MQ_ERR_ALIGNMENT;
@@ -268,7 +272,7 @@ mq_status mq_prefill_kv_rope(const void* X_bf16, const mq_nvfp4* X_q, int64_t M,
         return MQ_ERR_INVALID_ARG;
     const int64_t N = W_kv->rows, K = W_kv->cols;
     if (n_kv_heads < 1 || n_kv_heads > 4096 || N != 2 * n_kv_heads * 128) return MQ_ERR_SHAPE;
-    if (M < 1 || M > (int64_t)1 << 30 || K < 64 || K % 64 != 0 || K > (int64_t)1 << 30) return MQ_ERR_SHAPE;
+    if (M < 1 || M > kMaxDim || K < 64 || K % 64 != 0 || K > kMaxDim) return MQ_ERR_SHAPE;
     if (max_pos < 1 || num_slots < 1) return MQ_ERR_SHAPE;
     if (!aligned16(cos_sin) || !aligned16(k_cache) || !aligned16(v_cache) ||
         (reinterpret_cast<uintptr_t>(positions) & 3u) || (reinterpret_cast<uintptr_t>(slots) & 7u))
@@ -323,7 +327,7 @@ mq_status mq_rmsnorm_quantize(const void* X_bf16, int64_t M, int64_t K, const vo
 {
     if (X_bf16 == nullptr || gamma_bf16 == nullptr) return MQ_ERR_INVALID_ARG;
     if (!(eps >= 0.0f) || eps > 3.0e38f) return MQ_ERR_INVALID_ARG;
-    if (M < 1 || M > (int64_t)1 << 30 || K < 64 || K % 64 != 0 || K > (int64_t)1 << 30) return MQ_ERR_SHAPE;
+    if (M < 1 || M > kMaxDim || K < 64 || K % 64 != 0 || K > kMaxDim) return MQ_ERR_SHAPE;
     if (!aligned16(X_bf16) || !aligned16(gamma_bf16) || (h_debug != nullptr && !aligned16(h_debug)))
         return MQ_ERR_ALIGNMENT;
     mq_status st = check_nvfp4(out, M, K);
@@ -346,8 +350,8 @@ mq_status mq_prefill_linear(const void* X_bf16, const mq_nvfp4* X_q, int64_t M, 
     if (W == nullptr || W->codes == nullptr || W->scales == nullptr || W->alpha == nullptr) return MQ_ERR_INVALID_ARG;
     if (epi != MQ_EPI_BF16 && epi != MQ_EPI_SILU_MUL_NVFP4) return MQ_ERR_INVALID_ARG;
     const int64_t N = W->rows, K = W->cols;
-    if (M < 1 || M > (int64_t)1 << 30 || K < 64 || K % 64 != 0 || N < 16 || N % 16 != 0) return MQ_ERR_SHAPE;
-    if (N > (int64_t)1 << 30 || K > (int64_t)1 << 30) return MQ_ERR_SHAPE;
+    if (M < 1 || M > kMaxDim || K < 64 || K % 64 != 0 || N < 16 || N % 16 != 0) return MQ_ERR_SHAPE;
+    if (N > kMaxDim || K > kMaxDim) return MQ_ERR_SHAPE;
     mq_status st = check_nvfp4(W, N, K);
     if (st != MQ_OK) return st;
     if (epi == MQ_EPI_BF16) {
@@ -410,7 +414,7 @@ mq_status mq_decode_linear(const void* X_bf16, int64_t M, const void* W_bf16, in
 {
     if (X_bf16 == nullptr || W_bf16 == nullptr || Y_bf16 == nullptr) return MQ_ERR_INVALID_ARG;
     if (M < 1 || M > 256 || N < 16 || N % 16 != 0 || K < 64 || K % 64 != 0) return MQ_ERR_SHAPE;
-    if (N > (int64_t)1 << 30 || K > (int64_t)1 << 30) return MQ_ERR_SHAPE;
+    if (N > kMaxDim || K > kMaxDim) return MQ_ERR_SHAPE;
     if (!aligned16(X_bf16) || !aligned16(W_bf16) || !aligned16(Y_bf16)) return MQ_ERR_ALIGNMENT;
     mq_status st = check_ws(ws, ws_bytes, kWsControlBytes);
     if (st != MQ_OK) return st;
@@ -428,7 +432,7 @@ mq_status mq_decode_linear_nvfp4(const void* X_bf16, int64_t M, const mq_nvfp4* 
     if (W == nullptr || W->codes == nullptr || W->scales == nullptr || W->alpha == nullptr) return MQ_ERR_INVALID_ARG;
     const int64_t N = W->rows, K = W->cols;
     if (M < 1 || M > 128 || N < 16 || N % 16 != 0 || K < 64 || K % 64 != 0) return MQ_ERR_SHAPE;
-    if (N > (int64_t)1 << 30 || K > (int64_t)1 << 30) return MQ_ERR_SHAPE;
+    if (N > kMaxDim || K > kMaxDim) return MQ_ERR_SHAPE;
     mq_status st = check_nvfp4(W, N, K);
     if (st != MQ_OK) return st;
     if (!aligned16(X_bf16) || !aligned16(Y_bf16)) return MQ_ERR_ALIGNMENT;

@@ -126,6 +126,16 @@ def test_argument_errors_are_synchronous(lib):
     assert lib.mq_prefill_kv_rope(*args(P, 2, P, P, P + 4, P)) == 3          # slots 8-byte aligned
     assert lib.mq_prefill_kv_rope(*args(P, 2, P, P + 4, P, P)) == 3          # cos/sin 16-byte aligned
     assert lib.mq_prefill_kv_rope(*args(None, 2, P, P, P, P)) == 1           # neither X nor X_q
+    # sizes beyond 2^30 in any dimension are refused by every entry point
+    big, bigk = (1 << 30) + 128, (1 << 30) + 64
+    ob = _nv(big, 256)
+    assert lib.mq_quantize_weight(P, big, 256, 0, ctypes.byref(ob), ws, wsb, None) == 2
+    assert lib.mq_quantize_weight(P, 256, bigk, 0, ctypes.byref(_nv(256, bigk)), ws, wsb, None) == 2
+    assert lib.mq_quantize_activation(P, big, 256, None, ctypes.byref(ob), ws, wsb, None) == 2
+    assert lib.mq_quantize(P, big, 256, None, ctypes.c_uint(0), ctypes.byref(ob), ws, wsb, None) == 2
+    assert lib.mq_prefill_linear(P, None, big, ctypes.byref(w), 0, None, None, P, None, None, ws, wsb, None) == 2
+    assert lib.mq_decode_linear(P, 4, P, big, 256, P, ws, wsb, None) == 2
+    assert lib.mq_rmsnorm_quantize(P, big, 256, P, ctypes.c_float(1e-6), ctypes.byref(ob), None, ws, wsb, None) == 2
     # timeout self-test: timeout in (0, 2 s], a workspace, an aligned result slot
     assert lib.mq_selftest_timeout(ws, wsb, ctypes.c_uint64(0), None, None) == 1
     assert lib.mq_selftest_timeout(ws, wsb, ctypes.c_uint64(3 * 10 ** 9), None, None) == 1
