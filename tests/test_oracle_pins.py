@@ -546,3 +546,52 @@ def test_rope_scores_depend_only_on_relative_position():
         if delta >= 60:   # shifting only one side does change the score, well beyond the rounding noise
             c = _rope_f64(qs, np.array([p]), cs32)[0] @ _rope_f64(ks, np.array([pp + delta]), cs32)[0]
             assert abs(a - c) > 10 * abs(a - b)
+
+
+def test_rope_is_complex_multiplication_by_the_position_phase():
+    """Rotary embedding read as complex arithmetic: pairing channel i with i + 64 as
+    z_i = k_i + j k_{i+64}, position p multiplies z_i by exp(j p f_i), f_i = 1e6^(-2i/128).
+    numpy's complex product (from angles in float64, not the table) fixes the rotation's
+    direction and pairing, which the relative-position property alone does not: rotating
+    the other way, or pairing i with i + 1, keeps that property but fails here."""
+    rng = np.random.default_rng(73)
+    cs = wl.rope_cos_sin(4096)
+    f = 1.0e6 ** (-2.0 * np.arange(64) / 128)
+    yk = rng.standard_normal((6, 256))                        # two heads
+    pos = np.array([0, 1, 2, 17, 1000, 4095])
+    mine = _rope_f64(yk, pos, cs).reshape(6, 2, 128)
+    z = yk.reshape(6, 2, 2, 64)
+    zc = (z[:, :, 0] + 1j * z[:, :, 1]) * np.exp(1j * pos[:, None, None] * f[None, None, :])
+    ref = np.concatenate([zc.real, zc.imag], axis=2)           # [6, 2, 128]
+    bound = oracle.bf16_ulp(ref) + 1e-6 * (np.abs(z[:, :, 0]) + np.abs(z[:, :, 1])).repeat(2, axis=2)
+    assert np.all(np.abs(mine - ref) <= bound)
+    # closed form at position 1, frequency 0 (f_0 = 1): e_0 turns into (cos 1, sin 1)
+    e0 = np.zeros((1, 128))
+    e0[0, 0] = 1.0
+    r = _rope_f64(e0, np.array([1]), cs)[0]
+    assert r[0] == oracle.bf16_to_f64(oracle.round_bf16(np.array([np.cos(1.0)])))[0]
+    assert r[64] == oracle.bf16_to_f64(oracle.round_bf16(np.array([np.sin(1.0)])))[0]
+    assert np.count_nonzero(r) == 2
+
+
+@pytest.mark.parametrize("mistake", ["opposite_direction", "adjacent_pairs"])
+def test_rope_pin_catches_planted_mistakes(monkeypatch, mistake):
+    """Plant a plausible slip in the oracle's rotation (CPU only) and check that the
+    complex-multiplication pin fails: rotating by -p f_i (sin sign flipped), or pairing
+    channel i with i + 1 instead of i + 64."""
+    orig = oracle.kv_rope_rows
+
+    def planted(yk, yv, positions, cos_sin, head_dim=128):
+        yk = np.asarray(yk, dtype=np.float64)
+        if mistake == "opposite_direction":
+            cs = np.array(cos_sin, dtype=np.float32)
+            cs[:, head_dim // 2:] *= -1
+            return orig(yk, yv, positions, cs, head_dim)
+        M, n = yk.shape
+        k = yk.reshape(M, n // head_dim, head_dim // 2, 2).transpose(0, 1, 3, 2).reshape(M, n)
+        kr, v = orig(k, yv, positions, cos_sin, head_dim)
+        return kr.reshape(M, n // head_dim, 2, head_dim // 2).transpose(0, 1, 3, 2).reshape(M, n), v
+
+    monkeypatch.setattr(oracle, "kv_rope_rows", planted)
+    with pytest.raises(AssertionError):
+        test_rope_is_complex_multiplication_by_the_position_phase()
