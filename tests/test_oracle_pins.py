@@ -595,3 +595,22 @@ def test_rope_pin_catches_planted_mistakes(monkeypatch, mistake):
     monkeypatch.setattr(oracle, "kv_rope_rows", planted)
     with pytest.raises(AssertionError):
         test_rope_is_complex_multiplication_by_the_position_phase()
+
+
+def test_rmsnorm_eps_enters_under_the_root_and_the_mean_divides_by_k():
+    """Closed forms where eps is as large as the mean square, so that eps outside the root
+    (1/(sqrt(ms) + eps)) or a mean over K - 1 would change the result far beyond rounding."""
+    K = 256
+    g = wl.f32_to_bf16_bits(np.ones(K, np.float32))
+    # x = 2^-10 everywhere, eps = 2^-20: ms = 2^-20 exactly, ms + eps = 2^-19, rstd = 2^9.5
+    x = wl.f32_to_bf16_bits(np.full((1, K), 2.0 ** -10, np.float32))
+    h, r = oracle.rmsnorm(x, g, 2.0 ** -20)
+    assert r[0] == np.float32(2.0 ** 9.5)
+    t = np.float32(np.float32(2.0 ** -10) * np.float32(2.0 ** 9.5))        # fl32(x * rstd), gamma = 1
+    assert np.all(h[0] == oracle.round_bf16(np.array([float(t)]))[0])
+    # one non-zero element 16 in a row of K: ms = 256 / K = 1 exactly, eps = 3 -> rstd = 1/2
+    x = np.zeros((1, K), np.float32)
+    x[0, 5] = 16.0
+    h, r = oracle.rmsnorm(wl.f32_to_bf16_bits(x), g, 3.0)
+    assert r[0] == np.float32(0.5)
+    assert wl.bf16_bits_to_f32(h)[0, 5] == 8.0 and np.count_nonzero(wl.bf16_bits_to_f32(h)) == 1
