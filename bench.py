@@ -385,6 +385,9 @@ def measure_extras(mq, torch, dev, flush, hbm_gbs, fp4_peak, reps=10):
         q4 = [lambda W=W: mq.decode_linear_nvfp4(x, W, Y=y, ws=wsd) for W in Wq_copies]
         for f in bf + q4:
             f()
+        # the set-up above leaves the GPU idle for a while: ~50 ms of spinning first,
+        # so the timed calls do not start on a clock that is still ramping up
+        torch.cuda._sleep(100_000_000)
         ms = _time_rotating(torch, bf, 4 * reps)
         gbs = (2 * N * K + 2 * M * K + 2 * M * N) / (ms * 1e-3) / 1e9
         dec[str(M)] = {"ms": ms, "GB/s": gbs, "frac": gbs / hbm_gbs}
