@@ -51,7 +51,7 @@ FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 GEMM_SOURCES = ("phase_aware_nvfp4_b200/csrc/mq_gemm.cu", "phase_aware_nvfp4_b200/csrc/mq_device.cuh")
 QUANT_SOURCES = ("phase_aware_nvfp4_b200/csrc/mq_quant.cu", "phase_aware_nvfp4_b200/csrc/mq_device.cuh")
-COUNTERS = os.path.join(ROOT, "profiles", "ncu_counters.json")
+COUNTERS = os.path.join(ROOT, "profiles", "ncu_dram_bytes_gemm_and_quantizer_qwen3_8b_projections_M8192.json")
 
 
 def parse_args(argv=None):
