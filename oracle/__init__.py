@@ -16,10 +16,16 @@ Layering:
   * ``mq_oracle.c`` (compiled to ``liboracle.so``) holds the per-element
     arithmetic: E2M1 / E4M3 encode (exhaustive nearest search) and decode,
     the tensor scale, block quantization, dequantization, BF16 rounding and
-    the SiLU-mul of the MLP.
+    the SiLU-mul of the MLP; the opt-in per-block scale search (the paper's
+    "scale optimization", read as trying the Eq. 3 scale code and its two
+    E4M3 neighbours); and RMSNorm with its BF16 output (the producer of the
+    quantized activation).
   * The matmuls are numpy float64 ``@`` on the dequantized operands (a library
     primitive used as one step), followed by the tensor scales and BF16
     rounding in C.
+  * ``kv_rope_rows`` applies rotate-half rotary embedding to the K projection
+    output in float64 and rounds K and V to BF16 (the KV cache in the decode
+    precision, "Prefill-Decode Disaggregation Deployment").
 
 Every function here has at least one pin in ``tests/test_oracle_pins.py``
 against facts fixed by the format definitions or the mathematics (closed
