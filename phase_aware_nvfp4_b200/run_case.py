@@ -4,6 +4,7 @@
     python -m phase_aware_nvfp4_b200.run_case gemm   --M 8192  --N 12288 --K 4096
     python -m phase_aware_nvfp4_b200.run_case mlp    --M 8192  --N 24576 --K 4096
     python -m phase_aware_nvfp4_b200.run_case decode --M 1     --N 24576 --K 4096
+    python -m phase_aware_nvfp4_b200.run_case kv_rope --M 8192 --N 2048  --K 4096
 
 Inputs are prepared (and weights quantized) before the profiled calls; each
 iteration then launches only the operation named:
@@ -17,7 +18,10 @@ iteration then launches only the operation named:
 * ``decode``: the BF16 decode GEMM Y = X W^T (M <= 256);
 * ``decode_nvfp4``: the uniform-NVFP4 decode (tokens quantized on the fly,
   NVFP4 weight; M <= 128);
-* ``rmsnorm_quant``: RMSNorm fused with the NVFP4 quantization of its output.
+* ``rmsnorm_quant``: RMSNorm fused with the NVFP4 quantization of its output;
+* ``kv_rope``: the K/V projection (N = 2 x heads x 128, X already quantized)
+  with RoPE on the K heads and the BF16 KV-cache write in the GEMM epilogue;
+  positions uniform in [0, 40960), slots a permutation of the tokens.
 
 Prints the mean CUDA-event time per iteration.  The data recipe is the one the
 tests and the benchmark use (Student-t(3) activations with 1 % outlier
@@ -33,7 +37,7 @@ import numpy as np
 
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
-    ap.add_argument("op", choices=["quant", "gemm", "mlp", "decode", "decode_nvfp4", "rmsnorm_quant"])
+    ap.add_argument("op", choices=["quant", "gemm", "mlp", "decode", "decode_nvfp4", "rmsnorm_quant", "kv_rope"])
     ap.add_argument("--M", type=int, default=8192)
     ap.add_argument("--N", type=int, default=4096)
     ap.add_argument("--K", type=int, default=4096)
@@ -71,6 +75,20 @@ def main(argv=None) -> int:
             H = mq.nvfp4_empty(a.M, a.N // 2, dev)
             ah = torch.full((1,), 0.25, dtype=torch.float32, device=dev)
             run = lambda: mq.prefill_linear(W=Wq, Xq=Xq, epilogue=mq.MQ_EPI_SILU_MUL_NVFP4, alpha_h=ah, H=H, ws=ws)
+    elif a.op == "kv_rope":
+        if a.N % 256 != 0:
+            raise SystemExit("kv_rope needs N = 2 x heads x 128")
+        heads, max_pos = a.N // 256, 40960
+        Wq = mq.quantize_weight(dev_bf16(wl.normal_bf16(a.N, a.K, 0.02, 12)), ws=ws)
+        Xq = mq.quantize_activation(X, ws=ws)
+        cs = torch.from_numpy(wl.rope_cos_sin(max_pos)).to(dev)
+        rng = np.random.default_rng(14)
+        pos = torch.from_numpy(rng.integers(0, max_pos, size=a.M).astype(np.int32)).to(dev)
+        slots = torch.from_numpy(rng.permutation(a.M).astype(np.int64)).to(dev)
+        kc = torch.empty((a.M, heads, 128), dtype=torch.bfloat16, device=dev)
+        vc = torch.empty_like(kc)
+        run = lambda: mq.prefill_kv_rope(W=Wq, Xq=Xq, n_kv_heads=heads, positions=pos, cos_sin=cs, slots=slots,
+                                         k_cache=kc, v_cache=vc, ws=ws)
     elif a.op == "decode":
         W = dev_bf16(wl.normal_bf16(a.N, a.K, 0.02, 12))
         Y = torch.empty((a.M, a.N), dtype=torch.bfloat16, device=dev)
