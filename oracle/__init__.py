@@ -282,10 +282,20 @@ def num_threads() -> int:
 # --------------------------------------------------------------------------
 
 def rel_frobenius(y: np.ndarray, y_ref: np.ndarray) -> float:
-    y = np.asarray(y, dtype=np.float64)
-    y_ref = np.asarray(y_ref, dtype=np.float64)
-    den = np.linalg.norm(y_ref)
-    return float(np.linalg.norm(y - y_ref) / den) if den > 0 else float(np.linalg.norm(y - y_ref))
+    """Relative Frobenius error ||y - y_ref||_F / ||y_ref||_F over all elements, in float64.
+
+    The denominator is the reference's norm.  A zero reference has no relative
+    scale: the result is 0 when y is zero as well and +inf otherwise, so a gate
+    on it fails for any deviation instead of turning into an absolute one.
+    """
+    y = np.asarray(y, dtype=np.float64).ravel()
+    y_ref = np.asarray(y_ref, dtype=np.float64).ravel()
+    assert y.shape == y_ref.shape, f"shapes differ: {y.shape} vs {y_ref.shape}"
+    num = float(np.linalg.norm(y - y_ref))
+    den = float(np.linalg.norm(y_ref))
+    if den > 0:
+        return num / den
+    return 0.0 if num == 0 else float("inf")
 
 
 def bf16_ulp(v: np.ndarray) -> np.ndarray:

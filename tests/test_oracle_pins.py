@@ -614,3 +614,48 @@ def test_rmsnorm_eps_enters_under_the_root_and_the_mean_divides_by_k():
     h, r = oracle.rmsnorm(wl.f32_to_bf16_bits(x), g, 3.0)
     assert r[0] == np.float32(0.5)
     assert wl.bf16_bits_to_f32(h)[0, 5] == 8.0 and np.count_nonzero(wl.bf16_bits_to_f32(h)) == 1
+
+
+# ------------------------------------------------------------------ the error metric behind every tolerance gate
+
+def test_rel_frobenius_closed_forms():
+    """Closed forms of ||y - y_ref||_F / ||y_ref||_F (exact in binary64 for these integers):
+    a doubled reference gives exactly 1; an error orthogonal to the reference gives
+    ||e|| / ||y_ref|| (12/5 here) and NOT ||e|| / ||y|| (12/13), its square (144/25) or its
+    root; the norm runs over all elements of a matrix (1/sqrt(26)), not per row; a zero
+    reference gives 0 for a zero output and +inf otherwise."""
+    y_ref = np.array([0.0, 3.0, 4.0])
+    assert oracle.rel_frobenius(y_ref, y_ref) == 0.0
+    assert oracle.rel_frobenius(2.0 * y_ref, y_ref) == 1.0
+    assert oracle.rel_frobenius(y_ref + np.array([12.0, 0.0, 0.0]), y_ref) == 12.0 / 5.0
+    assert oracle.rel_frobenius(y_ref, y_ref + np.array([12.0, 0.0, 0.0])) == 12.0 / 13.0   # not symmetric
+    m_ref = np.array([[3.0, 4.0], [0.0, 1.0]])
+    m = m_ref + np.array([[0.0, 0.0], [1.0, 0.0]])
+    assert abs(oracle.rel_frobenius(m, m_ref) - 1.0 / math.sqrt(26.0)) <= 1e-16
+    assert oracle.rel_frobenius(np.zeros(4), np.zeros(4)) == 0.0
+    assert oracle.rel_frobenius(np.array([0.0, 1e-30, 0.0, 0.0]), np.zeros(4)) == math.inf
+
+
+@pytest.mark.parametrize("mistake", ["divide_by_output_norm", "no_root", "squared", "per_row_mean",
+                                     "absolute_on_zero_reference"])
+def test_rel_frobenius_pin_catches_planted_mistakes(monkeypatch, mistake):
+    """Plant a plausible slip in the metric (CPU only) and check the closed forms catch it."""
+    def planted(y, y_ref):
+        y = np.asarray(y, dtype=np.float64)
+        y_ref = np.asarray(y_ref, dtype=np.float64)
+        d = y - y_ref
+        if mistake == "divide_by_output_norm":
+            return float(np.linalg.norm(d) / np.linalg.norm(y))
+        if mistake == "no_root":
+            return float(np.sum(d * d) / np.sum(y_ref * y_ref))
+        if mistake == "squared":
+            return float(np.linalg.norm(d) / np.linalg.norm(y_ref)) ** 2
+        if mistake == "per_row_mean":
+            yr, dr = np.atleast_2d(y_ref), np.atleast_2d(d)
+            return float(np.mean(np.linalg.norm(dr, axis=-1) / np.linalg.norm(yr, axis=-1)))
+        den = np.linalg.norm(y_ref)
+        return float(np.linalg.norm(d) / den) if den > 0 else float(np.linalg.norm(d))
+
+    monkeypatch.setattr(oracle, "rel_frobenius", planted)
+    with pytest.raises(AssertionError):
+        test_rel_frobenius_closed_forms()
