@@ -177,11 +177,16 @@ MQ_API mq_status mq_decode_linear(const void* X_bf16, int64_t M, const void* W_b
  * outputs are still caller-owned device buffers.
  *   - M x K activations whose NVFP4 copy does not fit the array are rejected
  *     with MQ_ERR_WORKSPACE (the limit admits e.g. M = 8192 with K = 12288).
- *   - The first call on a device sets the array up (looks up its address,
- *     zeroes its control block, synchronizes that device); make that first
- *     call before any stream capture.
- *   - All calls share the one array: calls that overlap on the GPU (other
- *     streams, other host threads) race.  Serialize them.
+ *   - The first call on a device sets the array up: it looks up the array's
+ *     device address on that device (cudaGetSymbolAddress, which can load
+ *     the library's kernels).  Make that first call before any stream
+ *     capture.  A set-up that failed is not remembered: the next call
+ *     tries again.
+ *   - All calls share the one array, which keeps what the last call left
+ *     in it.  Calls that overlap on the GPU (other streams, other host
+ *     threads) race and give wrong results: serialize them.  Each call
+ *     first clears, on its own stream, the one counter that must start at
+ *     zero, so calls made after such an overlap are not affected by it.
  *   - Device-side errors (NaN/Inf in X, a pipeline timeout) are not reported
  *     by this call; mq_prefill_linear with a workspace reports them.
  * It calls no cudaMalloc, cudaFree or allocating library routine.

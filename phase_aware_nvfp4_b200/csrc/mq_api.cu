@@ -5,8 +5,7 @@
 #include <cstring>
 #include <mutex>
 
-#include "../../include/mixquant.h"
-#include "mq_internal.h"
+#include "mq_abi_checks.h"
 
 namespace mq {
 
@@ -119,31 +118,6 @@ Ws carve(void* ws, int64_t M, int64_t K)
         w.xq_scales = w.xq_codes + align_up(nvfp4_codes_bytes(M, K), kWsAlign);
     }
     return w;
-}
-
-// Largest M, N or K any call accepts: keeps every byte offset and element count
-// far inside 64 bits and every tensor-map coordinate inside 32 bits.
-constexpr int64_t kMaxDim = (int64_t)1 << 30;
-
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-mq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MQ_OK : MQ_ERR_CUDA; }
-
-mq_status check_device(DeviceInfo* di)
-{
-    if (device_info(di) != cudaSuccess) return MQ_ERR_CUDA;
-    if (di->cc_major != 10 || di->cc_minor != 0) return MQ_ERR_DEVICE;
-    return MQ_OK;
-}
-
-mq_status check_nvfp4(const mq_nvfp4* t, int64_t rows, int64_t cols)
-{
-    if (t == nullptr || t->codes == nullptr || t->scales == nullptr || t->alpha == nullptr)
-        return MQ_ERR_INVALID_ARG;
-    if (t->rows != rows || t->cols != cols) return MQ_ERR_SHAPE;
-    if (!aligned16(t->codes) || !aligned16(t->scales) || (reinterpret_cast<uintptr_t>(t->alpha) & 3u))
-        return MQ_ERR_ALIGNMENT;
-    return MQ_OK;
 }
 
 mq_status check_ws(void* ws, size_t ws_bytes, size_t need)
@@ -350,10 +324,9 @@ mq_status mq_prefill_linear(const void* X_bf16, const mq_nvfp4* X_q, int64_t M, 
     if (W == nullptr || W->codes == nullptr || W->scales == nullptr || W->alpha == nullptr) return MQ_ERR_INVALID_ARG;
     if (epi != MQ_EPI_BF16 && epi != MQ_EPI_SILU_MUL_NVFP4) return MQ_ERR_INVALID_ARG;
     const int64_t N = W->rows, K = W->cols;
-    if (M < 1 || M > kMaxDim || K < 64 || K % 64 != 0 || N < 16 || N % 16 != 0) return MQ_ERR_SHAPE;
-    if (N > kMaxDim || K > kMaxDim) return MQ_ERR_SHAPE;
-    mq_status st = check_nvfp4(W, N, K);
+    mq_status st = check_linear_shape(M, N, K);
     if (st != MQ_OK) return st;
+    if ((st = check_nvfp4(W, N, K)) != MQ_OK) return st;
     if (epi == MQ_EPI_BF16) {
         if (Y == nullptr) return MQ_ERR_INVALID_ARG;
         if (!aligned16(Y)) return MQ_ERR_ALIGNMENT;

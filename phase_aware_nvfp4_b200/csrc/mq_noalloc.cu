@@ -12,8 +12,7 @@
 // library holds this array until the process exits.
 #include <mutex>
 
-#include "../../include/mixquant.h"
-#include "mq_internal.h"
+#include "mq_abi_checks.h"
 
 namespace mq {
 namespace {
@@ -23,32 +22,26 @@ namespace {
 // with cudaGetSymbolAddress.
 static __device__ __align__(256) uint8_t g_noalloc_scratch[MQ_NOALLOC_SCRATCH_BYTES];
 
-struct ScratchState {
-    std::once_flag once;
-    cudaError_t setup_error = cudaSuccess;
-    uint8_t* ptr = nullptr;
-};
-
-ScratchState g_state[64];
+// Device address of the array, per device ordinal (device_info() refuses
+// ordinals >= 64).  Only a successful lookup is kept, so a first call that
+// failed (for example one made during stream capture) is retried by the next.
+std::mutex g_mu;
+uint8_t* g_ptr[64] = {};
 
 // Once per device, with that device current: look up the device address of
-// the scratch array and zero its control block (error bits and the amax
-// pass's block counter must start at zero; the kernels keep the counter
-// consistent afterwards).
-uint8_t* scratch_for_device(int dev, cudaError_t* err)
+// the scratch array.  Nothing in the array needs initialising here: every
+// call resets the one counter that must start at zero on its own stream.
+cudaError_t scratch_for_device(int dev, uint8_t** out)
 {
-    ScratchState& st = g_state[dev];
-    std::call_once(st.once, [&st] {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (g_ptr[dev] == nullptr) {
         void* p = nullptr;
-        st.setup_error = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (st.setup_error != cudaSuccess) return;
-        st.setup_error = cudaMemset(p, 0, kWsControlBytes);
-        if (st.setup_error != cudaSuccess) return;
-        st.setup_error = cudaDeviceSynchronize();
-        if (st.setup_error == cudaSuccess) st.ptr = static_cast<uint8_t*>(p);
-    });
-    *err = st.setup_error;
-    return st.ptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        g_ptr[dev] = static_cast<uint8_t*>(p);
+    }
+    *out = g_ptr[dev];
+    return cudaSuccess;
 }
 
 }  // namespace
@@ -59,24 +52,23 @@ using namespace mq;
 extern "C" MQ_API mq_status mq_prefill_linear_noalloc(const void* X_bf16, int64_t M, const mq_nvfp4* W,
                                                       const float* alpha_static, void* Y_bf16, mq_stream_t stream)
 {
+    // The same argument checks as mq_prefill_linear with X_bf16 and MQ_EPI_BF16.
     if (X_bf16 == nullptr || Y_bf16 == nullptr) return MQ_ERR_INVALID_ARG;
     if (W == nullptr || W->codes == nullptr || W->scales == nullptr || W->alpha == nullptr) return MQ_ERR_INVALID_ARG;
     const int64_t N = W->rows, K = W->cols;
-    if (M < 1 || M > (int64_t)1 << 30 || K < 64 || K % 64 != 0 || N < 16 || N % 16 != 0 || N > (int64_t)1 << 30)
-        return MQ_ERR_SHAPE;
-    auto a16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
-    if (!a16(X_bf16) || !a16(Y_bf16) || !a16(W->codes) || !a16(W->scales)) return MQ_ERR_ALIGNMENT;
+    mq_status st = check_linear_shape(M, N, K);
+    if (st != MQ_OK) return st;
+    if ((st = check_nvfp4(W, N, K)) != MQ_OK) return st;
+    if (!aligned16(X_bf16) || !aligned16(Y_bf16)) return MQ_ERR_ALIGNMENT;
     // The activation's NVFP4 copy plus the control block must fit the static array.
     const size_t codes_b = align_up(nvfp4_codes_bytes(M, K), kWsAlign);
     const size_t need = kWsControlBytes + codes_b + align_up(nvfp4_scales_bytes(M, K), kWsAlign);
     if (need > (size_t)MQ_NOALLOC_SCRATCH_BYTES) return MQ_ERR_WORKSPACE;
 
     DeviceInfo di;
-    if (device_info(&di) != cudaSuccess) return MQ_ERR_CUDA;
-    if (di.cc_major != 10 || di.cc_minor != 0) return MQ_ERR_DEVICE;
-    cudaError_t e = cudaSuccess;
-    uint8_t* base = scratch_for_device(di.device, &e);
-    if (base == nullptr || e != cudaSuccess) return MQ_ERR_CUDA;
+    if ((st = check_device(&di)) != MQ_OK) return st;
+    uint8_t* base = nullptr;
+    if (scratch_for_device(di.device, &base) != cudaSuccess) return MQ_ERR_CUDA;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     WsControl* ctrl = reinterpret_cast<WsControl*>(base);
@@ -84,6 +76,10 @@ extern "C" MQ_API mq_status mq_prefill_linear_noalloc(const void* X_bf16, int64_
     uint8_t* xq_codes = base + kWsControlBytes;
     uint8_t* xq_scales = xq_codes + codes_b;
 
+    // The amax pass counts finished blocks in the control block and its last
+    // block resets the counter; calls that overlapped on the GPU can leave it
+    // wrong, so each call starts from zero (stream-ordered, no allocation).
+    if (cudaMemsetAsync(&ctrl->amax_ticket, 0, sizeof(uint32_t), s) != cudaSuccess) return MQ_ERR_CUDA;
     const float* alpha_x = (alpha_static != nullptr) ? alpha_static : &ctrl->alpha;
     if (launch_quantize(X_bf16, M, K, alpha_static, &ctrl->alpha, xq_codes, xq_scales, 0, ctrl, partials, di, s) !=
         cudaSuccess)
@@ -102,5 +98,5 @@ extern "C" MQ_API mq_status mq_prefill_linear_noalloc(const void* X_bf16, int64_
     g.epilogue = 0;
     g.y = Y_bf16;
     g.ctrl = ctrl;
-    return launch_gemm_nvfp4(g, di, s) == cudaSuccess ? MQ_OK : MQ_ERR_CUDA;
+    return cuda_status(launch_gemm_nvfp4(g, di, s));
 }

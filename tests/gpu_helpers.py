@@ -77,3 +77,45 @@ def sample_rows(M: int, n: int = 64, seed: int = 0, extra=()) -> np.ndarray:
     rows = set(rng.choice(M, size=min(n, M), replace=False).tolist())
     rows |= {0, M - 1, *[int(e) for e in extra if 0 <= e < M]}
     return np.array(sorted(rows), dtype=np.int64)
+
+
+def block_rows(M: int, seed: int = 0, block: int = 128, extra=()) -> np.ndarray:
+    """One seeded random row in every `block`-row block of an M-row output, plus the first
+    and last rows: a tile-scheduler or raster slip that hits only some tiles shows up in
+    at least one sampled row."""
+    rng = np.random.default_rng(seed)
+    rows = {0, M - 1, *[int(e) for e in extra if 0 <= e < M]}
+    for b0 in range(0, M, block):
+        rows.add(int(rng.integers(b0, min(b0 + block, M))))
+    return np.array(sorted(rows), dtype=np.int64)
+
+
+def silu_mul_check(h_gpu_bits: np.ndarray, g64: np.ndarray, u64: np.ndarray, sg: np.ndarray, su: np.ndarray,
+                   rel_max: float = REL_FROB_MAX):
+    """Assert the fused epilogue's h = bf16(silu(g) u) is within tolerance of the oracle's.
+
+    g64, u64: the oracle's FP64 gate/up GEMM outputs (tensor scales applied); sg, su: their
+    sum_k |products| bounds (nvfp4_linear_rows' second result).  The GPU's g and u differ
+    from fl32(g64), fl32(u64) by at most dg = GAMMA*sg + 2^-22|g64| (tensor-core FP32
+    accumulation, two FP32 roundings of the tensor-scale multiply), likewise du.  With
+    |silu'| <= 1.1 and both sides rounding their own FP32 silu (expf vs libm exp, a few
+    binary32 ulps) and product before one BF16 rounding each:
+        |h_gpu - h_ref| <= ulp_bf16(max|h|) + 1.1 |u| dg + (|silu(g)| + 1.1 dg) du + 2^-19 |h_ref|.
+    Gates: rel-Frobenius <= rel_max and that bound on every element.
+    Returns (rel_frob, max_abs, bound_max)."""
+    hg = oracle.bf16_to_f64(h_gpu_bits)
+    g = np.asarray(g64, dtype=np.float64)
+    u = np.asarray(u64, dtype=np.float64)
+    h_ref = oracle.bf16_to_f64(oracle.silu_mul(g, u))
+    rel = oracle.rel_frobenius(hg, h_ref)
+    dg = GAMMA * np.asarray(sg) + 2.0 ** -22 * np.abs(g)
+    du = GAMMA * np.asarray(su) + 2.0 ** -22 * np.abs(u)
+    silu = np.abs(g / (1.0 + np.exp(-np.clip(g, -700.0, 700.0))))
+    bound = (np.maximum(oracle.bf16_ulp(h_ref), oracle.bf16_ulp(hg)) + 1.1 * np.abs(u) * dg
+             + (silu + 1.1 * dg) * du + 2.0 ** -19 * np.abs(h_ref))
+    err = np.abs(hg - h_ref)
+    bad = err > bound
+    assert rel <= rel_max, f"h rel-Frobenius {rel:.3e} > {rel_max}"
+    assert not bad.any(), (f"{int(bad.sum())} h elements over the bound; worst excess "
+                           f"{float((err - bound).max()):.3e} at {np.unravel_index(np.argmax(err - bound), err.shape)}")
+    return rel, float(err.max()), float(bound.max())

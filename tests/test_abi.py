@@ -144,6 +144,36 @@ def test_argument_errors_are_synchronous(lib):
     del h
 
 
+def test_noalloc_refuses_exactly_what_the_workspace_entry_point_refuses(lib):
+    """mq_prefill_linear_noalloc and mq_prefill_linear (BF16 X, BF16 epilogue) give the same
+    status for the same bad argument, before anything touches a device."""
+    P = 0x7F0000000000
+    ws, wsb = ctypes.c_void_p(P), ctypes.c_size_t(1 << 30)
+
+    def both(X, M, w, Y):
+        a = lib.mq_prefill_linear(X, None, M, ctypes.byref(w), 0, None, None, Y, None, None, ws, wsb, None)
+        b = lib.mq_prefill_linear_noalloc(X, M, ctypes.byref(w), None, Y, None)
+        return a, b
+
+    ok = _nv(256, 256)
+    cases = {
+        "alpha misaligned": (P, 128, mqb._NVFP4(P, P + 0x100000, P + 0x200002, 256, 256), P, 3),
+        "codes misaligned": (P, 128, mqb._NVFP4(P + 8, P + 0x100000, P + 0x200000, 256, 256), P, 3),
+        "null scales": (P, 128, mqb._NVFP4(P, 0, P + 0x200000, 256, 256), P, 1),
+        "K % 64": (P, 128, _nv(256, 200), P, 2),
+        "N % 16": (P, 128, _nv(250, 256), P, 2),
+        "M = 0": (P, 0, ok, P, 2),
+        "M > 2^30": (P, (1 << 30) + 1, ok, P, 2),
+        "K > 2^30": (P, 128, _nv(256, (1 << 30) + 64), P, 2),
+        "X misaligned": (P + 2, 128, ok, P, 3),
+        "Y misaligned": (P, 128, ok, P + 2, 3),
+        "Y null": (P, 128, ok, None, 1),
+        "X null": (None, 128, ok, P, 1),
+    }
+    for name, (X, M, w, Y, want) in cases.items():
+        assert both(X, M, w, Y) == (want, want), name
+
+
 def test_valid_call_without_gpu_reports_cuda_or_device_error(lib):
     import torch
     if torch.cuda.is_available():

@@ -7,7 +7,7 @@ import oracle
 from phase_aware_nvfp4_b200 import mixquant as mq
 from phase_aware_nvfp4_b200 import workloads as wl
 
-from gpu_helpers import gemm_check, nvfp4_host, require_gpu, to_dev, to_host_bits
+from gpu_helpers import gemm_check, nvfp4_host, require_gpu, silu_mul_check, to_dev, to_host_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -135,10 +135,8 @@ def test_fused_silu_mul_requant_epilogue(M, I, K):
 
     # (1) h vs the oracle's SiLU-mul of its own gate/up GEMM
     y64, sabs = oracle_linear(x, wgu)
-    h_ref = oracle.silu_mul(y64[:, :I], y64[:, I:])
     h_gpu = to_host_bits(h_dbg)
-    hr, hg = oracle.bf16_to_f64(h_ref), oracle.bf16_to_f64(h_gpu)
-    assert oracle.rel_frobenius(hg, hr) < 2e-3
+    silu_mul_check(h_gpu, y64[:, :I], y64[:, I:], sabs[:, :I], sabs[:, I:])
     # (2) codes and scales of h: bit-exact against the oracle quantizing the GPU's h with alpha_h
     codes, scales, _ = nvfp4_host(H)
     rc, rs = oracle.quantize(h_gpu, float(alpha_h))
