@@ -353,6 +353,39 @@ def _time_rotating(torch, calls, reps):
     return float(np.mean([a.elapsed_time(b) for a, b in evs]))
 
 
+def _decode_pair(mq, torch, dev, wl, Wm, Wq, hbm_gbs, reps, seed):
+    """BF16 decode and uniform-NVFP4 decode (tokens quantized on the fly) on one
+    weight [N, K] and its NVFP4 copy at M = 1, 8, 32, 64 tokens, timed on
+    rotating weight copies larger than L2 (weights cold, code warm).  HBM
+    roofline bytes: 2NK + 2MK + 2MN (BF16) and 0.5625NK + 2MK + 2MN (NVFP4)."""
+    N, K = Wm.shape
+    n_bf = max(2, -(-(400 << 20) // (2 * N * K)))          # copies: together > 3 x L2
+    n_q = max(2, -(-(400 << 20) // (N * K // 2)))
+    Wm_copies = [Wm] + [Wm.clone() for _ in range(n_bf - 1)]
+    Wq_copies = [Wq] + [mq.NVFP4Tensor(Wq.codes.clone(), Wq.scales.clone(), Wq.alpha.clone(), Wq.rows, Wq.cols)
+                        for _ in range(n_q - 1)]
+    dec, decq = {}, {}
+    for M in (1, 8, 32, 64):
+        x = _to_dev(torch, wl.heavy_tailed_bf16(M, K, seed + M), dev)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        wsd = mq.workspace(M, K, device=dev)
+        bf = [lambda W=W: mq.decode_linear(x, W, Y=y, ws=wsd) for W in Wm_copies]
+        q4 = [lambda W=W: mq.decode_linear_nvfp4(x, W, Y=y, ws=wsd) for W in Wq_copies]
+        for f in bf + q4:
+            f()
+        # the set-up above leaves the GPU idle for a while: ~50 ms of spinning first,
+        # so the timed calls do not start on a clock that is still ramping up
+        torch.cuda._sleep(100_000_000)
+        ms = _time_rotating(torch, bf, 4 * reps)
+        gbs = (2 * N * K + 2 * M * K + 2 * M * N) / (ms * 1e-3) / 1e9
+        dec[str(M)] = {"ms": ms, "GB/s": gbs, "frac": gbs / hbm_gbs}
+        msq = _time_rotating(torch, q4, 4 * reps)
+        gbs = (0.5625 * N * K + 2 * M * K + 2 * M * N) / (msq * 1e-3) / 1e9
+        decq[str(M)] = {"ms": msq, "GB/s": gbs, "frac": gbs / hbm_gbs, "speedup_vs_bf16": ms / msq}
+    del Wm_copies, Wq_copies
+    return dec, decq
+
+
 def measure_extras(mq, torch, dev, flush, hbm_gbs, fp4_peak, reps=10):
     """Side measurements of the other workloads (the main line is the projection step):
 
@@ -372,29 +405,11 @@ def measure_extras(mq, torch, dev, flush, hbm_gbs, fp4_peak, reps=10):
     Wm = _to_dev(torch, wl.normal_bf16(N, K, 0.02, 4001), dev)
     ws = mq.workspace(16384, K, device=dev)
     Wq = mq.quantize_weight(Wm, ws=ws)
-    # decode: weights cold (copies cycled, 4 x 100 MB BF16 / 12 x 28 MB NVFP4 > L2), code warm
-    Wm_copies = [Wm] + [Wm.clone() for _ in range(3)]
-    Wq_copies = [Wq] + [mq.NVFP4Tensor(Wq.codes.clone(), Wq.scales.clone(), Wq.alpha.clone(), Wq.rows, Wq.cols)
-                        for _ in range(11)]
-    dec, decq = {}, {}
-    for M in (1, 8, 32, 64):
-        x = _to_dev(torch, wl.heavy_tailed_bf16(M, K, 4000 + M), dev)
-        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-        wsd = mq.workspace(M, K, device=dev)
-        bf = [lambda W=W: mq.decode_linear(x, W, Y=y, ws=wsd) for W in Wm_copies]
-        q4 = [lambda W=W: mq.decode_linear_nvfp4(x, W, Y=y, ws=wsd) for W in Wq_copies]
-        for f in bf + q4:
-            f()
-        # the set-up above leaves the GPU idle for a while: ~50 ms of spinning first,
-        # so the timed calls do not start on a clock that is still ramping up
-        torch.cuda._sleep(100_000_000)
-        ms = _time_rotating(torch, bf, 4 * reps)
-        gbs = (2 * N * K + 2 * M * K + 2 * M * N) / (ms * 1e-3) / 1e9
-        dec[str(M)] = {"ms": ms, "GB/s": gbs, "frac": gbs / hbm_gbs}
-        msq = _time_rotating(torch, q4, 4 * reps)
-        gbs = (0.5625 * N * K + 2 * M * K + 2 * M * N) / (msq * 1e-3) / 1e9
-        decq[str(M)] = {"ms": msq, "GB/s": gbs, "frac": gbs / hbm_gbs, "speedup_vs_bf16": ms / msq}
-    del Wm_copies, Wq_copies
+    dec, decq = _decode_pair(mq, torch, dev, wl, Wm, Wq, hbm_gbs, reps, seed=4000)
+    # the other orientation of the same 4096 x 12288 master (K = 12288, N = 4096)
+    Wt = _to_dev(torch, wl.normal_bf16(K, N, 0.02, 4002), dev)
+    dec_t, decq_t = _decode_pair(mq, torch, dev, wl, Wt, mq.quantize_weight(Wt, ws=ws), hbm_gbs, reps, seed=4003)
+    del Wt
     Mp = 16384
     X = _to_dev(torch, wl.heavy_tailed_bf16(Mp, K, 4000), dev)
     Xq = mq.nvfp4_empty(Mp, K, dev)
@@ -470,6 +485,7 @@ def measure_extras(mq, torch, dev, flush, hbm_gbs, fp4_peak, reps=10):
         "roofline_decode": {"bound": "hbm", "kernel": "decode_bf16_kernel", "unit": "GB/s", "peak": hbm_gbs,
                             "achieved": dec["64"]["GB/s"], "frac": dec["64"]["frac"], "M": 64},
         "decode_nvfp4": decq,
+        "transposed_weight": [K, N], "decode_bf16_k12288": dec_t, "decode_nvfp4_k12288": decq_t,
         "prefill_nvfp4": {"M": Mp, "ms": ms, "TFLOP/s": 2 * Mp * N * K / (ms * 1e-3) / 1e12},
         "nvfp4_vs_bf16_rel_frobenius": err}
     del X, Xq, Y
@@ -522,10 +538,133 @@ def measure_extras(mq, torch, dev, flush, hbm_gbs, fp4_peak, reps=10):
                         "gate_up_TFLOP/s": fl_gu / (gu_ms * 1e-3) / 1e12,
                         "down_TFLOP/s": fl_dn / (dn_ms * 1e-3) / 1e12,
                         "gate_up_frac": fl_gu / (gu_ms * 1e-3) / 1e12 / fp4_peak}
+    # the unfused MLP with a dynamic alpha_h (R9's alternative): gate/up GEMM writing BF16 h,
+    # then the down projection quantizing h with amax|h| / 2688 (amax + quantize + GEMM)
+    Hb = torch.empty((Mm, I), dtype=torch.bfloat16, device=dev)
+    Y2 = torch.empty_like(Y)
+    wsh = mq.workspace(Mm, I, device=dev)
+    rec2 = []
+
+    def mlp_unfused():
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        e[0].record()
+        mq.quantize_activation(X, out=Xq, ws=wsm)
+        e[1].record()
+        mq.prefill_linear(W=Wgu, Xq=Xq, epilogue=mq.MQ_EPI_SILU_MUL_BF16, Y=Hb, ws=wsm)
+        e[2].record()
+        mq.prefill_linear(Hb, Wdn, Y=Y2, ws=wsh)
+        e[3].record()
+        rec2.append(e)
+    for _ in range(3):
+        mlp_unfused()
+    rec2.clear()
+    ms_u = _time_calls(torch, mlp_unfused, reps, flush)
+    # NVFP4-vs-BF16 error of both on 64 tokens (BF16 reference through this library's BF16 GEMM)
+    Wgu_bf = _to_dev(torch, wgu, dev)
+    Wdn_bf = _to_dev(torch, wdn, dev)
+    mlp()
+    torch.cuda.synchronize()
+    rows = torch.arange(0, Mm, Mm // 64, device=dev)
+    g = mq.decode_linear(X[rows].contiguous(), Wgu_bf).float()
+    hb = (torch.nn.functional.silu(g[:, :I]) * g[:, I:]).to(torch.bfloat16).contiguous()
+    yb = mq.decode_linear(hb, Wdn_bf).double()
+
+    def rel(yq):
+        return float(torch.linalg.norm(yq[rows].double() - yb) / torch.linalg.norm(yb))
+    out["fused_mlp"]["unfused_dynamic_alpha_h"] = {
+        "ms": ms_u, "TFLOP/s": (fl_gu + fl_dn) / (ms_u * 1e-3) / 1e12,
+        "gate_up_silu_bf16_ms": float(np.mean([e[1].elapsed_time(e[2]) for e in rec2])),
+        "down_with_amax_quant_ms": float(np.mean([e[2].elapsed_time(e[3]) for e in rec2])),
+        "speedup_of_fused_static": ms_u / ms,
+        "nvfp4_vs_bf16_rel_frobenius": rel(Y2), "note": "64 tokens; the fused static-alpha_h path on the "
+        "same tokens: see nvfp4_vs_bf16_rel_frobenius_fused_static"}
+    out["fused_mlp"]["nvfp4_vs_bf16_rel_frobenius_fused_static"] = rel(Y)
+    del Hb, Y2, wsh, Wgu_bf, Wdn_bf
     st = mq.async_status(wsm)
     if st != 0:
         raise RuntimeError(f"device error in the side measurements: {mq.STATUS_NAMES.get(st)}")
     return out
+
+
+def measure_ragged_mlp(mq, torch, dev, fp4_peak, reps=3):
+    """The ragged multi-turn prefill: 8 sequences of {2k, 4k, 8k, 8k, 16k, 16k, 32k, 42k}
+    tokens (131072 in all, the 131K long context) through one Qwen3-8B MLP: dynamic
+    activation quantization, gate/up GEMM with the SiLU-mul + NVFP4 requantization
+    epilogue (static alpha_h calibrated once), down GEMM.  39.58 TFLOP per pass
+    (2 * 131072 * (24576 * 4096 + 4096 * 12288)); the inputs (1 GB of X) are far
+    larger than L2.  Per-sequence NVFP4-vs-BF16 output error on 32 sampled tokens
+    of each sequence, the BF16 reference computed by the BF16 GEMM path of this
+    library (decode_linear, 256 rows) with the SiLU-mul in FP32."""
+    from phase_aware_nvfp4_b200 import workloads as wl
+    x, off = wl.ragged_heavy_tailed_bf16(wl.RAGGED_LENGTHS, 4096, 5000)
+    wgu, wdn = wl.mlp_weights(5000)
+    M, K, I = x.shape[0], x.shape[1], wdn.shape[1]
+    X = _to_dev(torch, x, dev)
+    del x
+    Wgu_bf = _to_dev(torch, wgu, dev)
+    Wdn_bf = _to_dev(torch, wdn, dev)
+    ws = mq.workspace(M, K, device=dev)
+    Wgu = mq.quantize_weight(Wgu_bf, gate_up_interleave=True, ws=ws)
+    Wdn = mq.quantize_weight(Wdn_bf, ws=ws)
+    Xq = mq.nvfp4_empty(M, K, dev)
+    H = mq.nvfp4_empty(M, I, dev)
+    Y = torch.empty((M, wdn.shape[0]), dtype=torch.bfloat16, device=dev)
+    # static alpha_h, calibrated once (offline): amax of h over this batch / (6 * 448)
+    mq.quantize_activation(X, out=Xq, ws=ws)
+    h_dbg = torch.empty((M, I), dtype=torch.bfloat16, device=dev)
+    one = torch.ones(1, dtype=torch.float32, device=dev)
+    mq.prefill_linear(W=Wgu, Xq=Xq, epilogue=mq.MQ_EPI_SILU_MUL_NVFP4, alpha_h=one, H=H, h_debug=h_dbg, ws=ws)
+    amax_h = float(h_dbg.float().abs().max())
+    del h_dbg
+    ah = torch.full((1,), amax_h / 2688.0 if amax_h > 0 else 1.0, dtype=torch.float32, device=dev)
+    H.alpha.copy_(ah)
+    rec = []
+
+    def mlp():
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        e[0].record()
+        mq.quantize_activation(X, out=Xq, ws=ws)
+        e[1].record()
+        mq.prefill_linear(W=Wgu, Xq=Xq, epilogue=mq.MQ_EPI_SILU_MUL_NVFP4, alpha_h=ah, H=H, ws=ws)
+        e[2].record()
+        mq.prefill_linear(W=Wdn, Xq=H, Y=Y, ws=ws)
+        e[3].record()
+        rec.append(e)
+    mlp()
+    torch.cuda.synchronize()
+    rec.clear()
+    for _ in range(reps):
+        mlp()
+    torch.cuda.synchronize()
+    ms = float(np.mean([e[0].elapsed_time(e[3]) for e in rec]))
+    q_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in rec]))
+    gu_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in rec]))
+    dn_ms = float(np.mean([e[2].elapsed_time(e[3]) for e in rec]))
+    st = mq.async_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device error in the ragged MLP: {mq.STATUS_NAMES.get(st)}")
+    fl_gu, fl_dn = 2 * M * wgu.shape[0] * K, 2 * M * wdn.shape[0] * I
+    tf = (fl_gu + fl_dn) / (ms * 1e-3) / 1e12
+    # per-sequence NVFP4-vs-BF16 error on 32 sampled tokens per sequence
+    rng = np.random.default_rng(5)
+    rows = np.concatenate([np.sort(rng.choice(np.arange(off[i], off[i + 1]), 32, replace=False))
+                           for i in range(len(wl.RAGGED_LENGTHS))])
+    ridx = torch.as_tensor(rows, device=dev)
+    g = mq.decode_linear(X[ridx].contiguous(), Wgu_bf).float()
+    hb = (torch.nn.functional.silu(g[:, :I]) * g[:, I:]).to(torch.bfloat16).contiguous()
+    yb = mq.decode_linear(hb, Wdn_bf).double()
+    yq = Y[ridx].double()
+    per_seq = []
+    for i in range(len(wl.RAGGED_LENGTHS)):
+        sl = slice(32 * i, 32 * (i + 1))
+        per_seq.append(float(torch.linalg.norm(yq[sl] - yb[sl]) / torch.linalg.norm(yb[sl])))
+    del X, Xq, H, Y, Wgu_bf, Wdn_bf
+    return {"M": M, "lengths": list(wl.RAGGED_LENGTHS), "gate_up": [wgu.shape[0], K], "down": [wdn.shape[0], I],
+            "flops": fl_gu + fl_dn, "ms": ms, "TFLOP/s": tf, "tokens_per_s": M / (ms * 1e-3),
+            "frac": tf / fp4_peak, "quant_ms": q_ms, "gate_up_silu_requant_ms": gu_ms, "down_ms": dn_ms,
+            "gate_up_TFLOP/s": fl_gu / (gu_ms * 1e-3) / 1e12, "down_TFLOP/s": fl_dn / (dn_ms * 1e-3) / 1e12,
+            "nvfp4_vs_bf16_rel_frobenius_per_sequence": per_seq, "reps": reps,
+            "l2": "inputs (1 GB) far larger than L2; no flush"}
 
 
 def measure_library_gemm(torch, w, Wq, Xq, Y, flush, fp4_peak, reps=10):
@@ -572,6 +711,67 @@ def measure_library_gemm(torch, w, Wq, Xq, Y, flush, fp4_peak, reps=10):
     return out
 
 
+def measure_e2e(torch, dist, world, dev, groups, xs_pin, X, Y, step, flops, K):
+    """End to end through the public API with host buffers.  Every step copies
+    its activations in from pinned host memory, runs the prefill pass and copies
+    every output back to pinned host memory; all of it is inside the timed
+    region.  The copies run on their own streams with two device buffer sets,
+    so step i + 1's upload and step i - 1's download overlap step i's compute
+    (PCIe is full duplex): the pipeline a serving loop would run."""
+    Xb = [X, {g: torch.empty_like(t) for g, t in X.items()}]
+    Yb = [Y, {n: torch.empty_like(t) for n, t in Y.items()}]
+    y_pin = [{n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for n, t in Y.items()} for _ in range(2)]
+    h2d = sum(t.numel() * 2 for t in xs_pin.values())
+    d2h = sum(t.numel() * 2 for t in Y.values())
+    ke = max(4, min(K, 20))
+    comp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+
+    def run(n_steps):
+        ev = lambda: torch.cuda.Event(enable_timing=False)
+        in_ready, x_free, y_ready, y_free = ([ev(), ev()] for _ in range(4))
+        for b in range(2):   # every buffer starts free
+            x_free[b].record(comp)
+            y_free[b].record(comp)
+        for i in range(n_steps):
+            b = i % 2
+            s_in.wait_event(x_free[b])
+            with torch.cuda.stream(s_in):
+                for g in groups:
+                    Xb[b][g].copy_(xs_pin[g], non_blocking=True)
+            in_ready[b].record(s_in)
+            comp.wait_event(in_ready[b])
+            comp.wait_event(y_free[b])
+            step(False, Xs=Xb[b], Ys=Yb[b])
+            x_free[b].record(comp)
+            y_ready[b].record(comp)
+            s_out.wait_event(y_ready[b])
+            with torch.cuda.stream(s_out):
+                for n in Y:
+                    y_pin[b][n].copy_(Yb[b][n], non_blocking=True)
+            y_free[b].record(s_out)
+        for b in range(2):
+            comp.wait_event(y_free[b])
+
+    run(3)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(comp)
+    s_in.wait_event(a)
+    s_out.wait_event(a)
+    run(ke)
+    b.record(comp)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(a.elapsed_time(b) / ke, dev)
+    return {"value": whole_job_tflops(flops, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": ke,
+            "h2d_GB/s": h2d / (e2e_ms * 1e-3) / 1e9, "d2h_GB/s": d2h / (e2e_ms * 1e-3) / 1e9,
+            "pipeline": "upload, compute and download on three streams, two buffer sets: uploads and "
+                        "downloads of neighbouring steps overlap each step's compute"}
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -612,17 +812,19 @@ def run_gpu(args):
 
     ev = {}
 
-    def step(record: bool, i: int = 0):
+    def step(record: bool, i: int = 0, Xs=None, Ys=None):
+        Xs = X if Xs is None else Xs
+        Ys = Y if Ys is None else Ys
         for g, ps in groups.items():
             if record:
                 ev[("q", g, i)][0].record()
-            mq.quantize_activation(X[g], out=Xq[g], ws=ws)
+            mq.quantize_activation(Xs[g], out=Xq[g], ws=ws)
             if record:
                 ev[("q", g, i)][1].record()
             for p in ps:
                 if record:
                     ev[("g", p.name, i)][0].record()
-                mq.prefill_linear(W=Wq[p.name], Xq=Xq[g], Y=Y[p.name], ws=ws)
+                mq.prefill_linear(W=Wq[p.name], Xq=Xq[g], Y=Ys[p.name], ws=ws)
                 if record:
                     ev[("g", p.name, i)][1].record()
 
@@ -710,36 +912,12 @@ def run_gpu(args):
     # end to end through the public API with host buffers: H2D of every
     # activation from pinned memory, the prefill pass, D2H of every output
     if not args.no_e2e:
-        y_pin = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for n, t in Y.items()}
-        h2d = sum(t.numel() * 2 for t in xs_pin.values())
-        d2h = sum(t.numel() * 2 for t in Y.values())
-        ke = max(3, min(K, 20))
-
-        def e2e_step():
-            for g in groups:
-                X[g].copy_(xs_pin[g], non_blocking=True)
-            step(False)
-            for n in Y:
-                y_pin[n].copy_(Y[n], non_blocking=True)
-
-        for _ in range(2):
-            e2e_step()
-        torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        for _ in range(ke):
-            e2e_step()
-        b.record()
-        torch.cuda.synchronize()
-        e2e_ms = max_over_ranks(a.elapsed_time(b) / ke, dev)
-        line["e2e"] = {"value": whole_job_tflops(flops, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                       "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": ke}
+        line["e2e"] = measure_e2e(torch, dist, world, dev, groups, xs_pin, X, Y, step, flops, K)
 
     if not args.no_extras:
         line["extras"] = measure_extras(mq, torch, dev, flush, hbm_gbs, fp4_peak)
         line["extras"]["library_nvfp4_gemm"] = measure_library_gemm(torch, w, Wq, Xq, Y, flush, fp4_peak)
+        line["extras"]["ragged_mlp_131072"] = measure_ragged_mlp(mq, torch, dev, fp4_peak)
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res = time_oracle(w, xs_h, ws_h, args.cpu_baseline_seconds, steps=1)

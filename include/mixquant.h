@@ -72,8 +72,9 @@ typedef enum mq_status {
 } mq_status;
 
 typedef enum mq_epilogue {
-    MQ_EPI_BF16 = 0,         /* Y = bf16(alpha_x alpha_w X W^T) */
-    MQ_EPI_SILU_MUL_NVFP4 = 1 /* h = bf16(silu(gate) * up), stored as NVFP4 with a static alpha_h */
+    MQ_EPI_BF16 = 0,           /* Y = bf16(alpha_x alpha_w X W^T) */
+    MQ_EPI_SILU_MUL_NVFP4 = 1, /* h = bf16(silu(gate) * up), stored as NVFP4 with a static alpha_h */
+    MQ_EPI_SILU_MUL_BF16 = 2   /* h = bf16(silu(gate) * up), stored as BF16 (the unfused MLP path) */
 } mq_epilogue;
 
 /* An NVFP4 tensor: views of caller-owned device buffers (layout above). */
@@ -142,6 +143,14 @@ MQ_API mq_status mq_quantize_activation(const void* X_bf16, int64_t M, int64_t K
  *                          Eq. 3) with the static device scale *alpha_h into
  *                          H_out ([M, I]; H_out->alpha is not written).
  *                          h_debug (optional, BF16 [M, I]) also receives h.
+ *   MQ_EPI_SILU_MUL_BF16   the same h, written as BF16 to Y ([M, I], 16-byte
+ *                          aligned) instead of being quantized.  Passing this h
+ *                          to a second mq_prefill_linear (X_bf16 = h) quantizes
+ *                          it with its dynamic tensor scale amax|h|/2688: the
+ *                          unfused MLP, whose alpha_h is exact for every batch
+ *                          but which writes and reads h in BF16, against the
+ *                          fused epilogue's static alpha_h (a scale the caller
+ *                          calibrated beforehand; blocks above it clip, Eq. 2).
  * Exactly one of X_bf16 / X_q is non-NULL.  With X_bf16, the activation is
  * quantized into the workspace (ws_bytes >= mq_workspace_bytes(M, K)) with
  * alpha_x = *alpha_static, or the dynamic amax scale when alpha_static is NULL.

@@ -322,13 +322,14 @@ mq_status mq_prefill_linear(const void* X_bf16, const mq_nvfp4* X_q, int64_t M, 
 {
     if ((X_bf16 == nullptr) == (X_q == nullptr)) return MQ_ERR_INVALID_ARG;
     if (W == nullptr || W->codes == nullptr || W->scales == nullptr || W->alpha == nullptr) return MQ_ERR_INVALID_ARG;
-    if (epi != MQ_EPI_BF16 && epi != MQ_EPI_SILU_MUL_NVFP4) return MQ_ERR_INVALID_ARG;
+    if (epi != MQ_EPI_BF16 && epi != MQ_EPI_SILU_MUL_NVFP4 && epi != MQ_EPI_SILU_MUL_BF16) return MQ_ERR_INVALID_ARG;
     const int64_t N = W->rows, K = W->cols;
     mq_status st = check_linear_shape(M, N, K);
     if (st != MQ_OK) return st;
     if ((st = check_nvfp4(W, N, K)) != MQ_OK) return st;
-    if (epi == MQ_EPI_BF16) {
+    if (epi == MQ_EPI_BF16 || epi == MQ_EPI_SILU_MUL_BF16) {
         if (Y == nullptr) return MQ_ERR_INVALID_ARG;
+        if (epi == MQ_EPI_SILU_MUL_BF16 && N % 128 != 0) return MQ_ERR_SHAPE;
         if (!aligned16(Y)) return MQ_ERR_ALIGNMENT;
     } else {
         if (alpha_h == nullptr) return MQ_ERR_INVALID_ARG;
@@ -370,7 +371,8 @@ mq_status mq_prefill_linear(const void* X_bf16, const mq_nvfp4* X_q, int64_t M, 
     g.M = M;
     g.N = N;
     g.K = K;
-    g.epilogue = (int)epi;
+    // kernel epilogues: 0 BF16 Y, 1 SiLU-mul -> NVFP4 h, 2 RoPE + KV cache, 3 SiLU-mul -> BF16 h
+    g.epilogue = (epi == MQ_EPI_SILU_MUL_BF16) ? 3 : (int)epi;
     g.y = Y;
     if (epi == MQ_EPI_SILU_MUL_NVFP4) {
         g.h_codes = H_out->codes;

@@ -105,11 +105,11 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 // interleaved in 16-row groups when quantized).  Produces 16 values of
 // h = bf16(silu(g) * u) and quantizes them as one NVFP4 block with the
 // static tensor scale alpha_h (Eq. 2 / Eq. 3 with alpha = alpha_h).
-__device__ __forceinline__ void silu_mul_quant_chunk(const uint32_t (&acc)[32], float alpha_ab, float alpha_h,
-                                                     float alpha_h_qmax, uint32_t (&codes)[2], uint32_t& scale,
-                                                     uint32_t (&hbits)[8])
+// h = bf16(silu(g) * u) of one 32-column chunk (16 gate columns, then the 16
+// matching up columns), with g, u = fl(acc * fl(alpha_x * alpha_w)); returns
+// the 16 values (exactly representable in BF16) and their |h| maximum.
+__device__ __forceinline__ float silu_mul_chunk(const uint32_t (&acc)[32], float alpha_ab, float (&h)[16])
 {
-    float h[16];
     float amax = 0.0f;
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
@@ -120,6 +120,15 @@ __device__ __forceinline__ void silu_mul_quant_chunk(const uint32_t (&acc)[32], 
         h[j] = hv;
         amax = fmaxf(amax, fabsf(hv));
     }
+    return amax;
+}
+
+__device__ __forceinline__ void silu_mul_quant_chunk(const uint32_t (&acc)[32], float alpha_ab, float alpha_h,
+                                                     float alpha_h_qmax, uint32_t (&codes)[2], uint32_t& scale,
+                                                     uint32_t (&hbits)[8])
+{
+    float h[16];
+    const float amax = silu_mul_chunk(acc, alpha_ab, h);
 #pragma unroll
     for (int j = 0; j < 8; ++j) hbits[j] = pack_bf16x2(h[2 * j], h[2 * j + 1]);
     const uint32_t sc = e4m3_round_sat(__fdiv_rn(amax, alpha_h_qmax));
@@ -235,6 +244,36 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const EpiScales& 
         return;
     }
     const int lane_ok = row < p.M;
+    if (EPI == 3) {
+        // SiLU-mul with a BF16 h output [M, N/2] in p.y (the unfused MLP path)
+        uint32_t hb[64];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(t_row + 32 * c, r);
+            tmem_wait_ld(r);
+            float h[16];
+            (void)silu_mul_chunk(r, es.alpha_ab, h);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) hb[8 * c + j] = pack_bf16x2(h[2 * j], h[2 * j + 1]);
+        }
+        tc_fence_before();
+        release();
+        const int hN = p.N / 2;
+        const int hcol0 = n_blk * (BN / 2);
+        if (lane_ok && hcol0 < hN) {
+            const int nch = min(8, (hN - hcol0) / 16);
+            uint16_t* hrow = static_cast<uint16_t*>(p.y) + row * (int64_t)hN + hcol0;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                if (c < nch) {
+                    reinterpret_cast<uint4*>(hrow)[2 * c] = make_uint4(hb[8 * c], hb[8 * c + 1], hb[8 * c + 2], hb[8 * c + 3]);
+                    reinterpret_cast<uint4*>(hrow)[2 * c + 1] =
+                        make_uint4(hb[8 * c + 4], hb[8 * c + 5], hb[8 * c + 6], hb[8 * c + 7]);
+                }
+        }
+        return;
+    }
     if (EPI == 0) {
         uint32_t out[128];
 #pragma unroll
@@ -574,6 +613,43 @@ __device__ __forceinline__ void epilogue_half_bf16_tma(const EpiScales& es, uint
     }
 }
 
+// Unfused MLP half-tile (EPI 3): the warp's 32 rows x 128 accumulator columns
+// are four 32-column gate/up chunks = 64 columns of h = bf16(silu(g) * u),
+// written as one 32 x 64 BF16 subtile through the staging buffer with one TMA
+// store (x0 = first h column, y0 = first row).
+template <class Barrier>
+__device__ __forceinline__ void epilogue_half_silu_bf16(const EpiScales& es, uint32_t t_col, int lane, uint8_t* stg,
+                                                        const CUtensorMap* tmap_y, int32_t x0, int32_t y0,
+                                                        Barrier arrive)
+{
+    uint32_t acc[4][32];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(t_col + 32 * c, acc[c]);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) tmem_wait_ld(acc[c]);
+    release_acc_warp(lane, arrive);
+    uint32_t hb[32];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        float h[16];
+        (void)silu_mul_chunk(acc[c], es.alpha_ab, h);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) hb[8 * c + j] = pack_bf16x2(h[2 * j], h[2 * j + 1]);
+    }
+    if (lane == 0) bulk_wait_group_read<0>();
+    __syncwarp();
+    uint8_t* rowp = stg + lane * 128;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        *reinterpret_cast<uint4*>(rowp + ((j ^ (lane & 7)) << 4)) = make_uint4(hb[4 * j], hb[4 * j + 1], hb[4 * j + 2], hb[4 * j + 3]);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        tma_store_2d(tmap_y, stg, x0, y0);
+        bulk_commit_group();
+    }
+}
+
 // Fused MLP half-tile (EPI 1): accumulator columns [128*half, 128*half + 128)
 // are four 32-column chunks (16 gate + 16 up each) = 64 h columns = one
 // 64-wide group of four NVFP4 blocks, whose four scale bytes form one 32-bit
@@ -663,7 +739,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_NUM_THREADS, 1)
         prefetch_tensormap(&tmap_b);
         prefetch_tensormap(&tmap_sfa);
         prefetch_tensormap(&tmap_sfb);
-        if (EPI == 0) prefetch_tensormap(&tmap_y);
+        if (EPI == 0 || EPI == 3) prefetch_tensormap(&tmap_y);
     }
     if (warp == 1) tmem_alloc_pair(tmem_slot, TMEM_COLS);
     tc_fence_before();
@@ -808,6 +884,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_NUM_THREADS, 1)
                 epilogue_half_bf16_tma(es, t_col, lane, stg, &tmap_y, n_blk * BN + 128 * half, (int32_t)row0, arrive);
             } else if (EPI == 1) {
                 epilogue_half_mlp(p, es, t_col, half, row0 + lane, n_blk, lane, arrive);
+            } else if (EPI == 3) {
+                epilogue_half_silu_bf16(es, t_col, lane, stg, &tmap_y, n_blk * (BN / 2) + 64 * half, (int32_t)row0,
+                                        arrive);
             } else {
                 uint32_t acc[4][32];
 #pragma unroll
@@ -819,7 +898,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_NUM_THREADS, 1)
             }
         }
         // every output store has finished before the CTA may leave
-        if (EPI == 0 && lane == 0) bulk_wait_group<0>();
+        if ((EPI == 0 || EPI == 3) && lane == 0) bulk_wait_group<0>();
     }
 
     tc_fence_before();
@@ -829,6 +908,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_NUM_THREADS, 1)
         tc_fence_after();
         tmem_dealloc_pair(tmem_base, TMEM_COLS);
     }
+}
+
+template <int EPI>
+cudaError_t launch_pair(int pairs, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsfa,
+                        const CUtensorMap& tsfb, const CUtensorMap& ty, const Params& p, cudaStream_t s)
+{
+    auto k = gemm_nvfp4_pair_kernel<EPI>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    k<<<2 * pairs, P_NUM_THREADS, P_SMEM_BYTES, s>>>(ta, tb, tsfa, tsfb, ty, p);
+    return cudaGetLastError();
+}
+
+template <int EPI>
+cudaError_t launch_single(int grid, const CUtensorMap& ta, const CUtensorMap& tb, const Params& p, cudaStream_t s)
+{
+    auto k = gemm_nvfp4_kernel<EPI>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    k<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, tb, p);
+    return cudaGetLastError();
 }
 
 }  // namespace
@@ -887,34 +987,27 @@ cudaError_t launch_gemm_nvfp4(const GemmArgs& a, const DeviceInfo& di, cudaStrea
         if (!make_tmap_3d(&tsfb, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.b_scales, 128, (uint64_t)p.sfb_atoms,
                           (uint64_t)p.sfb_rowblks, 512, (uint64_t)p.sfb_atoms * 512, 128, 4, 2))
             return cudaErrorInvalidValue;
-        // output Y [M rows, N] BF16 for the TMA-store epilogue: 64-column x 32-row boxes (one warp's rows)
+        // output for the TMA-store epilogues, 64-column x 32-row boxes (one warp's
+        // rows): Y [M, N] BF16 (EPI 0) or h [M, N/2] BF16 (EPI 3)
         CUtensorMap ty = tb;
-        if (a.epilogue == 0 &&
-            !make_tmap_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.y, (uint64_t)a.N, (uint64_t)a.M,
-                          (uint64_t)a.N * 2, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B))
-            return cudaErrorInvalidValue;
+        if (a.epilogue == 0 || a.epilogue == 3) {
+            const uint64_t cols = a.epilogue == 0 ? (uint64_t)a.N : (uint64_t)a.N / 2;
+            if (!make_tmap_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.y, cols, (uint64_t)a.M, cols * 2, 64, 32,
+                              CU_TENSOR_MAP_SWIZZLE_128B))
+                return cudaErrorInvalidValue;
+        }
         p.num_m_blk = (int)((a.M + 2 * BM - 1) / (2 * BM));
         p.num_n_blk = num_n_blk;
         p.num_tiles = p.num_m_blk * num_n_blk;
         p.n_fastest = a.M > a.N;   // A (M rows) is the larger operand: sweep N fastest
         const int pairs = std::min(p.num_tiles, di.num_sms / 2);
-        if (a.epilogue == 0) {
-            auto k = gemm_nvfp4_pair_kernel<0>;
-            cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM_BYTES);
-            if (e != cudaSuccess) return e;
-            k<<<2 * pairs, P_NUM_THREADS, P_SMEM_BYTES, s>>>(ta, tb, tsfa, tsfb, ty, p);
-        } else if (a.epilogue == 2) {
-            auto k = gemm_nvfp4_pair_kernel<2>;
-            cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM_BYTES);
-            if (e != cudaSuccess) return e;
-            k<<<2 * pairs, P_NUM_THREADS, P_SMEM_BYTES, s>>>(ta, tb, tsfa, tsfb, ty, p);
-        } else {
-            auto k = gemm_nvfp4_pair_kernel<1>;
-            cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM_BYTES);
-            if (e != cudaSuccess) return e;
-            k<<<2 * pairs, P_NUM_THREADS, P_SMEM_BYTES, s>>>(ta, tb, tsfa, tsfb, ty, p);
+        switch (a.epilogue) {
+            case 0: return launch_pair<0>(pairs, ta, tb, tsfa, tsfb, ty, p, s);
+            case 1: return launch_pair<1>(pairs, ta, tb, tsfa, tsfb, ty, p, s);
+            case 2: return launch_pair<2>(pairs, ta, tb, tsfa, tsfb, ty, p, s);
+            case 3: return launch_pair<3>(pairs, ta, tb, tsfa, tsfb, ty, p, s);
         }
-        return cudaGetLastError();
+        return cudaErrorInvalidValue;
     }
 
     // single-CTA kernel for short activations (M <= 128): 128 x 256 tiles
@@ -926,23 +1019,13 @@ cudaError_t launch_gemm_nvfp4(const GemmArgs& a, const DeviceInfo& di, cudaStrea
     p.num_tiles = p.num_m_blk * num_n_blk;
     p.n_fastest = 0;   // M <= 128: a single m block
     const int grid = std::min(p.num_tiles, di.num_sms);
-    if (a.epilogue == 0) {
-        auto k = gemm_nvfp4_kernel<0>;
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        k<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, tb, p);
-    } else if (a.epilogue == 2) {
-        auto k = gemm_nvfp4_kernel<2>;
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        k<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, tb, p);
-    } else {
-        auto k = gemm_nvfp4_kernel<1>;
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        k<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, tb, p);
+    switch (a.epilogue) {
+        case 0: return launch_single<0>(grid, ta, tb, p, s);
+        case 1: return launch_single<1>(grid, ta, tb, p, s);
+        case 2: return launch_single<2>(grid, ta, tb, p, s);
+        case 3: return launch_single<3>(grid, ta, tb, p, s);
     }
-    return cudaGetLastError();
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace mq

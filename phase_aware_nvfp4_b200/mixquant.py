@@ -27,6 +27,7 @@ LIB_PATH = os.path.join(_HERE, "libmixquant.so")
 MQ_OK = 0
 MQ_EPI_BF16 = 0
 MQ_EPI_SILU_MUL_NVFP4 = 1
+MQ_EPI_SILU_MUL_BF16 = 2
 WS_CONTROL_BYTES = 16384
 
 STATUS_NAMES = {0: "MQ_OK", 1: "MQ_ERR_INVALID_ARG", 2: "MQ_ERR_SHAPE", 3: "MQ_ERR_ALIGNMENT",
@@ -245,7 +246,8 @@ def quantize_activation(X, alpha_static=None, out: NVFP4Tensor | None = None, ws
 def prefill_linear(X=None, W: NVFP4Tensor = None, *, Xq: NVFP4Tensor | None = None, epilogue: int = MQ_EPI_BF16,
                    alpha_static=None, alpha_h=None, Y=None, H: NVFP4Tensor | None = None, h_debug=None, ws=None,
                    stream=None):
-    """mq_prefill_linear.  Returns Y (BF16 [M, N]) or H (NVFP4 [M, N/2])."""
+    """mq_prefill_linear.  Returns Y (BF16 [M, N]; BF16 h [M, N/2] with MQ_EPI_SILU_MUL_BF16)
+    or H (NVFP4 [M, N/2])."""
     torch = _torch()
     if (X is None) == (Xq is None):
         raise ValueError("give exactly one of X (BF16) and Xq (NVFP4)")
@@ -260,15 +262,17 @@ def prefill_linear(X=None, W: NVFP4Tensor = None, *, Xq: NVFP4Tensor | None = No
     h_c = None
     if epilogue == MQ_EPI_BF16:
         Y = Y if Y is not None else torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    elif epilogue == MQ_EPI_SILU_MUL_BF16:
+        Y = Y if Y is not None else torch.empty((M, N // 2), dtype=torch.bfloat16, device=dev)
     else:
         H = H or nvfp4_empty(M, N // 2, dev)
         h_c = H.c()
     _check(load().mq_prefill_linear(_ptr(X), ctypes.byref(xq_c) if xq_c is not None else None, M,
                                     ctypes.byref(w_c), int(epilogue), _ptr(alpha_static), _ptr(alpha_h),
-                                    _ptr(Y) if epilogue == MQ_EPI_BF16 else None,
+                                    _ptr(Y) if epilogue != MQ_EPI_SILU_MUL_NVFP4 else None,
                                     ctypes.byref(h_c) if h_c is not None else None, _ptr(h_debug), *_ws_args(ws),
                                     _stream(stream)), "mq_prefill_linear")
-    return Y if epilogue == MQ_EPI_BF16 else H
+    return H if epilogue == MQ_EPI_SILU_MUL_NVFP4 else Y
 
 
 def prefill_linear_noalloc(X, W: NVFP4Tensor, alpha_static=None, Y=None, stream=None):

@@ -22,9 +22,27 @@ from __future__ import annotations
 
 from dataclasses import dataclass, field
 
+import os
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 
 CHUNK_ROWS = 2048
+_MAX_THREADS = 8
+
+
+def _by_chunks(rows: int, fill):
+    """Run fill(c, r0, r1) for every CHUNK_ROWS chunk.  Each chunk has its own
+    generator, so the result does not depend on the order or the threads the
+    chunks run on; numpy drops the GIL inside the bulk draws and arithmetic."""
+    spans = [(c, r0, min(rows, r0 + CHUNK_ROWS)) for c, r0 in enumerate(range(0, rows, CHUNK_ROWS))]
+    threads = min(len(spans), _MAX_THREADS, os.cpu_count() or 1)
+    if threads <= 1:
+        for sp in spans:
+            fill(*sp)
+        return
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        list(ex.map(lambda sp: fill(*sp), spans))
 
 
 def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
@@ -45,10 +63,11 @@ def _gen(seed: int, tag: int, chunk: int) -> np.random.Generator:
 def normal_bf16(rows: int, cols: int, std: float, seed: int) -> np.ndarray:
     """N(0, std^2) as BF16, [rows, cols]."""
     out = np.empty((rows, cols), dtype=np.uint16)
-    for c, r0 in enumerate(range(0, rows, CHUNK_ROWS)):
-        r1 = min(rows, r0 + CHUNK_ROWS)
+
+    def fill(c, r0, r1):
         z = _gen(seed, 1, c).standard_normal((r1 - r0, cols), dtype=np.float32)
         out[r0:r1] = f32_to_bf16_bits(z * np.float32(std))
+    _by_chunks(rows, fill)
     return out
 
 
@@ -72,13 +91,13 @@ def heavy_tailed_bf16(rows: int, cols: int, seed: int, outlier_frac: float = 0.0
     colscale = np.ones(cols, dtype=np.float32)
     colscale[ch] = np.float32(outlier_scale)
     out = np.empty((rows, cols), dtype=np.uint16)
-    for c, r0 in enumerate(range(0, rows, CHUNK_ROWS)):
-        r1 = min(rows, r0 + CHUNK_ROWS)
-        g = _gen(seed, 3, c)
-        z = g.standard_normal((4, r1 - r0, cols), dtype=np.float32)
+
+    def fill(c, r0, r1):
+        z = _gen(seed, 3, c).standard_normal((4, r1 - r0, cols), dtype=np.float32)
         chi2 = z[1] * z[1] + z[2] * z[2] + z[3] * z[3]
         t = z[0] / np.sqrt(chi2 / np.float32(3.0))
         out[r0:r1] = f32_to_bf16_bits(t * colscale)
+    _by_chunks(rows, fill)
     return out
 
 

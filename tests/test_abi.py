@@ -94,6 +94,12 @@ def test_argument_errors_are_synchronous(lib):
     h_bad = _nv(128, 64)
     assert lib.mq_prefill_linear(P, None, 128, ctypes.byref(w), 1, None, P, None, ctypes.byref(h_bad), None, ws,
                                  wsb, None) == 2
+    # unfused MLP epilogue (BF16 h into Y): needs Y and N % 128; epilogue 3 does not exist
+    w336 = _nv(336, 256)
+    assert lib.mq_prefill_linear(P, None, 128, ctypes.byref(w336), 2, None, None, P, None, None, ws, wsb, None) == 2
+    assert lib.mq_prefill_linear(P, None, 128, ctypes.byref(w), 2, None, None, None, None, None, ws, wsb, None) == 1
+    assert lib.mq_prefill_linear(P, None, 128, ctypes.byref(w), 2, None, None, P + 8, None, None, ws, wsb, None) == 3
+    assert lib.mq_prefill_linear(P, None, 128, ctypes.byref(w), 3, None, None, P, None, None, ws, wsb, None) == 1
     # decode: M in [1, 256]
     assert lib.mq_decode_linear(P, 300, P, 256, 256, P, ws, wsb, None) == 2
     assert lib.mq_decode_linear(P, 4, P, 256, 100, P, ws, wsb, None) == 2

@@ -148,6 +148,36 @@ def test_fused_silu_mul_requant_epilogue(M, I, K):
     gemm_check(to_host_bits(y), yd64, sabsd)
 
 
+@pytest.mark.parametrize("M,I,K", [(128, 128, 256), (300, 256, 512), (256, 384, 1024), (1000, 192, 320)])
+def test_unfused_silu_mul_bf16_epilogue_and_dynamic_alpha_h(M, I, K):
+    """The unfused MLP path: gate/up GEMM with a BF16 h output (MQ_EPI_SILU_MUL_BF16), then the
+    down projection quantizing h with its own dynamic tensor scale.  h equals the fused
+    epilogue's h bit for bit (same arithmetic) and is within the h bound of the oracle; the down
+    projection is within the GEMM tolerance of the oracle quantizing the GPU's h with
+    alpha_h = amax|h| / 2688."""
+    x = wl.heavy_tailed_bf16(M, K, 41 + M)
+    wgu = wl.normal_bf16(2 * I, K, 0.02, 42 + I)
+    wdn = wl.normal_bf16(K, I, 0.02, 43 + I)
+    X = to_dev(x)
+    Wgu = mq.quantize_weight(to_dev(wgu), gate_up_interleave=True)
+    h_fused = torch.empty((M, I), dtype=torch.bfloat16, device="cuda")
+    mq.prefill_linear(X, Wgu, epilogue=mq.MQ_EPI_SILU_MUL_NVFP4, alpha_h=torch.ones(1, device="cuda"),
+                      h_debug=h_fused)
+    h = mq.prefill_linear(X, Wgu, epilogue=mq.MQ_EPI_SILU_MUL_BF16)
+    assert tuple(h.shape) == (M, I)
+    Wdn = mq.quantize_weight(to_dev(wdn))
+    y = mq.prefill_linear(h, Wdn)                 # dynamic alpha_h: amax + quantize of h
+    torch.cuda.synchronize()
+    hg = to_host_bits(h)
+    assert np.array_equal(hg, to_host_bits(h_fused))
+    y64, sabs = oracle_linear(x, wgu)
+    silu_mul_check(hg, y64[:, :I], y64[:, I:], sabs[:, :I], sabs[:, I:])
+    ah = oracle.tensor_alpha(hg)[1]
+    aw = oracle.tensor_alpha(wdn)[1]
+    yd64, sabsd = oracle.nvfp4_linear_rows((*oracle.quantize(hg, ah), ah), (*oracle.quantize(wdn, aw), aw))
+    gemm_check(to_host_bits(y), yd64, sabsd)
+
+
 def test_interleaved_weight_plain_epilogue_is_permuted_columns():
     M, I, K = 128, 128, 256
     x = wl.heavy_tailed_bf16(M, K, 5)
