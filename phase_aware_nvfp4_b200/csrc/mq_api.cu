@@ -33,6 +33,10 @@ cudaError_t device_info(DeviceInfo* out)
         d.cc_minor = v;
         if ((e = cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) return e;
         d.max_smem_optin = (size_t)v;
+        if ((e = cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev)) != cudaSuccess) return e;
+        d.smem_per_sm = (size_t)v;
+        if ((e = cudaDeviceGetAttribute(&v, cudaDevAttrReservedSharedMemoryPerBlock, dev)) != cudaSuccess) return e;
+        d.smem_reserved_per_cta = (size_t)v;
         cache[dev] = d;
         valid[dev] = true;
     }
@@ -416,6 +420,11 @@ mq_status mq_decode_linear_nvfp4(const void* X_bf16, int64_t M, const mq_nvfp4* 
     if ((st = check_device(&di)) != MQ_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const Ws w = carve(ws, M, K);
+    // One kernel that quantizes the tokens itself; when its token slice does not
+    // fit in shared memory, the quantization kernel and then the decode GEMM.
+    const cudaError_t fe = launch_decode_nvfp4_fused(X_bf16, M, alpha_static, W->codes, W->scales, W->alpha, N, K,
+                                                     Y_bf16, w.ctrl, di, s);
+    if (fe != cudaErrorNotSupported) return cuda_status(fe);
     const float* ax = nullptr;
     st = quantize_into(X_bf16, M, K, alpha_static, w.xq_codes, w.xq_scales, &w.ctrl->alpha, false, 0, w, di, s, &ax);
     if (st != MQ_OK) return st;

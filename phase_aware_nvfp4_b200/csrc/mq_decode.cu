@@ -120,6 +120,13 @@ __global__ void __launch_bounds__(D_THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // BF16 path: the previous kernel of the stream may have written X, W or Y.
+    // (The NVFP4 path waits where it first reads what its predecessor, the
+    // token quantization, wrote.)
+    if (!FMT) {
+        grid_dep_wait();
+        grid_dep_launch_dependents();
+    }
 
     if (warp == 0) {
         // TMA producer: whole warp (warp-uniform values), one elected lane issues
@@ -400,14 +407,339 @@ cudaError_t launch_shape(const DParams& p, int n_tiles, int smem, const CUtensor
     attr[0].val.clusterDim.x = (unsigned)p.split;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
-    // FMT 1 follows the token quantization on the stream: let it start early
+    // let the kernel be scheduled while its predecessor on the stream drains
+    // (it waits for that kernel before touching what it may have written)
     attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = FMT ? 2 : 1;
+    cfg.numAttrs = 2;
     e = cudaLaunchKernelEx(&cfg, kern, tw, tx, tsfw, tsfx, p);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
+}
+
+// ==========================================================================
+// Uniform-NVFP4 decode with the token quantization inside the kernel
+// ==========================================================================
+//
+// The tokens of a decode step are few (M <= 128), so every CTA quantizes the
+// slice of X its K range needs itself, straight into shared memory in the MMA
+// operand layout, while its producer warp already streams the weight: no
+// separate quantization launch, no global round trip of the codes.  The
+// dynamic tensor scale needs the maximum over all of X: each CTA takes the
+// maximum of its K slice, and the CTAs of a cluster (whose slices cover all
+// of K) exchange their maxima through distributed shared memory, so every
+// cluster obtains the same alpha_x = amax / 2688 without touching global
+// memory.
+//
+// Warps: 0 weight producer (TMA), 1 TMEM owner and MMA issuer, 2-9
+// quantizers (warps 2-5 then drain the accumulator).  Shared memory: the
+// weight ring (per stage 16 KiB of codes + 2 KiB of scale atoms), then the
+// resident token slice (per K stage MT x 128 bytes of codes with the 128-byte
+// swizzle + 2 KiB of scale atoms).
+constexpr int F_THREADS = 320;
+constexpr int F_QTHREADS = F_THREADS - 64;
+constexpr int F_RING = QW_CODES + Q_SF;   // 18 KiB
+constexpr int F_SMALL = 2048;             // barriers, exchange slots, encode table
+
+struct FParams {
+    const uint16_t* x;            // BF16 tokens [M, K]
+    const float* alpha_static;    // or nullptr: dynamic alpha_x
+    const float* alpha_w;
+    int M, N, K, MT;
+    int k_stages, split, stages;
+    int x_off, x_stage;           // resident token slice: offset, bytes per K stage
+    int bar_offset;
+    uint32_t tmem_cols, tmem_sf;
+    uint16_t* y;
+    WsControl* ctrl;
+};
+
+__global__ void __launch_bounds__(F_THREADS, 1)
+    decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_sfw,
+                        const FParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + p.bar_offset);
+    uint64_t* empty_bar = full_bar + p.stages;
+    uint64_t* acc_full = empty_bar + p.stages;
+    uint64_t* x_ready = acc_full + 1;
+    uint64_t* amax_bar = x_ready + 1;
+    uint32_t* amax_slot = reinterpret_cast<uint32_t*>(amax_bar + 1);   // [8], one per cluster rank
+    uint32_t* red_q = amax_slot + 8;                                   // [F_QTHREADS / 32]
+    uint32_t* tmem_slot = red_q + F_QTHREADS / 32;
+    volatile uint32_t* abort_flag = tmem_slot + 1;
+    float* enc_tab = reinterpret_cast<float*>(smem + p.bar_offset + 1024);   // [128]
+    uint8_t* xr = smem + p.x_off;
+    float* red = reinterpret_cast<float*>(smem);   // [MT][128] split-K partials, after the MMAs
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = (p.split > 1) ? cluster_rank() : 0u;
+    const int n_tile = blockIdx.x / p.split;
+    const int ks_begin = (int)(((int64_t)p.k_stages * rank) / p.split);
+    const int ks_end = (int)(((int64_t)p.k_stages * (rank + 1)) / p.split);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < p.stages; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], 1);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(x_ready, F_QTHREADS);
+        mbar_init(amax_bar, (uint32_t)p.split);
+        *abort_flag = 0;
+        fence_mbarrier_init();
+        prefetch_tensormap(&tmap_w);
+        prefetch_tensormap(&tmap_sfw);
+    }
+    if (warp == 1) tmem_alloc(tmem_slot, p.tmem_cols);
+    tc_fence_before();
+    __syncthreads();
+    if (p.split > 1) cluster_sync_all();   // every peer's barriers exist before any remote arrival
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    float alpha_x = 1.0f;
+    grid_dep_wait();   // the previous kernel of the stream may have written X, W or Y
+    grid_dep_launch_dependents();
+
+    if (warp == 0) {
+        // weight producer: whole warp, one elected lane issues
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        int last_stage = -1;
+        uint32_t last_parity = 0;
+        for (int ks = ks_begin; ks < ks_end; ++ks) {
+            if (!warp_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) {
+                ok = false;
+                break;
+            }
+            if (elect_one()) {
+                uint8_t* sw = smem + stage * F_RING;
+                mbar_arrive_expect_tx(&full_bar[stage], (uint32_t)F_RING);
+                tma_load_2d(sw, &tmap_w, &full_bar[stage], ks * (QBK / 2), n_tile * DBM);
+                tma_load_2d(sw + QW_CODES, &tmap_sfw, &full_bar[stage], 0, n_tile * (p.k_stages * 4) + ks * 4);
+            }
+            __syncwarp();
+            last_stage = stage;
+            last_parity = phase;
+            if (++stage == p.stages) stage = 0, phase ^= 1u;
+        }
+        if (!ok) {
+            if (lane == 0) {
+                post_error(p.ctrl, kErrTimeout);
+                *abort_flag = 1;
+            }
+            if (last_stage >= 0) (void)mbar_wait(&full_bar[last_stage], last_parity);
+        }
+    } else if (warp == 1) {
+        // MMA issuer: waits once for the quantized tokens, then consumes the ring
+        const uint32_t idesc = idesc_nvfp4(DBM, p.MT);
+        const uint32_t sfa_tmem = tmem_base + p.tmem_sf;
+        const uint32_t sfb_tmem = sfa_tmem + 16;
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = warp_wait(x_ready, 0, abort_flag), next_ready = false;
+        if (ok) tc_fence_after();
+        for (int ks = ks_begin; ks < ks_end && ok; ++ks) {
+            if (!next_ready && !warp_wait(&full_bar[stage], phase, abort_flag)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            {
+                const int ns = (stage + 1 == p.stages) ? 0 : stage + 1;
+                next_ready = warp_test(&full_bar[ns], ns == 0 ? (phase ^ 1u) : phase);
+            }
+            const uint8_t* xs = xr + (ks - ks_begin) * p.x_stage;
+            const uint64_t w_d = sdesc_kmajor_sw128(smem_u32(smem + stage * F_RING));
+            const uint64_t x_d = sdesc_kmajor_sw128(smem_u32(xs));
+            const uint64_t sfw_d = sdesc_sf_block(smem_u32(smem + stage * F_RING + QW_CODES));
+            const uint64_t sfx_d = sdesc_sf_block(smem_u32(xs + p.MT * (QBK / 2)));
+            if (elect_one()) {
+#pragma unroll
+                for (int kb = 0; kb < 4; ++kb) {
+                    tmem_cp_32x128b_x4(sfa_tmem + 4 * kb, sfw_d + (uint64_t)((kb * 512) >> 4));
+                    tmem_cp_32x128b_x4(sfb_tmem + 4 * kb, sfx_d + (uint64_t)((kb * 512) >> 4));
+                    umma_nvfp4(tmem_base, w_d + (uint64_t)((32 * kb) >> 4), x_d + (uint64_t)((32 * kb) >> 4), idesc,
+                               sfa_tmem + 4 * kb, sfb_tmem + 4 * kb, (ks > ks_begin || kb > 0) ? 1u : 0u);
+                }
+                tc_commit(&empty_bar[stage]);
+            }
+            __syncwarp();
+            if (++stage == p.stages) stage = 0, phase ^= 1u;
+        }
+        if (!ok && lane == 0) {
+            post_error(p.ctrl, kErrTimeout);
+            *abort_flag = 1;
+        }
+        if (elect_one()) tc_commit(acc_full);   // also "every MMA issued has finished" before TMEM is freed
+        __syncwarp();
+    } else {
+        // ---- token quantization of this CTA's K slice [k_lo, k_hi), all M tokens
+        const int qt = threadIdx.x - 64;
+        const int qw = qt >> 5;
+        const int nks = ks_end - ks_begin;
+        const int k_lo = ks_begin * QBK;
+        const int k_hi = min(ks_end * QBK, p.K);
+        // scale atoms start at zero: padding rows (m >= M) and blocks past K then
+        // contribute nothing to the MMA
+        for (int i = qt; i < nks * (Q_SF / 16); i += F_QTHREADS) {
+            const int s = i / (Q_SF / 16), j = i - s * (Q_SF / 16);
+            reinterpret_cast<uint4*>(xr + s * p.x_stage + p.MT * (QBK / 2))[j] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        bool ok = true;
+        if (p.alpha_static != nullptr) {
+            alpha_x = __ldg(p.alpha_static);
+        } else {
+            // |x| maximum of the slice (NaN/Inf excluded and flagged, as the amax pass does)
+            const int vpr = (k_hi - k_lo) / 8;
+            uint32_t mx = 0, bad = 0;
+            for (int v = qt; v < p.M * vpr; v += F_QTHREADS) {
+                const int m = v / vpr, c = v - m * vpr;
+                const uint4 q = __ldg(reinterpret_cast<const uint4*>(p.x + (int64_t)m * p.K + k_lo) + c);
+                amax_accum(q.x, mx, bad);
+                amax_accum(q.y, mx, bad);
+                amax_accum(q.z, mx, bad);
+                amax_accum(q.w, mx, bad);
+            }
+            uint32_t b = max(mx & 0xFFFFu, mx >> 16) | (bad ? 0x80000000u : 0u);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) b = fold_max_flag(b, __shfl_xor_sync(0xFFFFFFFFu, b, o));
+            if (lane == 0) red_q[qw] = b;
+            named_barrier_sync(1, F_QTHREADS);
+            b = 0;
+            for (int w = 0; w < F_QTHREADS / 32; ++w) b = fold_max_flag(b, red_q[w]);
+            if (p.split > 1) {
+                // every rank's slice maximum into every rank's slot; the slots of all
+                // ranks together cover K, so their fold is the maximum over all of X
+                if (qt == 0) {
+                    for (int q = 0; q < p.split; ++q) {
+                        st_cluster_u32(map_to_cta(smem_u32(&amax_slot[rank]), (uint32_t)q), b);
+                        mbar_arrive_cluster(map_to_cta(smem_u32(amax_bar), (uint32_t)q));
+                    }
+                }
+                ok = mbar_wait_cluster(amax_bar, 0);
+                b = 0;
+                for (int q = 0; q < p.split; ++q) b = fold_max_flag(b, amax_slot[q]);
+            }
+            const float amax = __uint_as_float((b & 0x7FFFu) << 16);
+            alpha_x = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
+            if ((b & 0x80000000u) && qt == 0 && n_tile == 0 && rank == 0) post_error(p.ctrl, kErrNonFinite);
+        }
+        if (!ok) {
+            if (qt == 0) post_error(p.ctrl, kErrTimeout);
+            *abort_flag = 1;
+        }
+        const QuantConsts qc = quant_consts(alpha_x);
+        if (qt < 128) {
+            const float d = __fmul_rn(alpha_x, e4m3_to_float((uint32_t)qt));
+            enc_tab[qt] = (d == 0.0f) ? 0.0f : __frcp_rn(d);
+        }
+        named_barrier_sync(1, F_QTHREADS);
+        // Eq. 3 / Eq. 2 per 16-element block, written in the MMA operand layout:
+        // codes row m of stage sl at (m/8)*1024 + (m%8)*128 + 16*(chunk ^ m%8),
+        // scale (m, block kb) at the atom offset of the scale layout
+        const int nb = (k_hi - k_lo) / 16;
+        for (int b = qt; b < p.M * nb; b += F_QTHREADS) {
+            const int m = b / nb, kb = b - m * nb;
+            const uint4* src = reinterpret_cast<const uint4*>(p.x + (int64_t)m * p.K + k_lo + kb * 16);
+            const uint4 u0 = __ldg(src), u1 = __ldg(src + 1);
+            const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+            uint32_t c0, c1;
+            const uint32_t sc = quant_block16(w, qc, enc_tab, c0, c1);
+            const int kbs = kb & 15;
+            uint8_t* tile = xr + (kb >> 4) * p.x_stage;
+            *reinterpret_cast<uint2*>(tile + (m >> 3) * 1024 + (m & 7) * 128 + ((((kbs >> 1) ^ (m & 7))) << 4) +
+                                      (kbs & 1) * 8) = make_uint2(c0, c1);
+            tile[p.MT * (QBK / 2) + (kbs >> 2) * 512 + (m & 31) * 16 + (m >> 5) * 4 + (kbs & 3)] = (uint8_t)sc;
+        }
+        fence_proxy_async_smem();   // the generic-proxy writes above are read by the tensor cores
+        mbar_arrive(x_ready);
+
+        if (warp < 6) {
+            // ---- epilogue: warp w drains TMEM lane group w % 4
+            const int lg = warp & 3;
+            const int row = 32 * lg + lane;
+            const int64_t n = (int64_t)n_tile * DBM + row;
+            const float out_scale = __fmul_rn(__ldg(p.alpha_w), alpha_x);
+            const bool have = mbar_wait(acc_full, 0) && !*abort_flag;
+            if (!have && lane == 0) post_error(p.ctrl, kErrTimeout);
+            tc_fence_after();
+            const uint32_t t_row = tmem_base + ((uint32_t)(32 * lg) << 16);
+            for (int c = 0; c < p.MT / 16; ++c) {
+                uint32_t r[16];
+                tmem_ld_32x32b_x16(t_row + 16 * c, r);
+                tmem_wait_ld(r);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const int m = 16 * c + j;
+                    const float v = have ? __uint_as_float(r[j]) : 0.0f;
+                    if (p.split > 1) {
+                        red[m * DBM + row] = v;
+                    } else if (m < p.M && n < p.N) {
+                        p.y[(int64_t)m * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(v, out_scale)));
+                    }
+                }
+            }
+        }
+    }
+
+    if (p.split > 1) {
+        // every CTA of the cluster holds its partial tile; CTA `rank` sums tokens
+        // m = rank, rank + split, ... over the ranks in rank order
+        cluster_sync_all();
+        if (warp >= 2 && warp < 6) {
+            const int row = 32 * (warp & 3) + lane;
+            const int64_t n = (int64_t)n_tile * DBM + row;
+            const float out_scale = __fmul_rn(__ldg(p.alpha_w), alpha_x);
+            for (int m = (int)rank; m < p.M; m += p.split) {
+                float acc = 0.0f;
+                const uint32_t laddr = smem_u32(&red[m * DBM + row]);
+                for (int q = 0; q < p.split; ++q) acc += ld_dsmem_f32(laddr, (uint32_t)q);
+                if (n < p.N) p.y[(int64_t)m * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(acc, out_scale)));
+            }
+        }
+        cluster_sync_all();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, p.tmem_cols);
+    }
+}
+
+// Resident CTAs of decode_fused_kernel in clusters of `cluster` with `smem` bytes.
+int fused_resident_ctas(int cluster, int smem, const DeviceInfo& di)
+{
+    static std::mutex mu;
+    static std::map<std::tuple<int, int, int>, int> cache;
+    const auto key = std::make_tuple(di.device, cluster, smem);
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+    int ctas = 0;
+    if (cudaFuncSetAttribute(decode_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess) {
+        cudaLaunchConfig_t cfg{};
+        cfg.gridDim = dim3((unsigned)(cluster * di.num_sms), 1, 1);
+        cfg.blockDim = dim3(F_THREADS, 1, 1);
+        cfg.dynamicSmemBytes = (size_t)smem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)cluster;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int clusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&clusters, decode_fused_kernel, &cfg) == cudaSuccess) ctas = clusters * cluster;
+    }
+    (void)cudaGetLastError();
+    cache[key] = ctas;
+    return ctas;
 }
 
 }  // namespace
@@ -479,6 +811,106 @@ cudaError_t launch_decode_nvfp4(const uint8_t* x_codes, const uint8_t* x_scales,
                       (uint64_t)sf_rowblks(M) * (uint64_t)p.sfx_atoms, 512, 128, 4, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     return launch_shape<1>(p, n_tiles, smem, tw, tx, tsfw, tsfx, s);
+}
+
+}  // namespace mq
+
+namespace mq {
+
+cudaError_t launch_decode_nvfp4_fused(const void* x, int64_t M, const float* alpha_static, const uint8_t* w_codes,
+                                      const uint8_t* w_scales, const float* alpha_w, int64_t N, int64_t K, void* y,
+                                      WsControl* ctrl, const DeviceInfo& di, cudaStream_t s)
+{
+    FParams p{};
+    p.x = static_cast<const uint16_t*>(x);
+    p.alpha_static = alpha_static;
+    p.alpha_w = alpha_w;
+    p.M = (int)M;
+    p.N = (int)N;
+    p.K = (int)K;
+    p.MT = (int)((M + 31) / 32 * 32);   // MMA N: a multiple of 32, at most 128
+    p.k_stages = (int)((K + QBK - 1) / QBK);
+    uint32_t acc_cols = 32;
+    while ((int)acc_cols < p.MT) acc_cols <<= 1;
+    p.tmem_sf = acc_cols;
+    p.tmem_cols = 32;
+    while (p.tmem_cols < acc_cols + 32) p.tmem_cols <<= 1;
+    p.x_stage = p.MT * (QBK / 2) + Q_SF;
+    p.y = static_cast<uint16_t*>(y);
+    p.ctrl = ctrl;
+    const int n_tiles = (int)((N + DBM - 1) / DBM);
+
+    // Launch shape: K split (cluster size) and ring depth.  Candidates must fit
+    // the token slice and the ring in shared memory, run in one wave and leave
+    // each CTA at most 64K token elements to quantize (every cluster quantizes
+    // all tokens for its weight rows, so this work is repeated per 128 rows);
+    // among them the most weight bytes in flight (saturating at ~16 MB) wins,
+    // then the larger grid.
+    constexpr int64_t kSaturateBytes = 16ll << 20;
+    int best_split = 0, best_st = 0, best_smem = 0;
+    int64_t best_score = -1;
+    for (int sp = 1; sp <= 8 && sp <= p.k_stages; sp *= 2) {
+        const int nks = (p.k_stages + sp - 1) / sp;
+        for (int st = std::min(8, nks); st >= std::min(2, nks); --st) {
+            const int body = std::max(st * F_RING + nks * p.x_stage, p.MT * DBM * 4);
+            int smem = (body + 1023) / 1024 * 1024 + F_SMALL + 1024;
+            // TMEM: the CTAs that can share an SM must fit its 512 columns (an
+            // allocation that cannot be served would wait for a CTA that may itself
+            // wait on a cluster peer), so pad the shared memory to cap them
+            const int tmem_cap = 512 / (int)p.tmem_cols;
+            const int per_sm_min = (int)(di.smem_per_sm / (size_t)(tmem_cap + 1)) + 1;   // bytes incl. reserve
+            smem = std::max<int>(smem, per_sm_min - (int)di.smem_reserved_per_cta);
+            smem = (smem + 1023) / 1024 * 1024;
+            if ((size_t)smem > di.max_smem_optin) continue;
+            const int ctas = n_tiles * sp;
+            const int active = fused_resident_ctas(sp, smem, di);
+            if (active <= 0 || ctas > active) continue;
+            if (M * (K / sp) > 65536) continue;
+            const int64_t score = std::min<int64_t>(kSaturateBytes, (int64_t)ctas * st * F_RING) * 1024 +
+                                  std::min(ctas, 1023);
+            if (score > best_score) {
+                best_score = score;
+                best_split = sp;
+                best_st = st;
+                best_smem = smem;
+            }
+        }
+    }
+    if (best_split == 0) return cudaErrorNotSupported;   // the caller takes the two-kernel path
+    p.split = best_split;
+    p.stages = best_st;
+    const int nks = (p.k_stages + p.split - 1) / p.split;
+    p.x_off = p.stages * F_RING;
+    const int body = std::max(p.x_off + nks * p.x_stage, p.MT * DBM * 4);
+    p.bar_offset = (body + 1023) / 1024 * 1024;
+
+    CUtensorMap tw, tsfw;
+    if (!make_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, (uint64_t)(K / 2), (uint64_t)N, (uint64_t)(K / 2),
+                      QBK / 2, DBM, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    if (!make_tmap_2d(&tsfw, CU_TENSOR_MAP_DATA_TYPE_UINT32, w_scales, 128,
+                      (uint64_t)sf_rowblks(N) * (uint64_t)sf_atoms_per_rowblk(K), 512, 128, 4,
+                      CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(decode_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, best_smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)(n_tiles * p.split), 1, 1);
+    cfg.blockDim = dim3(F_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = (size_t)best_smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)p.split;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    e = cudaLaunchKernelEx(&cfg, decode_fused_kernel, tw, tsfw, p);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
 }
 
 }  // namespace mq

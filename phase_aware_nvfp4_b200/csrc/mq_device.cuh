@@ -11,6 +11,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <utility>
 
 #include "mq_internal.h"
 
@@ -159,6 +160,28 @@ __device__ __forceinline__ bool elect_one()
 __device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void grid_dep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
 
+// Host side: launch `kern` with programmatic stream serialization, so its
+// CTAs may be scheduled (and run their set-up) while the previous kernel in
+// the stream drains.  Every kernel launched this way calls grid_dep_wait()
+// before its first access to global memory that another kernel may write,
+// so the stream order of memory effects is unchanged.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args&&... args)
+{
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 // --------------------------------------------------------------------------
 // TMA / bulk copies (global -> shared, completion on an mbarrier)
 // --------------------------------------------------------------------------
@@ -171,6 +194,12 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
             "r"(smem_u32(smem_dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
         : "memory");
+}
+
+// Prefetch `bytes` (a multiple of 16, 16-byte aligned source) into L2.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* gsrc, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gsrc), "r"(bytes) : "memory");
 }
 
 __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar)
@@ -365,6 +394,35 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
+// Store a 32-bit value into shared memory of a CTA of the cluster
+// (cluster_addr from map_to_cta).
+__device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v)
+{
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+
+// Bounded wait on a local mbarrier whose arrivals come from other CTAs of the
+// cluster (acquire at cluster scope, so their stores before a release arrive
+// are visible afterwards).
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity,
+                                                  uint64_t timeout_ns = kWaitTimeoutNs)
+{
+    const uint32_t a = smem_u32(bar);
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(a), "r"(parity)
+            : "memory");
+        if (ok) return true;
+        if (globaltimer_ns() - t0 > timeout_ns) return false;
+    }
+}
+
 // TMA tile load into this CTA's shared memory whose completion is signalled
 // on an mbarrier of either CTA of the pair (bar = shared::cluster address).
 __device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorMap* map, uint32_t bar, int32_t x,
@@ -540,6 +598,29 @@ __device__ __forceinline__ uint32_t e2m1x8_cvt(float v0, float v1, float v2, flo
     return out;
 }
 
+// Two binary32 products in one instruction (mul.rn.f32x2, sm_100): each lane
+// is the correctly rounded product, as __fmul_rn (no flush of subnormals).
+__device__ __forceinline__ void fmul2_rn(float a0, float a1, float b, float& d0, float& d1)
+{
+    uint64_t d;
+    const uint64_t a = ((uint64_t)__float_as_uint(a1) << 32) | __float_as_uint(a0);
+    const uint64_t bb = ((uint64_t)__float_as_uint(b) << 32) | __float_as_uint(b);
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(bb));
+    d0 = __uint_as_float((uint32_t)d);
+    d1 = __uint_as_float((uint32_t)(d >> 32));
+}
+
+// Two binary32 products of two pairs, (a0 * b0, a1 * b1), in one instruction.
+__device__ __forceinline__ void fmul2v_rn(float a0, float a1, float b0, float b1, float& d0, float& d1)
+{
+    uint64_t d;
+    const uint64_t a = ((uint64_t)__float_as_uint(a1) << 32) | __float_as_uint(a0);
+    const uint64_t b = ((uint64_t)__float_as_uint(b1) << 32) | __float_as_uint(b0);
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    d0 = __uint_as_float((uint32_t)d);
+    d1 = __uint_as_float((uint32_t)(d >> 32));
+}
+
 // Codes of eight values x[0..7] with encode scale enc = fl(1 / fl(alpha * sigma)):
 // code = Pi_FP4(x * enc) with the sign of x.  When enc overflowed to +inf
 // (alpha * sigma below 2^-128) a zero x would give 0 * inf = NaN, so that rare
@@ -552,8 +633,10 @@ __device__ __forceinline__ uint32_t e2m1x8_encode(const float (&x)[8], float enc
         for (int j = 0; j < 8; ++j) out |= e2m1_code(x[j], enc) << (4 * j);
         return out;
     }
-    return e2m1x8_cvt(__fmul_rn(x[0], enc), __fmul_rn(x[1], enc), __fmul_rn(x[2], enc), __fmul_rn(x[3], enc),
-                      __fmul_rn(x[4], enc), __fmul_rn(x[5], enc), __fmul_rn(x[6], enc), __fmul_rn(x[7], enc));
+    float m[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) fmul2_rn(x[2 * j], x[2 * j + 1], enc, m[2 * j], m[2 * j + 1]);
+    return e2m1x8_cvt(m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7]);
 }
 
 // Per-halfword unsigned maximum (PTX max.u16x2).  The magnitude bits of a
@@ -565,17 +648,41 @@ __device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b)
     return d;
 }
 
-// |bf16| maximum of 16 values held as 8 packed words (exact, NaN/Inf not
-// expected: a non-finite input is reported by the amax pass).
+// Per-lane max(|a|, |b|) of two BF16 pairs (max.xorsign.abs.bf16x2): the
+// magnitude is exact; the sign bit (xor of the inputs' signs) is discarded by
+// the caller.
+__device__ __forceinline__ uint32_t max_abs_bf16x2(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// |bf16| maximum of 16 values held as 8 packed words (exact for finite values;
+// a non-finite input is reported by the amax pass and its block is not
+// required to match anything).
 __device__ __forceinline__ float bf16x16_absmax(const uint32_t (&w)[8])
 {
-    const uint32_t m01 = max_u16x2(w[0] & 0x7FFF7FFFu, w[1] & 0x7FFF7FFFu);
-    const uint32_t m23 = max_u16x2(w[2] & 0x7FFF7FFFu, w[3] & 0x7FFF7FFFu);
-    const uint32_t m45 = max_u16x2(w[4] & 0x7FFF7FFFu, w[5] & 0x7FFF7FFFu);
-    const uint32_t m67 = max_u16x2(w[6] & 0x7FFF7FFFu, w[7] & 0x7FFF7FFFu);
-    const uint32_t m = max_u16x2(max_u16x2(m01, m23), max_u16x2(m45, m67));
-    const uint32_t b = max(m & 0xFFFFu, m >> 16);
+    const uint32_t m = max_abs_bf16x2(max_abs_bf16x2(max_abs_bf16x2(w[0], w[1]), max_abs_bf16x2(w[2], w[3])),
+                                      max_abs_bf16x2(max_abs_bf16x2(w[4], w[5]), max_abs_bf16x2(w[6], w[7])));
+    const uint32_t b = max(m & 0x7FFFu, (m >> 16) & 0x7FFFu);
     return __uint_as_float(b << 16);
+}
+
+// Per-halfword |bf16| maximum over the finite values of a 32-bit word pair,
+// plus a flag word that is non-zero if a NaN/Inf was seen.
+__device__ __forceinline__ void amax_accum(uint32_t w, uint32_t& mx, uint32_t& bad)
+{
+    const uint32_t mag = w & 0x7FFF7FFFu;
+    const uint32_t nonfin = __vcmpgeu2(mag, 0x7F807F80u);  // 0xFFFF per NaN/Inf halfword
+    bad |= nonfin;
+    mx = max_u16x2(mx, mag & ~nonfin);
+}
+
+// Fold of two (|bf16| maximum, non-finite flag in bit 31) words.
+__device__ __forceinline__ uint32_t fold_max_flag(uint32_t a, uint32_t b)
+{
+    return max(a & 0x7FFFFFFFu, b & 0x7FFFFFFFu) | ((a | b) & 0x80000000u);
 }
 
 // E4M3 codes (RNE, satfinite) of two non-negative values in one conversion:
@@ -599,6 +706,47 @@ __device__ __forceinline__ uint32_t e4m3_block_scale(float amax, float aq, float
     const uint32_t c = pair & 0xFFu;
     if (c == (pair >> 8)) return c;
     return e4m3_round_sat(__fdiv_rn(amax, aq));
+}
+
+// Per-block constants of the Eq. 2 / Eq. 3 arithmetic for one tensor scale.
+struct QuantConsts {
+    float alpha_qmax;       // fl(alpha * q_max)
+    float inv_lo, inv_hi;   // floats bracketing 1 / alpha_qmax (see e4m3_block_scale)
+};
+
+__device__ __forceinline__ QuantConsts quant_consts(float alpha)
+{
+    QuantConsts q;
+    q.alpha_qmax = __fmul_rn(alpha, 6.0f);
+    // When fl(1/alpha_qmax) is not a normal finite float the bracket [0, inf]
+    // sends every block to the exact division.
+    const float inv_near = __frcp_rn(q.alpha_qmax);
+    const bool inv_normal = inv_near >= 1.17549435e-38f && inv_near < 3.0e38f;
+    q.inv_lo = inv_normal ? __uint_as_float(__float_as_uint(inv_near) - 1u) : 0.0f;
+    q.inv_hi = inv_normal ? __uint_as_float(__float_as_uint(inv_near) + 1u) : __int_as_float(0x7F800000);
+    return q;
+}
+
+// Eq. 3 scale code and Eq. 2 codes of one 16-element block held as eight BF16
+// pairs (element 2j in the low half of w[j]); enc_tab[c] = fl(1 / fl(alpha * sigma_c)).
+// Codes: element j of the block in nibble j of c0 (j < 8) or c1 (j - 8).
+__device__ __forceinline__ uint32_t quant_block16(const uint32_t (&w)[8], const QuantConsts& qc,
+                                                  const float* enc_tab, uint32_t& c0, uint32_t& c1)
+{
+    const float amax = bf16x16_absmax(w);
+    const uint32_t sc = e4m3_block_scale(amax, qc.alpha_qmax, qc.inv_lo, qc.inv_hi);
+    const float enc = enc_tab[sc];
+    float f0[8], f1[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        f0[2 * j] = bf16_lo(w[j]);
+        f0[2 * j + 1] = bf16_hi(w[j]);
+        f1[2 * j] = bf16_lo(w[4 + j]);
+        f1[2 * j + 1] = bf16_hi(w[4 + j]);
+    }
+    c0 = e2m1x8_encode(f0, enc);
+    c1 = e2m1x8_encode(f1, enc);
+    return sc;
 }
 
 // Byte offset of scale (row r, 16-element block kb) in the MMA scale layout:

@@ -379,6 +379,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // set-up done: wait for the previous kernel of the stream (its outputs may
+    // be this GEMM's operands or scales), and let the next one get scheduled
+    grid_dep_wait();
+    grid_dep_launch_dependents();
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -580,18 +584,22 @@ __device__ __forceinline__ void epilogue_half_bf16_tma(const EpiScales& es, uint
                                                        const CUtensorMap* tmap_y, int32_t x0, int32_t y0,
                                                        Barrier arrive)
 {
+    // all four TMEM loads in flight, one wait, then release: the accumulator is
+    // handed back to the MMA warp after one load latency instead of four
+    uint32_t acc[4][32];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(t_col + 32 * c, acc[c]);
+    tmem_wait_ld(acc[0]);
+#pragma unroll
+    for (int c = 1; c < 4; ++c) tmem_wait_ld(acc[c]);
+    release_acc_warp(lane, arrive);
     uint32_t out[64];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(t_col + 32 * c, r);
-        tmem_wait_ld(r);
+    for (int c = 0; c < 4; ++c)
 #pragma unroll
         for (int j = 0; j < 16; ++j)
-            out[16 * c + j] = pack_bf16x2(__fmul_rn(__uint_as_float(r[2 * j]), es.alpha_ab),
-                                          __fmul_rn(__uint_as_float(r[2 * j + 1]), es.alpha_ab));
-    }
-    release_acc_warp(lane, arrive);
+            out[16 * c + j] = pack_bf16x2(__fmul_rn(__uint_as_float(acc[c][2 * j]), es.alpha_ab),
+                                          __fmul_rn(__uint_as_float(acc[c][2 * j + 1]), es.alpha_ab));
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
         // the store that last read the buffer is done reading it
@@ -647,6 +655,114 @@ __device__ __forceinline__ void epilogue_half_silu_bf16(const EpiScales& es, uin
     if (lane == 0) {
         tma_store_2d(tmap_y, stg, x0, y0);
         bulk_commit_group();
+    }
+}
+
+// KV half-tile (EPI 2) of the pair kernel: the warp's 32 tokens x one
+// 128-column head.  Same arithmetic as kv_rope_store, with the global traffic
+// of a warp coalesced through its 4 KiB staging buffer (rows swizzled by
+// 16-byte chunk, chunk ^ row % 8, so both the row-wise and the column-wise
+// passes are free of bank conflicts):
+//   - for K heads, the cos/sin values of the 32 tokens' positions come in four
+//     chunks of 16 frequencies: per chunk the warp loads 32 rows x (64 B of
+//     cos + 64 B of sin) with 16-byte loads, eight lanes per row
+//     (kv_stage_cos_sin; the first chunk is staged before the accumulator
+//     wait, so its latency overlaps the tile's MMAs), and each lane then reads
+//     its own token's values;
+//   - each rotated pair of columns is rounded to BF16 at once, and the result
+//     leaves in two 64-column halves: each lane writes its token's 128 bytes,
+//     then the warp stores eight lanes per 128-byte segment of a cache slot.
+// pos / slot / valid: this lane's token (loaded before the accumulator wait).
+__device__ __forceinline__ void kv_stage_cos_sin(const Params& p, uint8_t* stg, int lane, int32_t pos, int ch)
+{
+    const int sub = lane >> 3, piece = lane & 7;
+#pragma unroll 4
+    for (int j = 0; j < 8; ++j) {
+        const int r = sub + 4 * j;
+        const int32_t pr = __shfl_sync(0xFFFFFFFFu, pos, r);
+        const float* src =
+            p.cos_sin + (int64_t)pr * 128 + (piece < 4 ? 16 * ch + 4 * piece : 64 + 16 * ch + 4 * (piece - 4));
+        *reinterpret_cast<float4*>(stg + r * 128 + ((piece ^ (r & 7)) << 4)) =
+            __ldg(reinterpret_cast<const float4*>(src));
+    }
+    __syncwarp();
+}
+
+template <class Barrier>
+__device__ __forceinline__ void epilogue_half_kv(const Params& p, float alpha_ab, uint32_t t_col, int lane,
+                                                 uint8_t* stg, int hh, int32_t pos, int64_t slot, bool valid,
+                                                 Barrier arrive)
+{
+    uint32_t acc[4][32];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(t_col + 32 * c, acc[c]);
+    tmem_wait_ld(acc[0]);
+#pragma unroll
+    for (int c = 1; c < 4; ++c) tmem_wait_ld(acc[c]);
+    release_acc_warp(lane, arrive);
+
+    const bool is_k = hh < p.n_heads;
+    const int head = is_k ? hh : hh - p.n_heads;
+    uint32_t out[64];   // BF16 pairs: out[w] holds columns 2w, 2w + 1
+    if (is_k) {
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+            if (ch > 0) kv_stage_cos_sin(p, stg, lane, pos, ch);   // chunk 0 was staged before the wait
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                // cos and sin of frequencies 16 ch + 4 q .. + 3 from this token's staged row
+                const float4 cv = *reinterpret_cast<const float4*>(stg + lane * 128 + ((q ^ (lane & 7)) << 4));
+                const float4 sv = *reinterpret_cast<const float4*>(stg + lane * 128 + (((q + 4) ^ (lane & 7)) << 4));
+                const float cc[4] = {cv.x, cv.y, cv.z, cv.w};
+                const float ss[4] = {sv.x, sv.y, sv.z, sv.w};
+                float lo[4], hi[4];
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    const int i = 16 * ch + 4 * q + t;   // frequency: columns i and i + 64
+                    const float a = __fmul_rn(__uint_as_float(acc[i >> 5][i & 31]), alpha_ab);
+                    const float b = __fmul_rn(__uint_as_float(acc[(i + 64) >> 5][(i + 64) & 31]), alpha_ab);
+                    lo[t] = __fsub_rn(__fmul_rn(a, cc[t]), __fmul_rn(b, ss[t]));
+                    hi[t] = __fadd_rn(__fmul_rn(b, cc[t]), __fmul_rn(a, ss[t]));
+                }
+                const int w = 8 * ch + 2 * q;   // column 16 ch + 4 q = 2 w
+                out[w] = pack_bf16x2(lo[0], lo[1]);
+                out[w + 1] = pack_bf16x2(lo[2], lo[3]);
+                out[w + 32] = pack_bf16x2(hi[0], hi[1]);
+                out[w + 33] = pack_bf16x2(hi[2], hi[3]);
+            }
+            __syncwarp();   // the next chunk's loads overwrite the staging rows
+        }
+    } else {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                out[16 * c + j] = pack_bf16x2(__fmul_rn(__uint_as_float(acc[c][2 * j]), alpha_ab),
+                                              __fmul_rn(__uint_as_float(acc[c][2 * j + 1]), alpha_ab));
+    }
+    uint16_t* cache = is_k ? p.k_cache : p.v_cache;
+    const int sub = lane >> 3, piece = lane & 7;
+#pragma unroll
+    for (int hq = 0; hq < 2; ++hq) {
+        // this token's columns 64 hq .. 64 hq + 63, then eight lanes per cache row segment
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const int w = 32 * hq + 4 * q;
+            *reinterpret_cast<uint4*>(stg + lane * 128 + ((q ^ (lane & 7)) << 4)) =
+                make_uint4(out[w], out[w + 1], out[w + 2], out[w + 3]);
+        }
+        __syncwarp();
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int r = sub + 4 * j;
+            const int64_t sr = __shfl_sync(0xFFFFFFFFu, slot, r);
+            const int vr = __shfl_sync(0xFFFFFFFFu, valid ? 1 : 0, r);
+            if (vr) {
+                uint4* dst = reinterpret_cast<uint4*>(cache + (sr * p.n_heads + head) * 128 + 64 * hq) + piece;
+                *dst = *reinterpret_cast<const uint4*>(stg + r * 128 + ((piece ^ (r & 7)) << 4));
+            }
+        }
+        __syncwarp();
     }
 }
 
@@ -747,6 +863,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_NUM_THREADS, 1)
     cluster_barrier();   // both CTAs' barriers initialised and TMEM allocated
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // set-up done: wait for the previous kernel of the stream (its outputs may
+    // be this GEMM's operands or scales), and let the next one get scheduled
+    grid_dep_wait();
+    grid_dep_launch_dependents();
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer (both CTAs)
@@ -870,6 +990,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_NUM_THREADS, 1)
         for (int tile = pair; tile < p.num_tiles; tile += npairs) {
             int m_blk, n_blk;
             tile_coords(p, tile, m_blk, n_blk);
+            // KV epilogue: this lane's token position and cache slot, fetched
+            // before the accumulator wait; an out-of-range one posts kErrIndex
+            // and the token is not written
+            int32_t kv_pos = 0;
+            int64_t kv_slot = 0;
+            bool kv_valid = false;
+            if (EPI == 2) {
+                const int64_t m = (int64_t)m_blk * 2 * BM + (int64_t)rank * BM + 32 * lg + lane;
+                if (m < p.M) {
+                    const int32_t ps = __ldg(p.positions + m);
+                    const int64_t sl = __ldg(p.slots + m);
+                    kv_valid = ps >= 0 && ps < p.max_pos && sl >= 0 && sl < p.num_slots;
+                    if (kv_valid) {
+                        kv_pos = ps;
+                        kv_slot = sl;
+                    } else {
+                        post_error(p.ctrl, kErrIndex);
+                    }
+                }
+            }
+            if (EPI == 2 && 2 * n_blk + half < p.n_heads) kv_stage_cos_sin(p, stg, lane, kv_pos, 0);
             if (!warp_wait(acc_full, acc_phase, abort_flag)) {
                 if (lane == 0) {
                     post_error(p.ctrl, kErrTimeout);
@@ -888,13 +1029,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_NUM_THREADS, 1)
                 epilogue_half_silu_bf16(es, t_col, lane, stg, &tmap_y, n_blk * (BN / 2) + 64 * half, (int32_t)row0,
                                         arrive);
             } else {
-                uint32_t acc[4][32];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(t_col + 32 * c, acc[c]);
-#pragma unroll
-                for (int c = 0; c < 4; ++c) tmem_wait_ld(acc[c]);
-                release_acc_warp(lane, arrive);
-                kv_rope_store(p, es.alpha_ab, row0 + lane, 2 * n_blk + half, acc);
+                epilogue_half_kv(p, es.alpha_ab, t_col, lane, stg, 2 * n_blk + half, kv_pos, kv_slot, kv_valid,
+                                 arrive);
             }
         }
         // every output store has finished before the CTA may leave
@@ -917,8 +1053,7 @@ cudaError_t launch_pair(int pairs, const CUtensorMap& ta, const CUtensorMap& tb,
     auto k = gemm_nvfp4_pair_kernel<EPI>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    k<<<2 * pairs, P_NUM_THREADS, P_SMEM_BYTES, s>>>(ta, tb, tsfa, tsfb, ty, p);
-    return cudaGetLastError();
+    return launch_pdl(k, dim3(2 * pairs), dim3(P_NUM_THREADS), P_SMEM_BYTES, s, ta, tb, tsfa, tsfb, ty, p);
 }
 
 template <int EPI>
@@ -927,8 +1062,7 @@ cudaError_t launch_single(int grid, const CUtensorMap& ta, const CUtensorMap& tb
     auto k = gemm_nvfp4_kernel<EPI>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    k<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, tb, p);
-    return cudaGetLastError();
+    return launch_pdl(k, dim3(grid), dim3(NUM_THREADS), SMEM_BYTES, s, ta, tb, p);
 }
 
 }  // namespace

@@ -51,6 +51,8 @@ struct DeviceInfo {
     int num_sms;
     int cc_major, cc_minor;
     size_t max_smem_optin;
+    size_t smem_per_sm;           // shared memory of one SM
+    size_t smem_reserved_per_cta; // shared memory the runtime reserves per resident CTA
 };
 // Cached per device; returns cudaSuccess or the error of the attribute query.
 cudaError_t device_info(DeviceInfo* out);
@@ -128,6 +130,15 @@ cudaError_t launch_decode_bf16(const void* x, int64_t M, const void* w, int64_t 
 cudaError_t launch_decode_nvfp4(const uint8_t* x_codes, const uint8_t* x_scales, const float* alpha_x, int64_t M,
                                 const uint8_t* w_codes, const uint8_t* w_scales, const float* alpha_w, int64_t N,
                                 int64_t K, void* y, WsControl* ctrl, const DeviceInfo& di, cudaStream_t s);
+
+// Uniform-NVFP4 decode with the token quantization inside the kernel: X BF16
+// [M <= 128, K] is quantized (Eq. 2 / Eq. 3; dynamic alpha_x unless
+// alpha_static) by every CTA for its own K slice, straight into shared
+// memory.  Returns cudaErrorNotSupported (nothing launched) when no launch
+// shape fits the token slice in shared memory.
+cudaError_t launch_decode_nvfp4_fused(const void* x, int64_t M, const float* alpha_static, const uint8_t* w_codes,
+                                      const uint8_t* w_scales, const float* alpha_w, int64_t N, int64_t K, void* y,
+                                      WsControl* ctrl, const DeviceInfo& di, cudaStream_t s);
 
 // cuTensorMapEncodeTiled obtained from the driver at run time.
 bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t outer,

@@ -22,16 +22,6 @@ namespace mq {
 constexpr int kAmaxThreads = 512;
 constexpr int kAmaxUnroll = MQ_AMAX_UNROLL;
 
-// Per-halfword |bf16| maximum over the finite values of a 32-bit word pair,
-// plus a flag word that is non-zero if a NaN/Inf was seen.
-__device__ __forceinline__ void amax_accum(uint32_t w, uint32_t& mx, uint32_t& bad)
-{
-    const uint32_t mag = w & 0x7FFF7FFFu;
-    const uint32_t nonfin = __vcmpgeu2(mag, 0x7F807F80u);  // 0xFFFF per NaN/Inf halfword
-    bad |= nonfin;
-    mx = max_u16x2(mx, mag & ~nonfin);
-}
-
 // Fast path: magnitude maximum including NaN/Inf (two operations per word).
 // A maximum halfword >= 0x7F80 means a non-finite value was seen; only then
 // is the thread's range scanned again with amax_accum.
@@ -44,6 +34,8 @@ __global__ void __launch_bounds__(kAmaxThreads, MQ_AMAX_BLOCKS_PER_SM) amax_kern
                                                             float* __restrict__ alpha_out, WsControl* ctrl,
                                                             uint32_t* __restrict__ partials)
 {
+    grid_dep_wait();   // X may be the previous kernel's output
+    grid_dep_launch_dependents();
     uint32_t mx = 0, bad = 0;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     const int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -138,9 +130,8 @@ cudaError_t launch_amax(const void* x, int64_t n, float* alpha_out, WsControl* c
     if (blocks > cap) blocks = cap;
     if (blocks > kAmaxMaxBlocks) blocks = kAmaxMaxBlocks;
     if (blocks < 1) blocks = 1;
-    amax_kernel<<<(unsigned)blocks, kAmaxThreads, 0, s>>>(static_cast<const uint4*>(x), n_vec, alpha_out, ctrl,
-                                                         partials);
-    return cudaGetLastError();
+    return launch_pdl(amax_kernel, dim3((unsigned)blocks), dim3(kAmaxThreads), 0, s, static_cast<const uint4*>(x),
+                      n_vec, alpha_out, ctrl, partials);
 }
 
 // ==========================================================================
@@ -170,25 +161,12 @@ cudaError_t launch_amax(const void* x, int64_t n, float* alpha_out, WsControl* c
 constexpr int kQuantThreads = 256;
 constexpr int kQuantStepUnroll = MQ_QUANT_UNROLL;   // steps (2 rows per warp each) with loads in flight
 
-// Per-block constants of the Eq. 2 / Eq. 3 arithmetic for one tensor scale.
-struct QuantConsts {
-    float alpha_qmax;       // fl(alpha * q_max)
-    float inv_lo, inv_hi;   // floats bracketing 1 / alpha_qmax (see e4m3_block_scale)
-};
-
 // Fills enc_tab[c] = fl(1 / fl(alpha * sigma_c)) for every E4M3 code c (0 when
 // the product is 0) and returns the block-scale constants.  Every thread of
 // the block calls it; it ends with __syncthreads().
 __device__ __forceinline__ QuantConsts quant_setup(float alpha, float* enc_tab, float* dec_tab)
 {
-    QuantConsts q;
-    q.alpha_qmax = __fmul_rn(alpha, 6.0f);
-    // When fl(1/alpha_qmax) is not a normal finite float the bracket [0, inf]
-    // sends every block to the exact division.
-    const float inv_near = __frcp_rn(q.alpha_qmax);
-    const bool inv_normal = inv_near >= 1.17549435e-38f && inv_near < 3.0e38f;
-    q.inv_lo = inv_normal ? __uint_as_float(__float_as_uint(inv_near) - 1u) : 0.0f;
-    q.inv_hi = inv_normal ? __uint_as_float(__float_as_uint(inv_near) + 1u) : __int_as_float(0x7F800000);
+    const QuantConsts q = quant_consts(alpha);
     if (threadIdx.x < 128) {
         const float d = __fmul_rn(alpha, e4m3_to_float((uint32_t)threadIdx.x));
         enc_tab[threadIdx.x] = (d == 0.0f) ? 0.0f : __frcp_rn(d);
@@ -309,8 +287,9 @@ struct NormArgs {
 
 __device__ __forceinline__ uint32_t norm_pair(uint32_t xw, uint32_t gw, float r)
 {
-    const float lo = __fmul_rn(__fmul_rn(bf16_lo(xw), r), bf16_lo(gw));
-    const float hi = __fmul_rn(__fmul_rn(bf16_hi(xw), r), bf16_hi(gw));
+    float t0, t1, lo, hi;
+    fmul2_rn(bf16_lo(xw), bf16_hi(xw), r, t0, t1);             // fl(x * rstd)
+    fmul2v_rn(t0, t1, bf16_lo(gw), bf16_hi(gw), lo, hi);       // fl(fl(x * rstd) * gamma)
     const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<const uint32_t*>(&p);
 }
@@ -404,10 +383,6 @@ __device__ __forceinline__ void quant_tile(const uint16_t* __restrict__ x, int64
     __syncthreads();
 }
 
-__device__ __forceinline__ uint32_t fold_max_flag(uint32_t a, uint32_t b)
-{
-    return max(a & 0x7FFFFFFFu, b & 0x7FFFFFFFu) | ((a | b) & 0x80000000u);
-}
 
 __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p)
 {
@@ -449,9 +424,11 @@ __global__ void __launch_bounds__(kQuantThreads, MQ_QUANT_MIN_BLOCKS)
     const int blk = lane & 15;
     const int64_t chunks = (K + 255) / 256;
     const int64_t tiles = ((rows + 127) / 128) * chunks;
-    // a consumer launched with programmatic serialization (the uniform-NVFP4
-    // decode) may start now: it streams its weights and waits for this grid
-    // before it reads the quantized tokens
+    // X, the tensor scale and the outputs may be touched by the previous kernel
+    // of the stream; a consumer launched with programmatic serialization (the
+    // uniform-NVFP4 decode, the GEMM) may start now and waits for this grid
+    // before it reads what this kernel writes
+    grid_dep_wait();
     grid_dep_launch_dependents();
 
     float alpha;
@@ -580,8 +557,13 @@ cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float*
     cfg.dynamicSmemBytes = 0;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = single ? 1 : 0;   // blocks wait on one another only in the single-launch amax
+    if (single) {   // blocks wait on one another only in the single-launch amax
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+    } else {
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+    }
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     auto kern = scale_search ? quantize_kernel<true, false> : quantize_kernel<false, false>;
@@ -602,16 +584,7 @@ cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float*
 // maxima into alpha_h = amax/2688 (1 if 0; NaN/Inf excluded and reported).
 // Pass 2 is quantize_kernel<false, true>, which forms h again on load.
 constexpr int kNormThreads = 256;
-
-// (hi, lo) += b with Knuth's TwoSum: hi + lo keeps the sum to about 48 bits.
-__device__ __forceinline__ void ff_add(float& hi, float& lo, float b)
-{
-    const float s = __fadd_rn(hi, b);
-    const float bp = __fsub_rn(s, hi);
-    const float e = __fadd_rn(__fsub_rn(hi, __fsub_rn(s, bp)), __fsub_rn(b, bp));
-    hi = s;
-    lo = __fadd_rn(lo, e);
-}
+constexpr int64_t kNormGammaSmem = 8192;   // gamma elements staged in shared memory (16 KiB)
 
 __global__ void __launch_bounds__(kNormThreads) rmsnorm_amax_kernel(const uint16_t* __restrict__ x, int64_t rows,
                                                                     int64_t K, const uint16_t* __restrict__ gamma,
@@ -619,6 +592,8 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_amax_kernel(const uint16
                                                                     float* __restrict__ alpha_out, WsControl* ctrl,
                                                                     uint32_t* __restrict__ partials)
 {
+    grid_dep_wait();   // X may be the previous kernel's output
+    grid_dep_launch_dependents();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t wstride = (int64_t)gridDim.x * (kNormThreads / 32);
     uint32_t mx = 0, bad = 0;
@@ -626,19 +601,30 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_amax_kernel(const uint16
     // flight at once; a row of at most one chunk (K <= 4096) stays in
     // registers for the |h| pass, longer rows are read again (from L2).
     constexpr int kNormChunk = 16;
-    const uint4* gr = reinterpret_cast<const uint4*>(gamma);
     const int64_t nv = K / 8;
     const int64_t chunk = 32 * kNormChunk;
+    // gamma, read by every row, staged once per block in shared memory when it
+    // fits (K <= kNormGammaSmem elements)
+    extern __shared__ uint4 s_gamma[];
+    const bool g_smem = K <= kNormGammaSmem;
+    if (g_smem)
+        for (int64_t i = threadIdx.x; i < nv; i += kNormThreads) s_gamma[i] = __ldg(reinterpret_cast<const uint4*>(gamma) + i);
+    __syncthreads();
+    const uint4* gr = g_smem ? s_gamma : reinterpret_cast<const uint4*>(gamma);
+    // Each warp takes rows r, r + wstride, ...; while it works on one row, the
+    // next one is prefetched into L2 with one bulk prefetch.
     for (int64_t r = (int64_t)blockIdx.x * (kNormThreads / 32) + warp; r < rows; r += wstride) {
         const uint4* xr = reinterpret_cast<const uint4*>(x + r * K);
+        if (lane == 0 && r + wstride < rows)
+            bulk_prefetch_l2(x + (r + wstride) * K, (uint32_t)std::min<int64_t>(K * 2, (int64_t)1 << 20));
         uint4 v[kNormChunk];
         // sum of squares: each square of a BF16 value is exact in binary32
-        // (8 significant bits, for |x| in [2^-63, 2^63]); the running sum is an
-        // unevaluated pair (about 48 bits), converted to binary64 once per row,
-        // which stands for the binary64 sum of the definition (the two agree
-        // unless the sum lies within ~2^-45 relative of an FP32 rounding
-        // boundary of ms).  FP64 conversions per element would be the slow path.
-        float hi0 = 0.0f, lo0 = 0.0f, hi1 = 0.0f, lo1 = 0.0f;
+        // (8 significant bits, for |x| in [2^-63, 2^63]) and is added in
+        // binary64 (two running sums per lane, then a butterfly over the warp):
+        // the binary64 sum of the definition up to the order of the additions,
+        // which moves ms only when the sum lies within ~2^-40 relative of an
+        // FP32 rounding boundary.
+        double s[4] = {0.0, 0.0, 0.0, 0.0};   // four independent chains
         for (int64_t c0 = 0; c0 < nv; c0 += chunk) {
 #pragma unroll
             for (int u = 0; u < kNormChunk; ++u) {
@@ -651,21 +637,16 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_amax_kernel(const uint16
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const float a = bf16_lo(w[j]), b = bf16_hi(w[j]);
-                    ff_add(hi0, lo0, __fmul_rn(a, a));
-                    ff_add(hi1, lo1, __fmul_rn(b, b));
+                    float a2, b2;
+                    fmul2v_rn(a, b, a, b, a2, b2);
+                    s[(j & 1) * 2] = __dadd_rn(s[(j & 1) * 2], (double)a2);
+                    s[(j & 1) * 2 + 1] = __dadd_rn(s[(j & 1) * 2 + 1], (double)b2);
                 }
             }
         }
-        ff_add(hi0, lo0, hi1);
-        lo0 = __fadd_rn(lo0, lo1);
+        double ss = __dadd_rn(__dadd_rn(s[0], s[1]), __dadd_rn(s[2], s[3]));
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float oh = __shfl_xor_sync(0xFFFFFFFFu, hi0, o);
-            const float ol = __shfl_xor_sync(0xFFFFFFFFu, lo0, o);
-            ff_add(hi0, lo0, oh);
-            lo0 = __fadd_rn(lo0, ol);
-        }
-        const double ss = __dadd_rn((double)hi0, (double)lo0);
+        for (int o = 16; o > 0; o >>= 1) ss = __dadd_rn(ss, __shfl_xor_sync(0xFFFFFFFFu, ss, o));
         const float ms = __double2float_rn(__ddiv_rn(ss, (double)K));
         const float rs = __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(__dadd_rn((double)ms, (double)eps))));
         if (lane == 0) rstd[r] = rs;
@@ -681,7 +662,7 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_amax_kernel(const uint16
             for (int u = 0; u < kNormChunk; ++u) {
                 const int64_t i = c0 + lane + 32 * u;
                 if (i < nv) {
-                    const uint4 g = __ldg(gr + i);
+                    const uint4 g = g_smem ? gr[i] : __ldg(gr + i);
                     amax_accum(norm_pair(v[u].x, g.x, rs), mx, bad);
                     amax_accum(norm_pair(v[u].y, g.y, rs), mx, bad);
                     amax_accum(norm_pair(v[u].z, g.z, rs), mx, bad);
@@ -730,24 +711,29 @@ cudaError_t launch_rmsnorm_quantize(const void* x, int64_t rows, int64_t K, cons
                                     float* rstd, uint8_t* codes, uint8_t* scales, float* alpha_out, void* h_out,
                                     WsControl* ctrl, uint32_t* partials, const DeviceInfo& di, cudaStream_t s)
 {
+    // one wave of resident blocks; every warp then walks several rows
+    const size_t gsmem = (K <= kNormGammaSmem) ? (size_t)K * 2 : 0;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rmsnorm_amax_kernel, kNormThreads, gsmem) != cudaSuccess) {
+        (void)cudaGetLastError();
+        per_sm = 1;
+    }
     int64_t blocks = (rows + kNormThreads / 32 - 1) / (kNormThreads / 32);
-    blocks = std::min<int64_t>(blocks, (int64_t)di.num_sms * 8);
+    blocks = std::min<int64_t>(blocks, (int64_t)di.num_sms * std::max(1, per_sm));
     blocks = std::min<int64_t>(blocks, kAmaxMaxBlocks);
     blocks = std::max<int64_t>(blocks, 1);
-    rmsnorm_amax_kernel<<<(unsigned)blocks, kNormThreads, 0, s>>>(static_cast<const uint16_t*>(x), rows, K,
-                                                                  static_cast<const uint16_t*>(gamma), eps, rstd,
-                                                                  alpha_out, ctrl, partials);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(rmsnorm_amax_kernel, dim3((unsigned)blocks), dim3(kNormThreads), gsmem, s,
+                               static_cast<const uint16_t*>(x), rows, K, static_cast<const uint16_t*>(gamma), eps,
+                               rstd, alpha_out, ctrl, partials);
     if (e != cudaSuccess) return e;
     const int64_t tiles = ((rows + 127) / 128) * ((K + 255) / 256);
     const int occ = quantize_blocks_per_sm<false, true>(di);
     int64_t qb = std::min(tiles, (int64_t)di.num_sms * std::max(1, occ));
     qb = std::max<int64_t>(qb, 1);
     NormArgs na{static_cast<const uint16_t*>(gamma), rstd, static_cast<uint16_t*>(h_out)};
-    quantize_kernel<false, true><<<(unsigned)qb, kQuantThreads, 0, s>>>(static_cast<const uint16_t*>(x), rows, K,
-                                                                         alpha_out, alpha_out, codes, scales, 0, ctrl,
-                                                                         partials, na);
-    return cudaGetLastError();
+    return launch_pdl(quantize_kernel<false, true>, dim3((unsigned)qb), dim3(kQuantThreads), 0, s,
+                      static_cast<const uint16_t*>(x), rows, K, static_cast<const float*>(alpha_out), alpha_out,
+                      codes, scales, (int64_t)0, ctrl, partials, na);
 }
 
 __global__ void selftest_e2m1_kernel(unsigned long long* counts)

@@ -62,10 +62,14 @@ def _nvfp4_decode_check(x, w, y_gpu_bits, alpha_x=None):
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 256, 256), (7, 400, 1088), (32, 512, 1024), (64, 768, 2048),
-                                   (100, 272, 320), (128, 128, 4096), (1, 4096, 12288)])
+                                   (100, 272, 320), (128, 128, 4096), (1, 4096, 12288), (1, 12288, 4096),
+                                   (8, 12288, 4096), (64, 12288, 4096), (128, 4096, 12288)])
 def test_decode_nvfp4_vs_oracle(M, N, K):
     """Ragged tokens (MMA N padded to 32), ragged weight rows (N % 128 != 0) and a partial last
-    256-element stage (K % 256 != 0) are all covered."""
+    256-element stage (K % 256 != 0) are all covered, as are the launch shapes the call picks:
+    the single kernel that quantizes the tokens itself (K split over clusters of 1 to 8 CTAs
+    exchanging their slice maxima) and, where the token slice does not fit in shared memory
+    (128 tokens, K = 12288), the quantization kernel followed by the decode GEMM."""
     x = wl.heavy_tailed_bf16(M, K, 3 * M + K)
     w = wl.normal_bf16(N, K, 0.02, 5 * N + K)
     Wq = mq.quantize_weight(to_dev(w))
@@ -113,3 +117,21 @@ def test_decode_nvfp4_matches_prefill_on_same_weight():
     wc, wsc = oracle.quantize(w[:2048], aw)
     y64, sabs = oracle.nvfp4_linear_rows((*oracle.quantize(x, ax), ax), (wc, wsc, aw))
     gemm_check(to_host_bits(yd)[:, :2048], y64, sabs)
+
+
+def test_decode_nvfp4_reports_nonfinite_tokens():
+    """A NaN among the tokens is excluded from the tensor amax and reported as MQ_ERR_NONFINITE;
+    the other tokens are still quantized with the finite maximum."""
+    x = wl.heavy_tailed_bf16(4, 2048, 91)
+    x[2, 777] = 0x7FC0                       # BF16 NaN
+    w = wl.normal_bf16(512, 2048, 0.02, 92)
+    Wq = mq.quantize_weight(to_dev(w))
+    ws = mq.workspace(4, 2048)
+    y = mq.decode_linear_nvfp4(to_dev(x), Wq, ws=ws)
+    assert mq.async_status(ws) == 5          # MQ_ERR_NONFINITE
+    finite = np.array([0, 1, 3])
+    xf = x.copy()
+    xf[2, 777] = 0
+    ax = oracle.tensor_alpha(x)[1]           # NaN excluded, as on the device
+    assert ax == oracle.tensor_alpha(xf)[1]
+    _nvfp4_decode_check(x[finite], w, to_host_bits(y)[finite], alpha_x=ax)
