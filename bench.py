@@ -368,7 +368,7 @@ def _decode_pair(mq, torch, dev, wl, Wm, Wq, hbm_gbs, reps, seed):
     for M in (1, 8, 32, 64):
         x = _to_dev(torch, wl.heavy_tailed_bf16(M, K, seed + M), dev)
         y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-        wsd = mq.workspace(M, K, device=dev)
+        wsd = mq.decode_workspace(M, N, K, device=dev)
         bf = [lambda W=W: mq.decode_linear(x, W, Y=y, ws=wsd) for W in Wm_copies]
         q4 = [lambda W=W: mq.decode_linear_nvfp4(x, W, Y=y, ws=wsd) for W in Wq_copies]
         for f in bf + q4:

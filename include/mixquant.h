@@ -161,11 +161,23 @@ MQ_API mq_status mq_prefill_linear(const void* X_bf16, const mq_nvfp4* X_q, int6
                             mq_epilogue epi, const float* alpha_static, const float* alpha_h, void* Y,
                             const mq_nvfp4* H_out, void* h_debug, void* ws, size_t ws_bytes, mq_stream_t stream);
 
+/* Workspace bytes for mq_decode_linear and mq_decode_linear_nvfp4 on M
+ * tokens and an [N, K] weight: what mq_workspace_bytes(M, K) covers (its
+ * control block also holds one counter per 128 weight rows, for N up to
+ * 253952) and room for the FP32 partial sums of the K dimension split across
+ * up to 8 CTAs per 128 weight rows (8 * ceil(N/128) * M * 512 bytes).  With it, the decode splits K across independent CTAs that
+ * add their partials in a fixed order, so the weight stream covers every SM;
+ * a smaller workspace (at least MQ_WS_CONTROL_BYTES, or mq_workspace_bytes(M,
+ * K) for the NVFP4 decode) still works, with the K split limited to thread-
+ * block clusters.  Zero-filled once, like every workspace. */
+MQ_API size_t mq_decode_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
 /*
  * The precise decode path (section 3.3: decoding stays on the original BF16
  * weights): Y[M, N] = bf16(sum_k X[m, k] W[n, k]) with FP32 accumulation on
  * the tensor cores.  X BF16 [M, K] with 1 <= M <= 256, W BF16 [N, K], Y BF16
- * [M, N].  ws: >= MQ_WS_CONTROL_BYTES (error reporting only).
+ * [M, N].  ws: >= MQ_WS_CONTROL_BYTES; mq_decode_workspace_bytes(M, N, K)
+ * for the fastest launch shape.
  */
 MQ_API mq_status mq_decode_linear(const void* X_bf16, int64_t M, const void* W_bf16, int64_t N, int64_t K, void* Y_bf16,
                            void* ws, size_t ws_bytes, mq_stream_t stream);
@@ -277,7 +289,8 @@ MQ_API mq_status mq_rmsnorm_quantize(const void* X_bf16, int64_t M, int64_t K, c
  * weight from mq_quantize_weight (not gate/up interleaved).  The same weight
  * bytes as the prefill path; 0.5625 instead of 2 bytes per weight element
  * streamed per token batch.  M in [1, 128]; K % 64 == 0; N % 16 == 0; X and
- * Y 16-byte aligned.  Workspace: mq_workspace_bytes(M, K), zero-filled once.
+ * Y 16-byte aligned.  Workspace: mq_workspace_bytes(M, K), zero-filled once;
+ * mq_decode_workspace_bytes(M, N, K) for the fastest launch shape.
  * Errors as mq_prefill_linear. */
 MQ_API mq_status mq_decode_linear_nvfp4(const void* X_bf16, int64_t M, const mq_nvfp4* W, const float* alpha_static,
                                         void* Y_bf16, void* ws, size_t ws_bytes, mq_stream_t stream);

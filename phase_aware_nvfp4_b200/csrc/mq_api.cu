@@ -124,6 +124,35 @@ Ws carve(void* ws, int64_t M, int64_t K)
     return w;
 }
 
+// Decode workspace: the per-tile counters of the split-K reduction across
+// independent CTAs sit in the control block, behind the amax partials, at an
+// offset that does not depend on the shapes (so one workspace serves calls of
+// any shape: every counter is zero between calls); the FP32 partial tiles
+// follow what mq_workspace_bytes(M, K) covers (control block and the tokens'
+// NVFP4 copy), up to kDecodeMaxSplit CTAs per tile, M rows of 128 each.
+constexpr int64_t kDecodeMaxSplit = 8;
+constexpr size_t kDecodeCtrOffset = kWsPartialsOffset + (size_t)kAmaxMaxBlocks * 4u;
+constexpr int64_t kDecodeMaxTiles = (int64_t)((kWsControlBytes - kDecodeCtrOffset) / 4u);
+static_assert(kDecodeCtrOffset < kWsControlBytes, "decode counters inside the control block");
+
+size_t decode_ws_bytes(int64_t M, int64_t N, int64_t K)
+{
+    const int64_t n_tiles = (N + 127) / 128;
+    return align_up(ws_bytes_for(M, K), 256) + (size_t)kDecodeMaxSplit * (size_t)n_tiles * (size_t)M * 128u * 4u;
+}
+
+DecodeSplitWs decode_split_ws(void* ws, size_t ws_bytes, int64_t M, int64_t N, int64_t K)
+{
+    const int64_t n_tiles = (N + 127) / 128;
+    const size_t part_off = align_up(ws_bytes_for(M, K), 256);
+    const size_t two_splits = 2u * (size_t)n_tiles * (size_t)M * 128u * 4u;
+    if (n_tiles > kDecodeMaxTiles || ws_bytes < part_off + two_splits)
+        return DecodeSplitWs{nullptr, nullptr, 0};   // the K split stays inside clusters
+    uint8_t* b = static_cast<uint8_t*>(ws);
+    return DecodeSplitWs{reinterpret_cast<float*>(b + part_off), reinterpret_cast<uint32_t*>(b + kDecodeCtrOffset),
+                         ws_bytes - part_off};
+}
+
 mq_status check_ws(void* ws, size_t ws_bytes, size_t need)
 {
     if (ws == nullptr || ws_bytes < need) return MQ_ERR_WORKSPACE;
@@ -184,6 +213,12 @@ mq_status mq_nvfp4_sizes(int64_t rows, int64_t cols, size_t* codes_bytes, size_t
 }
 
 size_t mq_workspace_bytes(int64_t M, int64_t K) { return ws_bytes_for(M, K); }
+
+size_t mq_decode_workspace_bytes(int64_t M, int64_t N, int64_t K)
+{
+    if (M < 1 || N < 1 || K < 1) return kWsControlBytes;
+    return decode_ws_bytes(M, N, K);
+}
 
 mq_status mq_quantize_weight(const void* W_bf16, int64_t N, int64_t K, int gate_up_interleave, const mq_nvfp4* out,
                              void* ws, size_t ws_bytes, mq_stream_t stream)
@@ -400,8 +435,9 @@ mq_status mq_decode_linear(const void* X_bf16, int64_t M, const void* W_bf16, in
     DeviceInfo di;
     if ((st = check_device(&di)) != MQ_OK) return st;
     const Ws w = carve(ws, 0, 0);
+    const DecodeSplitWs sw = decode_split_ws(ws, ws_bytes, M, N, K);
     return cuda_status(
-        launch_decode_bf16(X_bf16, M, W_bf16, N, K, Y_bf16, w.ctrl, di, reinterpret_cast<cudaStream_t>(stream)));
+        launch_decode_bf16(X_bf16, M, W_bf16, N, K, Y_bf16, w.ctrl, sw, di, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 mq_status mq_decode_linear_nvfp4(const void* X_bf16, int64_t M, const mq_nvfp4* W, const float* alpha_static,
@@ -420,16 +456,17 @@ mq_status mq_decode_linear_nvfp4(const void* X_bf16, int64_t M, const mq_nvfp4* 
     if ((st = check_device(&di)) != MQ_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const Ws w = carve(ws, M, K);
+    const DecodeSplitWs sw = decode_split_ws(ws, ws_bytes, M, N, K);
     // One kernel that quantizes the tokens itself; when its token slice does not
     // fit in shared memory, the quantization kernel and then the decode GEMM.
     const cudaError_t fe = launch_decode_nvfp4_fused(X_bf16, M, alpha_static, W->codes, W->scales, W->alpha, N, K,
-                                                     Y_bf16, w.ctrl, di, s);
+                                                     Y_bf16, w.ctrl, sw, di, s);
     if (fe != cudaErrorNotSupported) return cuda_status(fe);
     const float* ax = nullptr;
     st = quantize_into(X_bf16, M, K, alpha_static, w.xq_codes, w.xq_scales, &w.ctrl->alpha, false, 0, w, di, s, &ax);
     if (st != MQ_OK) return st;
     return cuda_status(launch_decode_nvfp4(w.xq_codes, w.xq_scales, ax, M, W->codes, W->scales, W->alpha, N, K, Y_bf16,
-                                           w.ctrl, di, s));
+                                           w.ctrl, sw, di, s));
 }
 
 mq_status mq_unswizzle_scales(const mq_nvfp4* t, uint8_t* rowmajor_out, mq_stream_t stream)

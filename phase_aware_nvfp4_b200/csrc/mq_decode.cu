@@ -46,7 +46,38 @@ struct DParams {
     const float* alpha_x;
     uint16_t* y;
     WsControl* ctrl;
+    // K split across independent CTAs (gpart != 0) instead of a cluster: each
+    // writes its FP32 partial tile to `part`, the last of a tile's CTAs (by
+    // the per-tile counter) adds them in rank order and writes Y
+    int gpart;
+    float* part;
+    uint32_t* tile_ctr;
 };
+
+// Split-K reduction through global memory for one 128-row decode tile, run by
+// the 128 epilogue threads (named barrier 2; `row` = TMEM lane = W row of the
+// tile).  Every CTA of the tile has stored its partial part[tile][rank][m][row]
+// for m < M; the CTA that takes the last ticket of the tile's counter adds
+// the `split` partials in rank order (so the result does not depend on which
+// CTA finishes last), scales by out_scale and writes Y[m][n] in BF16, and
+// resets the counter for the next call.
+__device__ __forceinline__ void gsplit_reduce(float* part, uint32_t* tile_ctr, uint32_t* s_flag, int tile, int split,
+                                              int M, int N, int row, int lead, float out_scale, uint16_t* y)
+{
+    __threadfence();
+    named_barrier_sync(2, 128);
+    if (lead) *s_flag = (atomicAdd(&tile_ctr[tile], 1u) == (uint32_t)(split - 1)) ? 1u : 0u;
+    named_barrier_sync(2, 128);
+    if (*s_flag == 0u) return;
+    __threadfence();
+    const int64_t n = (int64_t)tile * DBM + row;
+    for (int m = 0; m < M; ++m) {
+        float acc = 0.0f;
+        for (int q = 0; q < split; ++q) acc += __ldcg(part + (((int64_t)tile * split + q) * M + m) * DBM + row);
+        if (n < N) y[(int64_t)m * N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(acc, out_scale)));
+    }
+    if (lead) tile_ctr[tile] = 0u;
+}
 
 __device__ __forceinline__ uint32_t cluster_rank()
 {
@@ -92,10 +123,11 @@ __global__ void __launch_bounds__(D_THREADS, 1)
     uint64_t* acc_full = empty_bar + p.stages;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
     volatile uint32_t* abort_flag = tmem_slot + 1;
+    uint32_t* s_last = tmem_slot + 2;
     float* red = reinterpret_cast<float*>(smem);  // [MT][128] partials, reuses the pipeline buffers
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint32_t rank = (p.split > 1) ? cluster_rank() : 0u;
+    const uint32_t rank = (p.split > 1) ? (p.gpart ? (uint32_t)(blockIdx.x % p.split) : cluster_rank()) : 0u;
     const int n_tile = blockIdx.x / p.split;
     const int ks_begin = (int)(((int64_t)p.k_stages * rank) / p.split);
     const int ks_end = (int)(((int64_t)p.k_stages * (rank + 1)) / p.split);
@@ -270,7 +302,9 @@ __global__ void __launch_bounds__(D_THREADS, 1)
             for (int j = 0; j < 16; ++j) {
                 const int m = 16 * c + j;
                 const float v = (have_acc && ok) ? __uint_as_float(r[j]) : 0.0f;
-                if (p.split > 1) {
+                if (p.split > 1 && p.gpart) {
+                    if (m < p.M) p.part[(((int64_t)n_tile * p.split + rank) * p.M + m) * DBM + row] = v;
+                } else if (p.split > 1) {
                     red[m * DBM + row] = v;
                 } else if (m < p.M && n < p.N) {
                     const float o = FMT ? __fmul_rn(v, out_scale) : v;
@@ -278,9 +312,12 @@ __global__ void __launch_bounds__(D_THREADS, 1)
                 }
             }
         }
+        if (p.split > 1 && p.gpart)
+            gsplit_reduce(p.part, p.tile_ctr, s_last, n_tile, p.split, p.M, p.N, row, warp == 2 && lane == 0,
+                          FMT ? out_scale : 1.0f, p.y);
     }
 
-    if (p.split > 1) {
+    if (p.split > 1 && !p.gpart) {
         // Every CTA of the cluster has its partial tile in shared memory; CTA
         // `rank` reduces tokens m = rank, rank + split, ... in rank order.
         cluster_sync_all();
@@ -390,6 +427,57 @@ int choose_shape(DParams& p, int n_tiles, const DeviceInfo& di)
     return p.bar_offset + 256 + 1024;
 }
 
+// Bytes of shared memory that keep the CTAs sharing an SM within its 512 TMEM
+// columns (each CTA allocates tmem_cols): smem is padded so that at most
+// 512 / tmem_cols CTAs fit.
+inline int pad_smem_for_tmem(int smem, uint32_t tmem_cols, const DeviceInfo& di)
+{
+    const int cap = 512 / (int)tmem_cols;
+    const int per_sm_min = (int)(di.smem_per_sm / (size_t)(cap + 1)) + 1;   // bytes incl. the runtime's reserve
+    smem = std::max<int>(smem, per_sm_min - (int)di.smem_reserved_per_cta);
+    return (smem + 1023) / 1024 * 1024;
+}
+
+// Launch shape with the K dimension split across independent CTAs that add
+// their FP32 partials through `part_bytes` of global workspace (gsplit_reduce):
+// unlike a cluster split, any number of CTAs per SM and any split 1..8 can be
+// used, so the weight stream can cover every SM.  One wave; the most weight
+// bytes in flight (saturating at ~16 MB) wins, then the grid closest to two
+// CTAs per SM.  Returns the dynamic shared memory size, or 0 when nothing fits.
+template <int FMT>
+int choose_shape_gpart(DParams& p, int n_tiles, const DeviceInfo& di, size_t part_bytes)
+{
+    constexpr int64_t kSaturateBytes = 16ll << 20;
+    const int stage_bytes = p.stage_bytes;
+    int best_split = 0, best_stages = 0, best_smem = 0;
+    int64_t best_score = -1;
+    for (int sp = 1; sp <= 8 && sp <= p.k_stages; ++sp) {
+        if (sp > 1 && (size_t)sp * n_tiles * p.M * DBM * 4 > part_bytes) break;
+        const int per_cta_stages = (p.k_stages + sp - 1) / sp;
+        for (int st = std::min(12, per_cta_stages); st >= std::min(2, per_cta_stages); --st) {
+            const int smem = pad_smem_for_tmem(st * stage_bytes + 256 + 1024, p.tmem_cols, di);
+            if ((size_t)smem > di.max_smem_optin) continue;
+            const int active = max_resident_ctas<FMT>(1, smem, di);
+            const int ctas = n_tiles * sp;
+            if (active <= 0 || ctas > active) continue;
+            const int64_t score = std::min<int64_t>(kSaturateBytes, (int64_t)ctas * st * stage_bytes) * 4096 +
+                                  std::min(ctas, 2 * di.num_sms);
+            if (score > best_score) {
+                best_score = score;
+                best_split = sp;
+                best_stages = st;
+                best_smem = smem;
+            }
+        }
+    }
+    if (best_split == 0) return 0;
+    p.split = best_split;
+    p.stages = best_stages;
+    p.gpart = 1;
+    p.bar_offset = p.stages * stage_bytes;
+    return best_smem;
+}
+
 template <int FMT>
 cudaError_t launch_shape(const DParams& p, int n_tiles, int smem, const CUtensorMap& tw, const CUtensorMap& tx,
                          const CUtensorMap& tsfw, const CUtensorMap& tsfx, cudaStream_t s)
@@ -404,7 +492,7 @@ cudaError_t launch_shape(const DParams& p, int n_tiles, int smem, const CUtensor
     cfg.stream = s;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)p.split;
+    attr[0].val.clusterDim.x = p.gpart ? 1u : (unsigned)p.split;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     // let the kernel be scheduled while its predecessor on the stream drains
@@ -453,6 +541,11 @@ struct FParams {
     uint32_t tmem_cols, tmem_sf;
     uint16_t* y;
     WsControl* ctrl;
+    // K split across independent CTAs (see DParams): every CTA then takes the
+    // amax over all of X itself instead of exchanging slice maxima in a cluster
+    int gpart;
+    float* part;
+    uint32_t* tile_ctr;
 };
 
 __global__ void __launch_bounds__(F_THREADS, 1)
@@ -470,12 +563,14 @@ __global__ void __launch_bounds__(F_THREADS, 1)
     uint32_t* red_q = amax_slot + 8;                                   // [F_QTHREADS / 32]
     uint32_t* tmem_slot = red_q + F_QTHREADS / 32;
     volatile uint32_t* abort_flag = tmem_slot + 1;
+    uint32_t* s_last = tmem_slot + 2;
     float* enc_tab = reinterpret_cast<float*>(smem + p.bar_offset + 1024);   // [128]
     uint8_t* xr = smem + p.x_off;
     float* red = reinterpret_cast<float*>(smem);   // [MT][128] split-K partials, after the MMAs
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint32_t rank = (p.split > 1) ? cluster_rank() : 0u;
+    const bool cluster = p.split > 1 && !p.gpart;
+    const uint32_t rank = (p.split > 1) ? (p.gpart ? (uint32_t)(blockIdx.x % p.split) : cluster_rank()) : 0u;
     const int n_tile = blockIdx.x / p.split;
     const int ks_begin = (int)(((int64_t)p.k_stages * rank) / p.split);
     const int ks_end = (int)(((int64_t)p.k_stages * (rank + 1)) / p.split);
@@ -496,7 +591,7 @@ __global__ void __launch_bounds__(F_THREADS, 1)
     if (warp == 1) tmem_alloc(tmem_slot, p.tmem_cols);
     tc_fence_before();
     __syncthreads();
-    if (p.split > 1) cluster_sync_all();   // every peer's barriers exist before any remote arrival
+    if (cluster) cluster_sync_all();   // every peer's barriers exist before any remote arrival
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     float alpha_x = 1.0f;
@@ -593,12 +688,14 @@ __global__ void __launch_bounds__(F_THREADS, 1)
         if (p.alpha_static != nullptr) {
             alpha_x = __ldg(p.alpha_static);
         } else {
-            // |x| maximum of the slice (NaN/Inf excluded and flagged, as the amax pass does)
-            const int vpr = (k_hi - k_lo) / 8;
+            // |x| maximum of the slice (NaN/Inf excluded and flagged, as the amax pass
+            // does); without a cluster to exchange slice maxima, of all of X
+            const int a_lo = cluster ? k_lo : 0, a_hi = cluster ? k_hi : p.K;
+            const int vpr = (a_hi - a_lo) / 8;
             uint32_t mx = 0, bad = 0;
             for (int v = qt; v < p.M * vpr; v += F_QTHREADS) {
                 const int m = v / vpr, c = v - m * vpr;
-                const uint4 q = __ldg(reinterpret_cast<const uint4*>(p.x + (int64_t)m * p.K + k_lo) + c);
+                const uint4 q = __ldg(reinterpret_cast<const uint4*>(p.x + (int64_t)m * p.K + a_lo) + c);
                 amax_accum(q.x, mx, bad);
                 amax_accum(q.y, mx, bad);
                 amax_accum(q.z, mx, bad);
@@ -611,7 +708,7 @@ __global__ void __launch_bounds__(F_THREADS, 1)
             named_barrier_sync(1, F_QTHREADS);
             b = 0;
             for (int w = 0; w < F_QTHREADS / 32; ++w) b = fold_max_flag(b, red_q[w]);
-            if (p.split > 1) {
+            if (cluster) {
                 // every rank's slice maximum into every rank's slot; the slots of all
                 // ranks together cover K, so their fold is the maximum over all of X
                 if (qt == 0) {
@@ -676,17 +773,22 @@ __global__ void __launch_bounds__(F_THREADS, 1)
                 for (int j = 0; j < 16; ++j) {
                     const int m = 16 * c + j;
                     const float v = have ? __uint_as_float(r[j]) : 0.0f;
-                    if (p.split > 1) {
+                    if (p.split > 1 && p.gpart) {
+                        if (m < p.M) p.part[(((int64_t)n_tile * p.split + rank) * p.M + m) * DBM + row] = v;
+                    } else if (p.split > 1) {
                         red[m * DBM + row] = v;
                     } else if (m < p.M && n < p.N) {
                         p.y[(int64_t)m * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(v, out_scale)));
                     }
                 }
             }
+            if (p.split > 1 && p.gpart)
+                gsplit_reduce(p.part, p.tile_ctr, s_last, n_tile, p.split, p.M, p.N, row,
+                              warp == 2 && lane == 0, out_scale, p.y);
         }
     }
 
-    if (p.split > 1) {
+    if (cluster) {
         // every CTA of the cluster holds its partial tile; CTA `rank` sums tokens
         // m = rank, rank + split, ... over the ranks in rank order
         cluster_sync_all();
@@ -722,7 +824,13 @@ int fused_resident_ctas(int cluster, int smem, const DeviceInfo& di)
     auto it = cache.find(key);
     if (it != cache.end()) return it->second;
     int ctas = 0;
-    if (cudaFuncSetAttribute(decode_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess) {
+    if (cudaFuncSetAttribute(decode_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
+        // nothing fits
+    } else if (cluster == 1) {
+        int per_sm = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_fused_kernel, F_THREADS, smem) == cudaSuccess)
+            ctas = per_sm * di.num_sms;
+    } else {
         cudaLaunchConfig_t cfg{};
         cfg.gridDim = dim3((unsigned)(cluster * di.num_sms), 1, 1);
         cfg.blockDim = dim3(F_THREADS, 1, 1);
@@ -745,7 +853,7 @@ int fused_resident_ctas(int cluster, int smem, const DeviceInfo& di)
 }  // namespace
 
 cudaError_t launch_decode_bf16(const void* x, int64_t M, const void* w, int64_t N, int64_t K, void* y,
-                               WsControl* ctrl, const DeviceInfo& di, cudaStream_t s)
+                               WsControl* ctrl, const DecodeSplitWs& sw, const DeviceInfo& di, cudaStream_t s)
 {
     DParams p{};
     p.M = (int)M;
@@ -759,7 +867,10 @@ cudaError_t launch_decode_bf16(const void* x, int64_t M, const void* w, int64_t 
     p.ctrl = ctrl;
     p.stage_bytes = W_STAGE + p.MT * DBK * 2;
     const int n_tiles = (int)((N + DBM - 1) / DBM);
-    const int smem = choose_shape<0>(p, n_tiles, di);
+    p.part = sw.part;
+    p.tile_ctr = sw.tile_ctr;
+    int smem = (sw.part != nullptr) ? choose_shape_gpart<0>(p, n_tiles, di, sw.part_bytes) : 0;
+    if (smem == 0) smem = choose_shape<0>(p, n_tiles, di);
 
     CUtensorMap tw, tx;
     if (!make_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w, (uint64_t)K, (uint64_t)N, (uint64_t)K * 2, DBK, DBM,
@@ -773,7 +884,8 @@ cudaError_t launch_decode_bf16(const void* x, int64_t M, const void* w, int64_t 
 
 cudaError_t launch_decode_nvfp4(const uint8_t* x_codes, const uint8_t* x_scales, const float* alpha_x, int64_t M,
                                 const uint8_t* w_codes, const uint8_t* w_scales, const float* alpha_w, int64_t N,
-                                int64_t K, void* y, WsControl* ctrl, const DeviceInfo& di, cudaStream_t s)
+                                int64_t K, void* y, WsControl* ctrl, const DecodeSplitWs& sw, const DeviceInfo& di,
+                                cudaStream_t s)
 {
     DParams p{};
     p.M = (int)M;
@@ -794,7 +906,10 @@ cudaError_t launch_decode_nvfp4(const uint8_t* x_codes, const uint8_t* x_scales,
     p.ctrl = ctrl;
     p.stage_bytes = QW_CODES + p.MT * (QBK / 2) + 2 * Q_SF;
     const int n_tiles = (int)((N + DBM - 1) / DBM);
-    const int smem = choose_shape<1>(p, n_tiles, di);
+    p.part = sw.part;
+    p.tile_ctr = sw.tile_ctr;
+    int smem = (sw.part != nullptr) ? choose_shape_gpart<1>(p, n_tiles, di, sw.part_bytes) : 0;
+    if (smem == 0) smem = choose_shape<1>(p, n_tiles, di);
 
     CUtensorMap tw, tx, tsfw, tsfx;
     if (!make_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, (uint64_t)(K / 2), (uint64_t)N, (uint64_t)(K / 2),
@@ -819,7 +934,7 @@ namespace mq {
 
 cudaError_t launch_decode_nvfp4_fused(const void* x, int64_t M, const float* alpha_static, const uint8_t* w_codes,
                                       const uint8_t* w_scales, const float* alpha_w, int64_t N, int64_t K, void* y,
-                                      WsControl* ctrl, const DeviceInfo& di, cudaStream_t s)
+                                      WsControl* ctrl, const DecodeSplitWs& sw, const DeviceInfo& di, cudaStream_t s)
 {
     FParams p{};
     p.x = static_cast<const uint16_t*>(x);
@@ -846,10 +961,16 @@ cudaError_t launch_decode_nvfp4_fused(const void* x, int64_t M, const float* alp
     // all tokens for its weight rows, so this work is repeated per 128 rows);
     // among them the most weight bytes in flight (saturating at ~16 MB) wins,
     // then the larger grid.
+    //   With a partial workspace, the K split runs over independent CTAs (any
+    // split 1..8, several CTAs per SM; each CTA takes the amax over all of X,
+    // at most 512K elements); otherwise over a cluster (split a power of two).
     constexpr int64_t kSaturateBytes = 16ll << 20;
-    int best_split = 0, best_st = 0, best_smem = 0;
+    int best_split = 0, best_st = 0, best_smem = 0, best_gpart = 0;
     int64_t best_score = -1;
-    for (int sp = 1; sp <= 8 && sp <= p.k_stages; sp *= 2) {
+    const bool can_gpart = sw.part != nullptr && (p.alpha_static != nullptr || M * K <= (int64_t)1 << 19);
+    for (int sp = 1; sp <= 8 && sp <= p.k_stages; ++sp) {
+        const bool gp = can_gpart && (sp == 1 || (size_t)sp * n_tiles * M * DBM * 4 <= sw.part_bytes);
+        if (!gp && (sp & (sp - 1)) != 0) continue;   // a cluster split is a power of two
         const int nks = (p.k_stages + sp - 1) / sp;
         for (int st = std::min(8, nks); st >= std::min(2, nks); --st) {
             const int body = std::max(st * F_RING + nks * p.x_stage, p.MT * DBM * 4);
@@ -863,22 +984,26 @@ cudaError_t launch_decode_nvfp4_fused(const void* x, int64_t M, const float* alp
             smem = (smem + 1023) / 1024 * 1024;
             if ((size_t)smem > di.max_smem_optin) continue;
             const int ctas = n_tiles * sp;
-            const int active = fused_resident_ctas(sp, smem, di);
+            const int active = fused_resident_ctas(gp ? 1 : sp, smem, di);
             if (active <= 0 || ctas > active) continue;
             if (M * (K / sp) > 65536) continue;
-            const int64_t score = std::min<int64_t>(kSaturateBytes, (int64_t)ctas * st * F_RING) * 1024 +
-                                  std::min(ctas, 1023);
+            const int64_t score = std::min<int64_t>(kSaturateBytes, (int64_t)ctas * st * F_RING) * 4096 +
+                                  std::min(ctas, 2 * di.num_sms);
             if (score > best_score) {
                 best_score = score;
                 best_split = sp;
                 best_st = st;
                 best_smem = smem;
+                best_gpart = gp ? 1 : 0;
             }
         }
     }
     if (best_split == 0) return cudaErrorNotSupported;   // the caller takes the two-kernel path
     p.split = best_split;
     p.stages = best_st;
+    p.gpart = best_gpart;
+    p.part = sw.part;
+    p.tile_ctr = sw.tile_ctr;
     const int nks = (p.k_stages + p.split - 1) / p.split;
     p.x_off = p.stages * F_RING;
     const int body = std::max(p.x_off + nks * p.x_stage, p.MT * DBM * 4);
@@ -901,7 +1026,7 @@ cudaError_t launch_decode_nvfp4_fused(const void* x, int64_t M, const float* alp
     cfg.stream = s;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)p.split;
+    attr[0].val.clusterDim.x = p.gpart ? 1u : (unsigned)p.split;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -121,15 +121,25 @@ struct GemmArgs {
 };
 cudaError_t launch_gemm_nvfp4(const GemmArgs& a, const DeviceInfo& di, cudaStream_t s);
 
+// Workspace of the decode kernels' split-K reduction across independent CTAs:
+// per 128-row weight tile a counter (zero when idle) and up to `part_bytes` of
+// FP32 partial tiles.  part == nullptr: the K split uses clusters instead.
+struct DecodeSplitWs {
+    float* part;
+    uint32_t* tile_ctr;
+    size_t part_bytes;
+};
+
 // BF16 decode linear: Y[M,N] = X[M,K] W[N,K]^T, FP32 accumulation.
 cudaError_t launch_decode_bf16(const void* x, int64_t M, const void* w, int64_t N, int64_t K, void* y,
-                               WsControl* ctrl, const DeviceInfo& di, cudaStream_t s);
+                               WsControl* ctrl, const DecodeSplitWs& sw, const DeviceInfo& di, cudaStream_t s);
 
 // Uniform-NVFP4 decode: Y[M,N] = bf16(fl(alpha_w*alpha_x) * sum_k dequant)
 // with X [M <= 128, K] and W [N, K] both NVFP4 (codes, MMA-layout scales).
 cudaError_t launch_decode_nvfp4(const uint8_t* x_codes, const uint8_t* x_scales, const float* alpha_x, int64_t M,
                                 const uint8_t* w_codes, const uint8_t* w_scales, const float* alpha_w, int64_t N,
-                                int64_t K, void* y, WsControl* ctrl, const DeviceInfo& di, cudaStream_t s);
+                                int64_t K, void* y, WsControl* ctrl, const DecodeSplitWs& sw, const DeviceInfo& di,
+                                cudaStream_t s);
 
 // Uniform-NVFP4 decode with the token quantization inside the kernel: X BF16
 // [M <= 128, K] is quantized (Eq. 2 / Eq. 3; dynamic alpha_x unless
@@ -138,7 +148,7 @@ cudaError_t launch_decode_nvfp4(const uint8_t* x_codes, const uint8_t* x_scales,
 // shape fits the token slice in shared memory.
 cudaError_t launch_decode_nvfp4_fused(const void* x, int64_t M, const float* alpha_static, const uint8_t* w_codes,
                                       const uint8_t* w_scales, const float* alpha_w, int64_t N, int64_t K, void* y,
-                                      WsControl* ctrl, const DeviceInfo& di, cudaStream_t s);
+                                      WsControl* ctrl, const DecodeSplitWs& sw, const DeviceInfo& di, cudaStream_t s);
 
 // cuTensorMapEncodeTiled obtained from the driver at run time.
 bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t outer,

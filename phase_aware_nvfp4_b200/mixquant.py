@@ -12,7 +12,7 @@ Names mirror the C ABI: ``quantize_weight``, ``quantize_activation``,
 ``prefill_linear_noalloc``, ``prefill_kv_rope``, ``rmsnorm_quantize``,
 ``decode_linear`` (BF16), ``decode_linear_nvfp4``, ``unswizzle_scales``,
 ``async_status``, ``selftest_e2m1``, ``selftest_timeout``, ``nvfp4_sizes``,
-``workspace_bytes``.
+``workspace_bytes``, ``decode_workspace_bytes``.
 """
 from __future__ import annotations
 
@@ -38,7 +38,8 @@ STATUS_NAMES = {0: "MQ_OK", 1: "MQ_ERR_INVALID_ARG", 2: "MQ_ERR_SHAPE", 3: "MQ_E
 EXPORTS = ("mq_status_string", "mq_version", "mq_nvfp4_sizes", "mq_workspace_bytes", "mq_quantize_weight",
            "mq_quantize_activation", "mq_prefill_linear", "mq_decode_linear", "mq_unswizzle_scales",
            "mq_async_status", "mq_prefill_linear_noalloc", "mq_selftest_e2m1", "mq_selftest_timeout",
-           "mq_decode_linear_nvfp4", "mq_quantize", "mq_rmsnorm_quantize", "mq_prefill_kv_rope")
+           "mq_decode_linear_nvfp4", "mq_quantize", "mq_rmsnorm_quantize", "mq_prefill_kv_rope",
+           "mq_decode_workspace_bytes")
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
@@ -76,6 +77,8 @@ def load(path: str = LIB_PATH):
             lib.mq_nvfp4_sizes.restype = i32
             lib.mq_workspace_bytes.argtypes = [i64, i64]
             lib.mq_workspace_bytes.restype = sz
+            lib.mq_decode_workspace_bytes.argtypes = [i64, i64, i64]
+            lib.mq_decode_workspace_bytes.restype = sz
             lib.mq_quantize_weight.argtypes = [vp, i64, i64, i32, nvp, vp, sz, vp]
             lib.mq_quantize_weight.restype = i32
             lib.mq_quantize_activation.argtypes = [vp, i64, i64, vp, nvp, vp, sz, vp]
@@ -158,6 +161,17 @@ def nvfp4_empty(rows: int, cols: int, device=None) -> NVFP4Tensor:
     return NVFP4Tensor(torch.empty((rows, cols // 2), dtype=torch.uint8, device=device),
                        torch.zeros(sb, dtype=torch.uint8, device=device),
                        torch.zeros(1, dtype=torch.float32, device=device), rows, cols)
+
+
+def decode_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(load().mq_decode_workspace_bytes(M, N, K))
+
+
+def decode_workspace(M: int, N: int, K: int, device=None):
+    """A zero-filled workspace for the decode calls on M tokens and an [N, K] weight."""
+    torch = _torch()
+    device = device or torch.device("cuda", torch.cuda.current_device())
+    return torch.zeros(decode_workspace_bytes(M, N, K), dtype=torch.uint8, device=device)
 
 
 def workspace(M: int = 0, K: int = 0, device=None):
@@ -292,7 +306,7 @@ def decode_linear(X, W, Y=None, ws=None, stream=None):
     M, K = X.shape
     N = W.shape[0]
     Y = Y if Y is not None else torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
-    ws = ws if ws is not None else workspace(device=X.device)
+    ws = ws if ws is not None else decode_workspace(M, N, K, X.device)
     _check(load().mq_decode_linear(_ptr(X), M, _ptr(W), N, K, _ptr(Y), *_ws_args(ws), _stream(stream)),
            "mq_decode_linear")
     return Y
@@ -303,7 +317,7 @@ def decode_linear_nvfp4(X, W: NVFP4Tensor, alpha_static=None, Y=None, ws=None, s
     torch = _torch()
     M = X.shape[0]
     Y = Y if Y is not None else torch.empty((M, W.rows), dtype=torch.bfloat16, device=X.device)
-    ws = ws if ws is not None else workspace(M, W.cols, X.device)
+    ws = ws if ws is not None else decode_workspace(M, W.rows, W.cols, X.device)
     w_c = W.c()
     _check(load().mq_decode_linear_nvfp4(_ptr(X), M, ctypes.byref(w_c), _ptr(alpha_static), _ptr(Y), *_ws_args(ws),
                                          _stream(stream)), "mq_decode_linear_nvfp4")

@@ -58,6 +58,11 @@ def test_sizes(lib):
     assert mqb.workspace_bytes(8192, 4096) >= mqb.WS_CONTROL_BYTES + cb
     with pytest.raises(mqb.MQError):
         mqb.nvfp4_sizes(8, 100)
+    # decode workspace: the NVFP4 token copy, then 8 splits x 96 tiles x M x 128 FP32 partials
+    # (the per-tile counters live in the control block)
+    wq = mqb.workspace_bytes(4, 4096)
+    assert mqb.decode_workspace_bytes(4, 12288, 4096) == -(-wq // 256) * 256 + 8 * 96 * 4 * 128 * 4
+    assert mqb.decode_workspace_bytes(0, 12288, 4096) == mqb.WS_CONTROL_BYTES
 
 
 class _NV(ctypes.Structure):

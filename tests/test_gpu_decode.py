@@ -135,3 +135,33 @@ def test_decode_nvfp4_reports_nonfinite_tokens():
     ax = oracle.tensor_alpha(x)[1]           # NaN excluded, as on the device
     assert ax == oracle.tensor_alpha(xf)[1]
     _nvfp4_decode_check(x[finite], w, to_host_bits(y)[finite], alpha_x=ax)
+
+
+@pytest.mark.parametrize("M,N,K", [(8, 1024, 4096), (8, 12288, 4096), (64, 4096, 2048)])
+def test_decode_cluster_split_with_a_small_workspace(M, N, K):
+    """With only the control block (BF16) or mq_workspace_bytes(M, K) (NVFP4) as workspace, the K
+    split runs over thread-block clusters (partials added through distributed shared memory);
+    the default decode workspace splits K over independent CTAs instead.  Both are within the
+    oracle's tolerance, and each path repeated on its workspace gives the same bits (the
+    split-K sums run in a fixed order; the per-tile counters reset themselves)."""
+    from gpu_helpers import gemm_check
+    x = wl.heavy_tailed_bf16(M, K, 7 * M + N)
+    w = wl.normal_bf16(N, K, 0.02, 11 * N + K)
+    X, Wd = to_dev(x), to_dev(w)
+    Wq = mq.quantize_weight(Wd)
+    small, small_q = mq.workspace(), mq.workspace(M, K)
+    big = mq.decode_workspace(M, N, K)
+    outs = []
+    for ws in (small, big):
+        y1 = to_host_bits(mq.decode_linear(X, Wd, ws=ws))
+        y2 = to_host_bits(mq.decode_linear(X, Wd, ws=ws))
+        assert np.array_equal(y1, y2)
+        decode_check(y1, x, w)
+        outs.append(y1)
+    for ws in (small_q, big):
+        y1 = to_host_bits(mq.decode_linear_nvfp4(X, Wq, ws=ws))
+        y2 = to_host_bits(mq.decode_linear_nvfp4(X, Wq, ws=ws))
+        assert np.array_equal(y1, y2)
+        _nvfp4_decode_check(x, w, y1)
+    for ws in (small, small_q, big):
+        assert mq.async_status(ws) == 0
