@@ -164,8 +164,9 @@ MQ_API mq_status mq_prefill_linear(const void* X_bf16, const mq_nvfp4* X_q, int6
 /* Workspace bytes for mq_decode_linear and mq_decode_linear_nvfp4 on M
  * tokens and an [N, K] weight: what mq_workspace_bytes(M, K) covers (its
  * control block also holds one counter per 128 weight rows, for N up to
- * 253952) and room for the FP32 partial sums of the K dimension split across
- * up to 8 CTAs per 128 weight rows (8 * ceil(N/128) * M * 512 bytes).  With it, the decode splits K across independent CTAs that
+ * 253952) and, for M <= 16, room for the FP32 partial sums of the K
+ * dimension split across up to 8 CTAs per 128 weight rows (8 * ceil(N/128) *
+ * M * 512 bytes).  With it, the decode splits K across independent CTAs that
  * add their partials in a fixed order, so the weight stream covers every SM;
  * a smaller workspace (at least MQ_WS_CONTROL_BYTES, or mq_workspace_bytes(M,
  * K) for the NVFP4 decode) still works, with the K split limited to thread-

@@ -135,9 +135,12 @@ constexpr size_t kDecodeCtrOffset = kWsPartialsOffset + (size_t)kAmaxMaxBlocks *
 constexpr int64_t kDecodeMaxTiles = (int64_t)((kWsControlBytes - kDecodeCtrOffset) / 4u);
 static_assert(kDecodeCtrOffset < kWsControlBytes, "decode counters inside the control block");
 
+constexpr int64_t kDecodeMaxGpartTokens = 16;   // the decode kernels split K this way up to 16 tokens
+
 size_t decode_ws_bytes(int64_t M, int64_t N, int64_t K)
 {
     const int64_t n_tiles = (N + 127) / 128;
+    if (M > kDecodeMaxGpartTokens || n_tiles > kDecodeMaxTiles) return ws_bytes_for(M, K);
     return align_up(ws_bytes_for(M, K), 256) + (size_t)kDecodeMaxSplit * (size_t)n_tiles * (size_t)M * 128u * 4u;
 }
 

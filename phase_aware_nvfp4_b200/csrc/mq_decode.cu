@@ -54,6 +54,9 @@ struct DParams {
     uint32_t* tile_ctr;
 };
 
+constexpr int kDecodeMaxSplit = 8;        // CTAs per 128-row tile in the split-K through the workspace
+constexpr int kDecodeMaxGpartTokens = 16; // tokens up to which that split is used (its reduction is serial per tile)
+
 // Split-K reduction through global memory for one 128-row decode tile, run by
 // the 128 epilogue threads (named barrier 2; `row` = TMEM lane = W row of the
 // tile).  Every CTA of the tile has stored its partial part[tile][rank][m][row]
@@ -71,10 +74,25 @@ __device__ __forceinline__ void gsplit_reduce(float* part, uint32_t* tile_ctr, u
     if (*s_flag == 0u) return;
     __threadfence();
     const int64_t n = (int64_t)tile * DBM + row;
-    for (int m = 0; m < M; ++m) {
-        float acc = 0.0f;
-        for (int q = 0; q < split; ++q) acc += __ldcg(part + (((int64_t)tile * split + q) * M + m) * DBM + row);
-        if (n < N) y[(int64_t)m * N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(acc, out_scale)));
+    const float* base = part + (int64_t)tile * split * M * DBM + row;
+    for (int m0 = 0; m0 < M; m0 += 4) {
+        // the partials of four tokens from all splits in flight at once, then
+        // each token's sum in rank order
+        float v[4][kDecodeMaxSplit];
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+#pragma unroll
+            for (int q = 0; q < kDecodeMaxSplit; ++q)
+                v[t][q] = (m0 + t < M && q < split) ? __ldcg(base + ((int64_t)q * M + m0 + t) * DBM) : 0.0f;
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            float acc = 0.0f;
+#pragma unroll
+            for (int q = 0; q < kDecodeMaxSplit; ++q)
+                if (q < split) acc += v[t][q];
+            if (m0 + t < M && n < N)
+                y[(int64_t)(m0 + t) * N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(acc, out_scale)));
+        }
     }
     if (lead) tile_ctr[tile] = 0u;
 }
@@ -447,11 +465,12 @@ inline int pad_smem_for_tmem(int smem, uint32_t tmem_cols, const DeviceInfo& di)
 template <int FMT>
 int choose_shape_gpart(DParams& p, int n_tiles, const DeviceInfo& di, size_t part_bytes)
 {
+    if (p.M > kDecodeMaxGpartTokens) return 0;
     constexpr int64_t kSaturateBytes = 16ll << 20;
     const int stage_bytes = p.stage_bytes;
     int best_split = 0, best_stages = 0, best_smem = 0;
     int64_t best_score = -1;
-    for (int sp = 1; sp <= 8 && sp <= p.k_stages; ++sp) {
+    for (int sp = 1; sp <= kDecodeMaxSplit && sp <= p.k_stages; ++sp) {
         if (sp > 1 && (size_t)sp * n_tiles * p.M * DBM * 4 > part_bytes) break;
         const int per_cta_stages = (p.k_stages + sp - 1) / sp;
         for (int st = std::min(12, per_cta_stages); st >= std::min(2, per_cta_stages); --st) {
@@ -967,7 +986,8 @@ cudaError_t launch_decode_nvfp4_fused(const void* x, int64_t M, const float* alp
     constexpr int64_t kSaturateBytes = 16ll << 20;
     int best_split = 0, best_st = 0, best_smem = 0, best_gpart = 0;
     int64_t best_score = -1;
-    const bool can_gpart = sw.part != nullptr && (p.alpha_static != nullptr || M * K <= (int64_t)1 << 19);
+    const bool can_gpart = sw.part != nullptr && M <= kDecodeMaxGpartTokens &&
+                           (p.alpha_static != nullptr || M * K <= (int64_t)1 << 19);
     for (int sp = 1; sp <= 8 && sp <= p.k_stages; ++sp) {
         const bool gp = can_gpart && (sp == 1 || (size_t)sp * n_tiles * M * DBM * 4 <= sw.part_bytes);
         if (!gp && (sp & (sp - 1)) != 0) continue;   // a cluster split is a power of two

@@ -92,11 +92,13 @@ def main(argv=None) -> int:
     elif a.op == "decode":
         W = dev_bf16(wl.normal_bf16(a.N, a.K, 0.02, 12))
         Y = torch.empty((a.M, a.N), dtype=torch.bfloat16, device=dev)
-        run = lambda: mq.decode_linear(X, W, Y=Y, ws=ws)
+        wsd = mq.decode_workspace(a.M, a.N, a.K, device=dev)
+        run = lambda: mq.decode_linear(X, W, Y=Y, ws=wsd)
     else:
         Wq = mq.quantize_weight(dev_bf16(wl.normal_bf16(a.N, a.K, 0.02, 12)), ws=ws)
         Y = torch.empty((a.M, a.N), dtype=torch.bfloat16, device=dev)
-        run = lambda: mq.decode_linear_nvfp4(X, Wq, Y=Y, ws=ws)
+        wsd = mq.decode_workspace(a.M, a.N, a.K, device=dev)
+        run = lambda: mq.decode_linear_nvfp4(X, Wq, Y=Y, ws=wsd)
     for _ in range(a.warmup):
         run()
     torch.cuda.synchronize()
