@@ -1010,7 +1010,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_NUM_THREADS, 1)
                     }
                 }
             }
-            if (EPI == 2 && 2 * n_blk + half < p.n_heads) kv_stage_cos_sin(p, stg, lane, kv_pos, 0);
+            if (EPI == 2 && 2 * n_blk + half < p.n_heads) {
+                // this token's cos/sin row (512 B) into L2 for the later chunks,
+                // and the first chunk of all 32 rows staged now
+                if (kv_valid) bulk_prefetch_l2(p.cos_sin + (int64_t)kv_pos * 128, 512);
+                kv_stage_cos_sin(p, stg, lane, kv_pos, 0);
+            }
             if (!warp_wait(acc_full, acc_phase, abort_flag)) {
                 if (lane == 0) {
                     post_error(p.ctrl, kErrTimeout);
@@ -1040,6 +1045,286 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_NUM_THREADS, 1)
     tc_fence_before();
     __syncthreads();
     cluster_barrier();   // no CTA leaves while its peer may still read its smem or TMEM
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    }
+}
+
+// ==========================================================================
+// Wide CTA-pair kernel (BF16 epilogue): 256 x 384 output tile per pair
+// ==========================================================================
+//
+// The same pipeline with a 384-column tile: per k-block two pair MMAs share
+// the A operand, one over tile columns 0..255 (N = 256: B rows 0..127 from
+// the leader, 128..255 from its peer) and one over columns 256..383 (N = 128:
+// rows 256..319 from the leader, 320..383 from its peer).  Per SM and k-block
+// that is 128 rows of A and 192 rows of B for 128 x 384 products, against 128
+// and 128 for 128 x 256 in the square tile: a sixth fewer operand bytes per
+// FLOP, and with a quarter fewer tile changes the accumulator hand-over to the
+// epilogue is paid less often.  TMEM: accumulator columns 0..383, scale
+// factors from 384 (A: 4 columns per k-block, B: 12).  Shared memory: four
+// 48 KiB stages.  A tile narrower than 384 (the last one, when N % 384 == 256)
+// issues only the N = 256 MMA.
+constexpr int W_STAGES = 4;
+constexpr int W_B0 = 128 * BK_BYTES;                 // B rows for the N = 256 MMA
+constexpr int W_B1 = 64 * BK_BYTES;                  // B rows for the N = 128 MMA
+constexpr int W_B_STAGE = W_B0 + W_B1;               // 24 KiB
+constexpr int W_SFB_STAGE = 3 * 2048;                // three 128-row blocks x 4 atoms
+constexpr int W_STAGE_BYTES = A_STAGE + W_B_STAGE + SFA_STAGE + W_SFB_STAGE;
+constexpr int W_OFF_A = 0;
+constexpr int W_OFF_B = W_OFF_A + W_STAGES * A_STAGE;
+constexpr int W_OFF_SFA = W_OFF_B + W_STAGES * W_B_STAGE;
+constexpr int W_OFF_SFB = W_OFF_SFA + W_STAGES * SFA_STAGE;
+constexpr int W_OFF_STG = W_OFF_SFB + W_STAGES * W_SFB_STAGE;
+constexpr int W_OFF_BAR = W_OFF_STG + 8 * P_STG_BYTES;
+constexpr int W_SMEM_BYTES = W_OFF_BAR + 256 + 1024;
+constexpr int WN = 384;
+constexpr uint32_t W_TMEM_SF = 384;
+constexpr uint32_t W_IDESC0 = idesc_nvfp4(2 * BM, 256);
+constexpr uint32_t W_IDESC1 = idesc_nvfp4(2 * BM, 128);
+static_assert(W_SMEM_BYTES <= 232448, "wide pair kernel shared memory");
+
+// Epilogue of the wide kernel: warp (lane group lg, half) drains accumulator
+// columns [192 half, 192 half + ncols) (ncols is 192, or 64 for the second
+// half of a 256-wide tile), releases the accumulator, and stores 64-column
+// BF16 subtiles through its staging buffer.
+template <class Barrier>
+__device__ __forceinline__ void epilogue_wide_bf16(const EpiScales& es, uint32_t t_col, int ncols, int lane,
+                                                   uint8_t* stg, const CUtensorMap* tmap_y, int32_t x0, int32_t y0,
+                                                   Barrier arrive)
+{
+    // one 32-column load at a time, packed to BF16 at once: the packed row
+    // (96 registers) and one raw chunk stay within the register budget
+    uint32_t out[96];
+#pragma unroll
+    for (int c = 0; c < 6; ++c) {
+        if (32 * c < ncols) {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(t_col + 32 * c, r);
+            tmem_wait_ld(r);
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                out[16 * c + j] = pack_bf16x2(__fmul_rn(__uint_as_float(r[2 * j]), es.alpha_ab),
+                                              __fmul_rn(__uint_as_float(r[2 * j + 1]), es.alpha_ab));
+        }
+    }
+    release_acc_warp(lane, arrive);
+#pragma unroll
+    for (int q = 0; q < 3; ++q) {
+        if (64 * q >= ncols) break;
+        if (lane == 0) bulk_wait_group_read<0>();
+        __syncwarp();
+        uint8_t* rowp = stg + lane * 128;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int w = 32 * q + 4 * j;
+            *reinterpret_cast<uint4*>(rowp + ((j ^ (lane & 7)) << 4)) =
+                make_uint4(out[w], out[w + 1], out[w + 2], out[w + 3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_2d(tmap_y, stg, x0 + 64 * q, y0);
+            bulk_commit_group();
+        }
+    }
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_NUM_THREADS, 1)
+    gemm_nvfp4_wide_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                           const __grid_constant__ CUtensorMap tmap_b64, const __grid_constant__ CUtensorMap tmap_sfa,
+                           const __grid_constant__ CUtensorMap tmap_sfb3, const __grid_constant__ CUtensorMap tmap_y,
+                           const Params p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + W_OFF_BAR);
+    uint64_t* empty_bar = full_bar + W_STAGES;
+    uint64_t* acc_full = empty_bar + W_STAGES;
+    uint64_t* acc_empty = acc_full + 1;
+    uint64_t* mma_done = acc_empty + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+    volatile uint32_t* abort_flag = tmem_slot + 1;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int pair = blockIdx.x >> 1;
+    const int npairs = gridDim.x >> 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < W_STAGES; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], 1);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, 2 * P_EPI_WARPS);
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        fence_mbarrier_init();
+        prefetch_tensormap(&tmap_a);
+        prefetch_tensormap(&tmap_b);
+        prefetch_tensormap(&tmap_b64);
+        prefetch_tensormap(&tmap_sfa);
+        prefetch_tensormap(&tmap_sfb3);
+        prefetch_tensormap(&tmap_y);
+    }
+    if (warp == 1) tmem_alloc_pair(tmem_slot, TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    cluster_barrier();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    grid_dep_wait();
+    grid_dep_launch_dependents();
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer (both CTAs)
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        const uint32_t full0 = map_to_cta(smem_u32(&full_bar[0]), 0);
+        for (int tile = pair; tile < p.num_tiles && ok; tile += npairs) {
+            int m_blk, n_blk;
+            tile_coords(p, tile, m_blk, n_blk);
+            const int a_row = m_blk * 2 * BM + (int)rank * BM;
+            const int n0 = n_blk * WN;
+            const int sfa_row = (m_blk * 2 + (int)rank) * p.sfa_atoms;
+            for (int ks = 0; ks < p.k_stages; ++ks) {
+                if (!warp_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                if (elect_one()) {
+                    if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2u * W_STAGE_BYTES);
+                    const uint32_t bar = full0 + 8u * (uint32_t)stage;
+                    uint8_t* sb = smem + W_OFF_B + stage * W_B_STAGE;
+                    tma_load_2d_pair(smem + W_OFF_A + stage * A_STAGE, &tmap_a, bar, ks * BK_BYTES, a_row);
+                    tma_load_2d_pair(sb, &tmap_b, bar, ks * BK_BYTES, n0 + (int)rank * 128);
+                    tma_load_2d_pair(sb + W_B0, &tmap_b64, bar, ks * BK_BYTES, n0 + 256 + (int)rank * 64);
+                    tma_load_2d_pair(smem + W_OFF_SFA + stage * SFA_STAGE, &tmap_sfa, bar, 0, sfa_row + ks * 4);
+                    tma_load_3d_pair(smem + W_OFF_SFB + stage * W_SFB_STAGE, &tmap_sfb3, bar, 0, ks * 4, 3 * n_blk);
+                }
+                __syncwarp();
+                if (++stage == W_STAGES) stage = 0, phase ^= 1u;
+            }
+        }
+        if (!ok && lane == 0) {
+            post_error(p.ctrl, kErrTimeout);
+            *abort_flag = 1;
+        }
+        if (ok) {
+            for (int s = 0; s < W_STAGES; ++s) {
+                (void)mbar_wait(&empty_bar[stage], phase ^ 1u);
+                if (++stage == W_STAGES) stage = 0, phase ^= 1u;
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer (leader CTA)
+        if (leader) {
+            const uint64_t a_desc0 = sdesc_kmajor_sw128(smem_u32(smem + W_OFF_A));
+            const uint64_t b_desc0 = sdesc_kmajor_sw128(smem_u32(smem + W_OFF_B));
+            const uint64_t sfa_desc0 = sdesc_sf_block(smem_u32(smem + W_OFF_SFA));
+            const uint64_t sfb_desc0 = sdesc_sf_block(smem_u32(smem + W_OFF_SFB));
+            const uint32_t sfa_tmem = tmem_base + W_TMEM_SF;
+            const uint32_t sfb_tmem = sfa_tmem + 16;
+            int stage = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            bool ok = true, next_ready = false;
+            for (int tile = pair; tile < p.num_tiles && ok; tile += npairs) {
+                int m_blk, n_blk;
+                tile_coords(p, tile, m_blk, n_blk);
+                const bool wide = p.N - n_blk * WN > 256;   // else only the N = 256 MMA
+                if (!warp_wait(acc_empty, acc_phase ^ 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                for (int ks = 0; ks < p.k_stages; ++ks) {
+                    if (!next_ready && !warp_wait(&full_bar[stage], phase, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    {
+                        const int ns = (stage + 1 == W_STAGES) ? 0 : stage + 1;
+                        next_ready = warp_test(&full_bar[ns], ns == 0 ? (phase ^ 1u) : phase);
+                    }
+                    const uint64_t a_d = a_desc0 + (uint64_t)((stage * A_STAGE) >> 4);
+                    const uint64_t b0_d = b_desc0 + (uint64_t)((stage * W_B_STAGE) >> 4);
+                    const uint64_t b1_d = b0_d + (uint64_t)(W_B0 >> 4);
+                    const uint64_t sfa_d = sfa_desc0 + (uint64_t)((stage * SFA_STAGE) >> 4);
+                    const uint64_t sfb_d = sfb_desc0 + (uint64_t)((stage * W_SFB_STAGE) >> 4);
+                    if (elect_one()) {
+#pragma unroll
+                        for (int kb = 0; kb < 4; ++kb) {
+                            const uint32_t acc = (ks | kb) != 0 ? 1u : 0u;
+                            tmem_cp_32x128b_x4_pair(sfa_tmem + 4 * kb, sfa_d + (uint64_t)((kb * 512) >> 4));
+                            tmem_cp_32x128b_x4_pair(sfb_tmem + 12 * kb, sfb_d + (uint64_t)((kb * 512) >> 4));
+                            tmem_cp_32x128b_x4_pair(sfb_tmem + 12 * kb + 4, sfb_d + (uint64_t)((2048 + kb * 512) >> 4));
+                            if (wide)
+                                tmem_cp_32x128b_x4_pair(sfb_tmem + 12 * kb + 8,
+                                                        sfb_d + (uint64_t)((4096 + kb * 512) >> 4));
+                            umma_nvfp4_pair(tmem_base, a_d + (uint64_t)((kb * 32) >> 4), b0_d + (uint64_t)((kb * 32) >> 4),
+                                            W_IDESC0, sfa_tmem + 4 * kb, sfb_tmem + 12 * kb, acc);
+                            if (wide)
+                                umma_nvfp4_pair(tmem_base + 256, a_d + (uint64_t)((kb * 32) >> 4),
+                                                b1_d + (uint64_t)((kb * 32) >> 4), W_IDESC1, sfa_tmem + 4 * kb,
+                                                sfb_tmem + 12 * kb + 8, acc);
+                        }
+                        tc_commit_pair_mc(&empty_bar[stage], 0x3);
+                    }
+                    __syncwarp();
+                    if (++stage == W_STAGES) stage = 0, phase ^= 1u;
+                }
+                if (!ok) break;
+                if (elect_one()) tc_commit_pair_mc(acc_full, 0x3);
+                __syncwarp();
+                acc_phase ^= 1u;
+            }
+            if (!ok && lane == 0) {
+                post_error(p.ctrl, kErrTimeout);
+                *abort_flag = 1;
+            }
+            if (elect_one()) tc_commit_pair(mma_done);
+            __syncwarp();
+            (void)mbar_wait(mma_done, 0);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue (both CTAs)
+        const int lg = warp & 3;
+        const int half = (warp - 2) >> 2;
+        EpiScales es = epi_scales<0>(p);
+        const uint32_t leader_acc_empty = map_to_cta(smem_u32(acc_empty), 0);
+        const uint32_t t_col = tmem_base + ((uint32_t)(32 * lg) << 16) + (uint32_t)(192 * half);
+        uint8_t* stg = smem + W_OFF_STG + (warp - 2) * P_STG_BYTES;
+        auto arrive = [&] { mbar_arrive_cluster(leader_acc_empty); };
+        uint32_t acc_phase = 0;
+        for (int tile = pair; tile < p.num_tiles; tile += npairs) {
+            int m_blk, n_blk;
+            tile_coords(p, tile, m_blk, n_blk);
+            if (!warp_wait(acc_full, acc_phase, abort_flag)) {
+                if (lane == 0) {
+                    post_error(p.ctrl, kErrTimeout);
+                    *abort_flag = 1;
+                }
+                break;
+            }
+            acc_phase ^= 1u;
+            tc_fence_after();
+            const int64_t row0 = (int64_t)m_blk * 2 * BM + (int64_t)rank * BM + 32 * lg;
+            const int width = min(WN, p.N - n_blk * WN);          // 384, or 256 for a last narrower tile
+            const int ncols = min(192, width - 192 * half);       // 192 or 64
+            epilogue_wide_bf16(es, t_col, ncols, lane, stg, &tmap_y, n_blk * WN + 192 * half, (int32_t)row0, arrive);
+        }
+        if (lane == 0) bulk_wait_group<0>();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_barrier();
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc_pair(tmem_base, TMEM_COLS);
@@ -1131,9 +1416,27 @@ cudaError_t launch_gemm_nvfp4(const GemmArgs& a, const DeviceInfo& di, cudaStrea
                 return cudaErrorInvalidValue;
         }
         p.num_m_blk = (int)((a.M + 2 * BM - 1) / (2 * BM));
+        p.n_fastest = a.M > a.N;   // A (M rows) is the larger operand: sweep N fastest
+        if (a.epilogue == 0 && a.N >= 3072 && (a.N % WN == 0 || a.N % WN == 256)) {
+            // 256 x 384 tiles (the last one 256 wide when N % 384 == 256)
+            CUtensorMap tb64, tsfb3;
+            if (!make_tmap_2d(&tb64, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.b_codes, (uint64_t)(a.K / 2), (uint64_t)a.N,
+                              (uint64_t)(a.K / 2), BK_BYTES, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+                return cudaErrorInvalidValue;
+            if (!make_tmap_3d(&tsfb3, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.b_scales, 128, (uint64_t)p.sfb_atoms,
+                              (uint64_t)p.sfb_rowblks, 512, (uint64_t)p.sfb_atoms * 512, 128, 4, 3))
+                return cudaErrorInvalidValue;
+            p.num_n_blk = (int)((a.N + WN - 1) / WN);
+            p.num_tiles = p.num_m_blk * p.num_n_blk;
+            const int pairs = std::min(p.num_tiles, di.num_sms / 2);
+            cudaError_t e = cudaFuncSetAttribute(gemm_nvfp4_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 W_SMEM_BYTES);
+            if (e != cudaSuccess) return e;
+            return launch_pdl(gemm_nvfp4_wide_kernel, dim3(2 * pairs), dim3(P_NUM_THREADS), W_SMEM_BYTES, s, ta, tb,
+                              tb64, tsfa, tsfb3, ty, p);
+        }
         p.num_n_blk = num_n_blk;
         p.num_tiles = p.num_m_blk * num_n_blk;
-        p.n_fastest = a.M > a.N;   // A (M rows) is the larger operand: sweep N fastest
         const int pairs = std::min(p.num_tiles, di.num_sms / 2);
         switch (a.epilogue) {
             case 0: return launch_pair<0>(pairs, ta, tb, tsfa, tsfb, ty, p, s);

@@ -109,8 +109,12 @@ def main(argv=None) -> int:
     e1.record()
     torch.cuda.synchronize()
     st = mq.async_status(ws)
+    if st == 0 and a.op in ("decode", "decode_nvfp4"):
+        st = mq.async_status(wsd)
     ms = e0.elapsed_time(e1) / max(1, a.iters)
-    print(f"{a.op} M={a.M} N={a.N} K={a.K}: {ms * 1e3:.1f} us per call (status {mq.STATUS_NAMES.get(st, st)})")
+    flops = 2.0 * a.M * a.N * a.K if a.op in ("gemm", "mlp", "kv_rope", "decode", "decode_nvfp4") else 0.0
+    rate = f", {flops / (ms * 1e-3) / 1e12:.0f} TFLOP/s" if flops else ""
+    print(f"{a.op} M={a.M} N={a.N} K={a.K}: {ms * 1e3:.1f} us per call{rate} (status {mq.STATUS_NAMES.get(st, st)})")
     return 0 if st == 0 else 1
 
 
