@@ -353,11 +353,27 @@ def _time_rotating(torch, calls, reps):
     return float(np.mean([a.elapsed_time(b) for a, b in evs]))
 
 
+def _time_stream(torch, calls, reps):
+    """Mean device time (ms) per call of `reps` calls issued back to back,
+    cycling through `calls` as _time_rotating does: the decode of a layer stack,
+    where each call's launch overlaps the previous call's tail."""
+    torch.cuda._sleep(2_000_000)   # the GPU busy while the host enqueues the calls
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for i in range(reps):
+        calls[i % len(calls)]()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps
+
+
 def _decode_pair(mq, torch, dev, wl, Wm, Wq, hbm_gbs, reps, seed):
     """BF16 decode and uniform-NVFP4 decode (tokens quantized on the fly) on one
     weight [N, K] and its NVFP4 copy at M = 1, 8, 32, 64 tokens, timed on
-    rotating weight copies larger than L2 (weights cold, code warm).  HBM
-    roofline bytes: 2NK + 2MK + 2MN (BF16) and 0.5625NK + 2MK + 2MN (NVFP4)."""
+    rotating weight copies larger than L2 (weights cold, code warm): `ms` per
+    isolated call (a spin kernel before each, so every call pays its launch
+    and ramp), `ms_stream` per call of a back-to-back sequence.  HBM roofline
+    bytes: 2NK + 2MK + 2MN (BF16) and 0.5625NK + 2MK + 2MN (NVFP4)."""
     N, K = Wm.shape
     n_bf = max(2, -(-(400 << 20) // (2 * N * K)))          # copies: together > 3 x L2
     n_q = max(2, -(-(400 << 20) // (N * K // 2)))
@@ -377,11 +393,18 @@ def _decode_pair(mq, torch, dev, wl, Wm, Wq, hbm_gbs, reps, seed):
         # so the timed calls do not start on a clock that is still ramping up
         torch.cuda._sleep(100_000_000)
         ms = _time_rotating(torch, bf, 4 * reps)
-        gbs = (2 * N * K + 2 * M * K + 2 * M * N) / (ms * 1e-3) / 1e9
-        dec[str(M)] = {"ms": ms, "GB/s": gbs, "frac": gbs / hbm_gbs}
+        ms_s = _time_stream(torch, bf, 4 * reps)
+        by = 2 * N * K + 2 * M * K + 2 * M * N
+        gbs = by / (ms * 1e-3) / 1e9
+        dec[str(M)] = {"ms": ms, "GB/s": gbs, "frac": gbs / hbm_gbs,
+                       "ms_stream": ms_s, "frac_stream": by / (ms_s * 1e-3) / 1e9 / hbm_gbs}
         msq = _time_rotating(torch, q4, 4 * reps)
-        gbs = (0.5625 * N * K + 2 * M * K + 2 * M * N) / (msq * 1e-3) / 1e9
-        decq[str(M)] = {"ms": msq, "GB/s": gbs, "frac": gbs / hbm_gbs, "speedup_vs_bf16": ms / msq}
+        msq_s = _time_stream(torch, q4, 4 * reps)
+        byq = 0.5625 * N * K + 2 * M * K + 2 * M * N
+        gbs = byq / (msq * 1e-3) / 1e9
+        decq[str(M)] = {"ms": msq, "GB/s": gbs, "frac": gbs / hbm_gbs, "speedup_vs_bf16": ms / msq,
+                        "ms_stream": msq_s, "frac_stream": byq / (msq_s * 1e-3) / 1e9 / hbm_gbs,
+                        "speedup_vs_bf16_stream": ms_s / msq_s}
     del Wm_copies, Wq_copies
     return dec, decq
 
@@ -483,7 +506,8 @@ def measure_extras(mq, torch, dev, flush, hbm_gbs, fp4_peak, reps=10):
     out["phase_aware_pair"] = {
         "weight": [N, K], "decode_bf16": dec,
         "roofline_decode": {"bound": "hbm", "kernel": "decode_bf16_kernel", "unit": "GB/s", "peak": hbm_gbs,
-                            "achieved": dec["64"]["GB/s"], "frac": dec["64"]["frac"], "M": 64},
+                            "achieved": dec["64"]["GB/s"], "frac": dec["64"]["frac"], "M": 64,
+                            "frac_stream": dec["64"]["frac_stream"]},
         "decode_nvfp4": decq,
         "transposed_weight": [K, N], "decode_bf16_k12288": dec_t, "decode_nvfp4_k12288": decq_t,
         "prefill_nvfp4": {"M": Mp, "ms": ms, "TFLOP/s": 2 * Mp * N * K / (ms * 1e-3) / 1e12},

@@ -21,9 +21,9 @@ namespace mq {
 namespace {
 
 constexpr int DBM = 128;                 // W rows per tile (UMMA M)
-constexpr int DBK = 64;                  // K elements per stage (128 bytes of BF16)
+constexpr int DBK = 64;                  // K elements per TMA box (128 bytes of BF16)
 constexpr int D_THREADS = 192;
-constexpr int W_STAGE = DBM * DBK * 2;   // 16 KiB
+constexpr int W_STAGE = DBM * DBK * 2;   // 16 KiB per box
 
 // NVFP4 weights (FMT 1): 256 K-elements per stage = 128 bytes of codes per
 // row, plus four 512-byte scale atoms for the 128 W rows and four for the
@@ -35,6 +35,8 @@ constexpr int Q_SF = 4 * 512;             // 2 KiB
 struct DParams {
     int M, N, K, MT;
     int k_stages;       // total K stages
+    int kbox;           // FMT 0: TMA boxes of DBK elements per stage (one wait, commit and
+                        // hand-over per stage: larger stages issue fewer of them per byte)
     int split;          // cluster size along K
     int stages;         // pipeline depth
     int stage_bytes;
@@ -133,8 +135,9 @@ __global__ void __launch_bounds__(D_THREADS, 1)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    constexpr int W_TILE = FMT ? QW_CODES : W_STAGE;
-    const int x_tile = FMT ? p.MT * (QBK / 2) : p.MT * DBK * 2;
+    const int W_TILE = FMT ? QW_CODES : W_STAGE * p.kbox;
+    const int x_box = p.MT * DBK * 2;   // FMT 0: bytes of one token box
+    const int x_tile = FMT ? p.MT * (QBK / 2) : x_box * p.kbox;
     const int stage_bytes = p.stage_bytes;
     uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + p.bar_offset);
     uint64_t* empty_bar = full_bar + p.stages;
@@ -234,8 +237,11 @@ __global__ void __launch_bounds__(D_THREADS, 1)
                     tma_load_2d(sw + W_TILE + x_tile, &tmap_sfw, &full_bar[stage], 0, n_tile * p.sfw_atoms + ks * 4);
                     tma_load_2d(sw + W_TILE + x_tile + Q_SF, &tmap_sfx, &full_bar[stage], 0, ks * 4);
                 } else {
-                    tma_load_2d(sw, &tmap_w, &full_bar[stage], ks * DBK, n_tile * DBM);
-                    tma_load_2d(sw + W_TILE, &tmap_x, &full_bar[stage], ks * DBK, 0);
+                    for (int b = 0; b < p.kbox; ++b) {
+                        const int kx = (ks * p.kbox + b) * DBK;   // boxes past K read zeros
+                        tma_load_2d(sw + b * W_STAGE, &tmap_w, &full_bar[stage], kx, n_tile * DBM);
+                        tma_load_2d(sw + W_TILE + b * x_box, &tmap_x, &full_bar[stage], kx, 0);
+                    }
                 }
             }
             __syncwarp();
@@ -275,17 +281,23 @@ __global__ void __launch_bounds__(D_THREADS, 1)
             const uint64_t x_d = w_d + (uint64_t)(W_TILE >> 4);
             const uint64_t sf_d = sf_desc0 + (uint64_t)((stage * stage_bytes) >> 4);
             if (elect_one()) {
+                if (FMT) {
 #pragma unroll
-                for (int kb = 0; kb < 4; ++kb) {
-                    const uint32_t acc = (ks > ks_begin || kb > 0) ? 1u : 0u;
-                    if (FMT) {
+                    for (int kb = 0; kb < 4; ++kb) {
+                        const uint32_t acc = (ks > ks_begin || kb > 0) ? 1u : 0u;
                         tmem_cp_32x128b_x4(sfa_tmem + 4 * kb, sf_d + (uint64_t)((kb * 512) >> 4));
                         tmem_cp_32x128b_x4(sfb_tmem + 4 * kb, sf_d + (uint64_t)((Q_SF + kb * 512) >> 4));
                         umma_nvfp4(tmem_base, w_d + (uint64_t)((32 * kb) >> 4), x_d + (uint64_t)((32 * kb) >> 4), idesc,
                                    sfa_tmem + 4 * kb, sfb_tmem + 4 * kb, acc);
-                    } else {
-                        umma_bf16(tmem_base, w_d + (uint64_t)((32 * kb) >> 4), x_d + (uint64_t)((32 * kb) >> 4), idesc,
-                                  acc);
+                    }
+                } else {
+                    for (int b = 0; b < p.kbox; ++b) {
+                        const uint64_t wb = w_d + (uint64_t)((b * W_STAGE) >> 4);
+                        const uint64_t xb = x_d + (uint64_t)((b * x_box) >> 4);
+#pragma unroll
+                        for (int kb = 0; kb < 4; ++kb)
+                            umma_bf16(tmem_base, wb + (uint64_t)((32 * kb) >> 4), xb + (uint64_t)((32 * kb) >> 4),
+                                      idesc, (ks > ks_begin || b > 0 || kb > 0) ? 1u : 0u);
                     }
                 }
                 tc_commit(&empty_bar[stage]);
@@ -879,12 +891,14 @@ cudaError_t launch_decode_bf16(const void* x, int64_t M, const void* w, int64_t 
     p.N = (int)N;
     p.K = (int)K;
     p.MT = (int)((M + 15) / 16 * 16);
-    p.k_stages = (int)((K + DBK - 1) / DBK);
+    // two boxes (128 K elements) per stage once K has a few stages of them
+    p.kbox = (K >= 8 * 2 * DBK) ? 2 : 1;
+    p.k_stages = (int)((K + DBK * p.kbox - 1) / (DBK * p.kbox));
     p.tmem_cols = 32;
     while ((int)p.tmem_cols < p.MT) p.tmem_cols <<= 1;
     p.y = static_cast<uint16_t*>(y);
     p.ctrl = ctrl;
-    p.stage_bytes = W_STAGE + p.MT * DBK * 2;
+    p.stage_bytes = (W_STAGE + p.MT * DBK * 2) * p.kbox;
     const int n_tiles = (int)((N + DBM - 1) / DBM);
     p.part = sw.part;
     p.tile_ctr = sw.tile_ctr;
@@ -912,6 +926,7 @@ cudaError_t launch_decode_nvfp4(const uint8_t* x_codes, const uint8_t* x_scales,
     p.K = (int)K;
     p.MT = (int)((M + 31) / 32 * 32);   // MMA N: a multiple of 32, at most 128
     p.k_stages = (int)((K + QBK - 1) / QBK);
+    p.kbox = 1;
     uint32_t acc_cols = 32;
     while ((int)acc_cols < p.MT) acc_cols <<= 1;
     p.tmem_sf = acc_cols;                // A scales at +0..15, B scales at +16..31
