@@ -991,7 +991,7 @@ cudaError_t launch_decode_nvfp4_fused(const void* x, int64_t M, const float* alp
 
     // Launch shape: K split (cluster size) and ring depth.  Candidates must fit
     // the token slice and the ring in shared memory, run in one wave and leave
-    // each CTA at most 64K token elements to quantize (every cluster quantizes
+    // each CTA at most 32K token elements to quantize (every cluster quantizes
     // all tokens for its weight rows, so this work is repeated per 128 rows);
     // among them the most weight bytes in flight (saturating at ~16 MB) wins,
     // then the larger grid.
@@ -1021,7 +1021,7 @@ cudaError_t launch_decode_nvfp4_fused(const void* x, int64_t M, const float* alp
             const int ctas = n_tiles * sp;
             const int active = fused_resident_ctas(gp ? 1 : sp, smem, di);
             if (active <= 0 || ctas > active) continue;
-            if (M * (K / sp) > 65536) continue;
+            if (M * (K / sp) > 32768) continue;
             const int64_t score = std::min<int64_t>(kSaturateBytes, (int64_t)ctas * st * F_RING) * 4096 +
                                   std::min(ctas, 2 * di.num_sms);
             if (score > best_score) {

@@ -63,7 +63,8 @@ def _nvfp4_decode_check(x, w, y_gpu_bits, alpha_x=None):
 
 @pytest.mark.parametrize("M,N,K", [(1, 256, 256), (7, 400, 1088), (32, 512, 1024), (64, 768, 2048),
                                    (100, 272, 320), (128, 128, 4096), (1, 4096, 12288), (1, 12288, 4096),
-                                   (8, 12288, 4096), (64, 12288, 4096), (128, 4096, 12288)])
+                                   (8, 12288, 4096), (16, 12288, 4096), (16, 4096, 12288), (64, 12288, 4096),
+                                   (128, 4096, 12288)])
 def test_decode_nvfp4_vs_oracle(M, N, K):
     """Ragged tokens (MMA N padded to 32), ragged weight rows (N % 128 != 0) and a partial last
     256-element stage (K % 256 != 0) are all covered, as are the launch shapes the call picks:
