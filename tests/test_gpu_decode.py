@@ -64,13 +64,15 @@ def _nvfp4_decode_check(x, w, y_gpu_bits, alpha_x=None):
 @pytest.mark.parametrize("M,N,K", [(1, 256, 256), (7, 400, 1088), (32, 512, 1024), (64, 768, 2048),
                                    (100, 272, 320), (128, 128, 4096), (1, 4096, 12288), (1, 12288, 4096),
                                    (8, 12288, 4096), (16, 12288, 4096), (16, 4096, 12288), (64, 12288, 4096),
-                                   (128, 4096, 12288)])
+                                   (128, 4096, 12288), (2, 400, 1024), (3, 1024, 2048), (4, 12288, 4096),
+                                   (2, 4096, 12288), (1, 272, 8192)])
 def test_decode_nvfp4_vs_oracle(M, N, K):
     """Ragged tokens (MMA N padded to 32), ragged weight rows (N % 128 != 0) and a partial last
     256-element stage (K % 256 != 0) are all covered, as are the launch shapes the call picks:
     the single kernel that quantizes the tokens itself (K split over clusters of 1 to 8 CTAs
-    exchanging their slice maxima) and, where the token slice does not fit in shared memory
-    (128 tokens, K = 12288), the quantization kernel followed by the decode GEMM."""
+    exchanging their slice maxima, or over independent CTAs adding partials through the
+    workspace) and, above 32K token elements per CTA or where the token slice does not fit in
+    shared memory, the quantization kernel followed by the decode GEMM."""
     x = wl.heavy_tailed_bf16(M, K, 3 * M + K)
     w = wl.normal_bf16(N, K, 0.02, 5 * N + K)
     Wq = mq.quantize_weight(to_dev(w))
@@ -80,14 +82,16 @@ def test_decode_nvfp4_vs_oracle(M, N, K):
     print(f"nvfp4 decode M={M} N={N} K={K}: rel-Frobenius {rel:.2e}")
 
 
-def test_decode_nvfp4_static_alpha_and_grid_inputs_exact():
+@pytest.mark.parametrize("M,K", [(16, 512), (3, 2048)])
+def test_decode_nvfp4_static_alpha_and_grid_inputs_exact(M, K):
     """Grid-valued inputs whose blocks all hold a 6: X with a static alpha of 1 and W with a 2688
     anchor alone in its block (alpha_w = 1) get block scales of exactly 1 (448 for the anchor), so
-    Y = bf16(X W^T) exactly (the FP32 sums stay below 2^24 quarter units)."""
+    Y = bf16(X W^T) exactly (the FP32 sums stay below 2^24 quarter units), on the quantization
+    kernel + decode GEMM (16 tokens) and on the single kernel (3 tokens)."""
     rng = np.random.default_rng(3)
     grid = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6], np.float32)
-    xi = (rng.choice(grid, size=(16, 512)) * rng.choice([-1, 1], size=(16, 512))).astype(np.float32)
-    wi = (rng.choice(grid, size=(256, 512)) * rng.choice([-1, 1], size=(256, 512))).astype(np.float32)
+    xi = (rng.choice(grid, size=(M, K)) * rng.choice([-1, 1], size=(M, K))).astype(np.float32)
+    wi = (rng.choice(grid, size=(256, K)) * rng.choice([-1, 1], size=(256, K))).astype(np.float32)
     xi[:, ::16] = 6.0
     wi[:, ::16] = 6.0
     wi[0, :16] = 0.0
@@ -98,6 +102,25 @@ def test_decode_nvfp4_static_alpha_and_grid_inputs_exact():
     torch.cuda.synchronize()
     exact = xi.astype(np.float64) @ wi.T.astype(np.float64)
     assert np.array_equal(to_host_bits(y), oracle.round_bf16(exact))
+
+
+@pytest.mark.parametrize("M,N,K", [(4, 12288, 4096), (1, 4096, 12288)])
+def test_decode_nvfp4_repeatable_and_static_alpha(M, N, K):
+    """The single-kernel decode gives the same bits on a repeated call (split-K partials added in
+    rank order), and with a static alpha_x equal to the tokens' own amax / 2688 it gives the same
+    bits as with the dynamic one (every CTA derives the same alpha_x)."""
+    x = wl.heavy_tailed_bf16(M, K, 5 * M + N)
+    w = wl.normal_bf16(N, K, 0.02, 13 * N + K)
+    Wq = mq.quantize_weight(to_dev(w))
+    X = to_dev(x)
+    y1 = to_host_bits(mq.decode_linear_nvfp4(X, Wq))
+    y2 = to_host_bits(mq.decode_linear_nvfp4(X, Wq))
+    assert np.array_equal(y1, y2)
+    ax = oracle.tensor_alpha(x)[1]
+    y3 = to_host_bits(mq.decode_linear_nvfp4(X, Wq, alpha_static=torch.full((1,), ax, dtype=torch.float32,
+                                                                             device="cuda")))
+    assert np.array_equal(y1, y3)
+    _nvfp4_decode_check(x, w, y1, alpha_x=ax)
 
 
 def test_decode_nvfp4_matches_prefill_on_same_weight():

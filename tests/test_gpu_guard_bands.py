@@ -117,7 +117,7 @@ def test_decode_linear_bf16(M, N, K):
     assert mq.async_status(ws) == 0
 
 
-@pytest.mark.parametrize("M,N,K", [(7, 400, 320), (100, 272, 4096)])
+@pytest.mark.parametrize("M,N,K", [(7, 400, 320), (100, 272, 4096), (3, 400, 2048), (1, 272, 8192)])
 def test_decode_linear_nvfp4(M, N, K):
     ws = ws_guarded(M, K)
     W = mq.quantize_weight(to_dev(wl.normal_bf16(N, K, 0.02, N)))
