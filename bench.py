@@ -360,7 +360,9 @@ def _time_stream(torch, calls, reps):
     """Mean device time (ms) per call of `reps` calls issued back to back,
     cycling through `calls` as _time_rotating does: the decode of a layer stack,
     where each call's launch overlaps the previous call's tail."""
-    torch.cuda._sleep(2_000_000)   # the GPU busy while the host enqueues the calls
+    # the GPU spins (~5 ms) while the host enqueues all the calls, so that the
+    # timed span holds device work only, not host launch overhead
+    torch.cuda._sleep(10_000_000)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record()
     for i in range(reps):
