@@ -69,12 +69,12 @@ constexpr int kDecodeMaxGpartTokens = 16; // tokens up to which that split is us
 __device__ __forceinline__ void gsplit_reduce(float* part, uint32_t* tile_ctr, uint32_t* s_flag, int tile, int split,
                                               int M, int N, int row, int lead, float out_scale, uint16_t* y)
 {
-    __threadfence();
+    // every thread's partial stores precede the lead's ticket, whose release
+    // covers them; the last CTA's threads read after its acquire
     named_barrier_sync(2, 128);
-    if (lead) *s_flag = (atomicAdd(&tile_ctr[tile], 1u) == (uint32_t)(split - 1)) ? 1u : 0u;
+    if (lead) *s_flag = (atom_add_acq_rel_gpu(&tile_ctr[tile], 1u) == (uint32_t)(split - 1)) ? 1u : 0u;
     named_barrier_sync(2, 128);
     if (*s_flag == 0u) return;
-    __threadfence();
     const int64_t n = (int64_t)tile * DBM + row;
     const float* base = part + (int64_t)tile * split * M * DBM + row;
     for (int m0 = 0; m0 < M; m0 += 4) {

@@ -157,6 +157,27 @@ __device__ __forceinline__ bool elect_one()
 // that kernel has completed and its memory operations are visible, and
 // grid_dep_launch_dependents() lets the next kernel start early.  Both are
 // no-ops when the launch has no such dependency.
+// Ticket of a "last one folds" hand-off between CTAs: an atomic add with
+// acquire-release semantics at GPU scope.  The release orders the caller's
+// earlier writes, and (being cumulative) those its CTA made before a barrier
+// with the caller, before the increment; the acquire makes every write that
+// the earlier incrementers released visible after it, to the caller and to its
+// CTA after a barrier.  No full fence is needed around it.
+__device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(uint32_t* p, uint32_t v)
+{
+    uint32_t old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
+// Relaxed (not ordering) read of a 32-bit word written by other CTAs.
+__device__ __forceinline__ uint32_t ld_relaxed_gpu_u32(const uint32_t* p)
+{
+    uint32_t v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
 __device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void grid_dep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
 

@@ -87,14 +87,13 @@ __global__ void __launch_bounds__(kAmaxThreads, MQ_AMAX_BLOCKS_PER_SM) amax_kern
         for (int w = 0; w < kAmaxThreads / 32; ++w)
             b = max(b & 0x7FFFFFFFu, warp_max[w] & 0x7FFFFFFFu) | ((b | warp_max[w]) & 0x80000000u);
         partials[blockIdx.x] = b;
-        __threadfence();
-        const uint32_t ticket = atomicAdd(&ctrl->amax_ticket, 1u);
+        const uint32_t ticket = atom_add_acq_rel_gpu(&ctrl->amax_ticket, 1u);   // releases the partial
         is_last = (ticket == gridDim.x - 1);
     }
     __syncthreads();
     if (!is_last) return;
-    // The last block to finish folds all partial maxima.
-    __threadfence();
+    // The last block to finish folds all partial maxima (visible after its
+    // ticket's acquire and the barrier).
     uint32_t b = 0;
     for (int j = threadIdx.x; j < (int)gridDim.x; j += blockDim.x) {
         const uint32_t p = __ldcg(partials + j);
@@ -116,8 +115,7 @@ __global__ void __launch_bounds__(kAmaxThreads, MQ_AMAX_BLOCKS_PER_SM) amax_kern
         // tensor scale: amax / (q_max * E4M3_max) = amax / 2688, or 1 for an all-zero tensor
         *alpha_out = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
         if (r & 0x80000000u) post_error(ctrl, kErrNonFinite);
-        ctrl->amax_ticket = 0;  // ready for the next pass on this workspace
-        __threadfence();
+        ctrl->amax_ticket = 0;  // ready for the next pass on this workspace (visible at kernel end)
     }
 }
 
@@ -436,7 +434,10 @@ __global__ void __launch_bounds__(kQuantThreads, MQ_QUANT_MIN_BLOCKS)
         alpha = *alpha_static;
     } else {
         uint32_t* epoch = &ctrl->epoch;
-        if (threadIdx.x == 0) s_epoch = ld_acquire_u32(epoch);
+        // the epoch before this pass (a relaxed read: it cannot see this pass's
+        // publication, which follows every block's ticket, and it does not hold
+        // back the loads below)
+        if (threadIdx.x == 0) s_epoch = ld_relaxed_gpu_u32(epoch);
         // ---- pass 1: |x| maximum of this block's tiles
         uint32_t mx = 0;
         for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x)
@@ -458,14 +459,13 @@ __global__ void __launch_bounds__(kQuantThreads, MQ_QUANT_MIN_BLOCKS)
             uint32_t b = 0;
             for (int w = 0; w < kQuantThreads / 32; ++w) b = fold_max_flag(b, s_red[w]);
             partials[blockIdx.x] = b;
-            __threadfence();
-            const uint32_t ticket = atomicAdd(&ctrl->amax_ticket, 1u);
+            const uint32_t ticket = atom_add_acq_rel_gpu(&ctrl->amax_ticket, 1u);   // releases the partial
             s_last = (ticket == gridDim.x - 1);
         }
         __syncthreads();
         if (s_last) {
-            // every block's maximum is in `partials`: fold them, publish alpha
-            __threadfence();
+            // every block's maximum is in `partials` (visible after the ticket's
+            // acquire and the barrier): fold them, publish alpha
             uint32_t b = 0;
             for (int j = threadIdx.x; j < (int)gridDim.x; j += blockDim.x) b = fold_max_flag(b, __ldcg(partials + j));
 #pragma unroll
@@ -480,8 +480,7 @@ __global__ void __launch_bounds__(kQuantThreads, MQ_QUANT_MIN_BLOCKS)
                 *alpha_out = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
                 if (r & 0x80000000u) post_error(ctrl, kErrNonFinite);
                 ctrl->amax_ticket = 0;   // ready for the next pass on this workspace
-                __threadfence();
-                st_release_u32(epoch, s_epoch + 1u);
+                st_release_u32(epoch, s_epoch + 1u);   // orders alpha and the reset before it
             }
         }
         // ---- every block: wait for the published alpha
@@ -682,13 +681,11 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_amax_kernel(const uint16
         uint32_t b = 0;
         for (int w = 0; w < kNormThreads / 32; ++w) b = fold_max_flag(b, s_red[w]);
         partials[blockIdx.x] = b;
-        __threadfence();
-        is_last = (atomicAdd(&ctrl->amax_ticket, 1u) == gridDim.x - 1);
+        is_last = (atom_add_acq_rel_gpu(&ctrl->amax_ticket, 1u) == gridDim.x - 1);   // releases the partial
     }
     __syncthreads();
     if (!is_last) return;
     // the last block folds every block's maximum, all threads at once
-    __threadfence();
     uint32_t b = 0;
     for (int j = threadIdx.x; j < (int)gridDim.x; j += kNormThreads) b = fold_max_flag(b, __ldcg(partials + j));
 #pragma unroll
@@ -702,8 +699,7 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_amax_kernel(const uint16
         const float amax = __uint_as_float((b & 0x7FFFu) << 16);
         *alpha_out = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
         if (b & 0x80000000u) post_error(ctrl, kErrNonFinite);
-        ctrl->amax_ticket = 0;
-        __threadfence();
+        ctrl->amax_ticket = 0;   // visible at kernel end
     }
 }
 
