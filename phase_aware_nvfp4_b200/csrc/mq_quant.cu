@@ -9,6 +9,9 @@
 // a launch on the decode-sized inputs.
 #include <mutex>
 
+#include <map>
+#include <utility>
+
 #include "mq_device.cuh"
 
 namespace mq {
@@ -405,7 +408,7 @@ __device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v)
 //     (bounded; a wait that runs out posts kErrTimeout and the block stops).
 //     The quantization pass then walks the tiles in the opposite order, so
 //     the lines read last by the amax pass, still in L2, are read first.
-template <bool SEARCH, bool NORM>
+template <bool SEARCH, bool NORM, bool CLUSTER = false>
 __global__ void __launch_bounds__(kQuantThreads, MQ_QUANT_MIN_BLOCKS)
     quantize_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t K, const float* __restrict__ alpha_static,
                     float* __restrict__ alpha_out, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
@@ -416,6 +419,7 @@ __global__ void __launch_bounds__(kQuantThreads, MQ_QUANT_MIN_BLOCKS)
     __shared__ float dec_tab[128];   // fl(alpha * sigma) for every E4M3 code sigma
     __shared__ uint32_t s_red[kQuantThreads / 32];
     __shared__ uint32_t s_epoch, s_last, s_ok;
+    __shared__ uint32_t s_slot[CLUSTER ? 16 : 1];   // cluster hand-off: one maximum per CTA
     __shared__ float s_alpha;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int half = lane >> 4;
@@ -432,6 +436,42 @@ __global__ void __launch_bounds__(kQuantThreads, MQ_QUANT_MIN_BLOCKS)
     float alpha;
     if (alpha_static != nullptr) {
         alpha = *alpha_static;
+    } else if (CLUSTER) {
+        // The whole grid is one thread-block cluster: each CTA's maximum goes
+        // straight into a slot of every CTA's shared memory and two cluster
+        // barriers replace the global ticket, fold and spin.
+        const int cluster = (int)gridDim.x;
+        const uint32_t rank = cluster_ctarank();
+        cluster_barrier();   // every CTA runs before its shared memory is written remotely
+        uint32_t mx = 0;
+        for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x)
+            mx = amax_tile(x, rows, K, interleave_half, t / chunks, t % chunks, warp, half, blk, mx);
+        uint32_t m = max(mx & 0xFFFFu, mx >> 16);
+        if (m >= 0x7F80u) {
+            uint32_t bad = 0;
+            mx = 0;
+            for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x)
+                mx = amax_tile_finite(x, rows, K, interleave_half, t / chunks, t % chunks, warp, half, blk, mx, bad);
+            m = max(mx & 0xFFFFu, mx >> 16) | (bad ? 0x80000000u : 0u);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fold_max_flag(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+        if (lane == 0) s_red[warp] = m;
+        __syncthreads();
+        if (threadIdx.x < cluster) {
+            uint32_t b = 0;
+            for (int w = 0; w < kQuantThreads / 32; ++w) b = fold_max_flag(b, s_red[w]);
+            st_cluster_u32(map_to_cta(smem_u32(&s_slot[rank]), (uint32_t)threadIdx.x), b);
+        }
+        cluster_barrier();   // release / acquire: every CTA's slot is written
+        uint32_t r = 0;
+        for (int q = 0; q < cluster; ++q) r = fold_max_flag(r, s_slot[q]);
+        const float amax = __uint_as_float((r & 0x7FFFu) << 16);
+        alpha = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
+        if (rank == 0 && threadIdx.x == 0) {
+            *alpha_out = alpha;
+            if (r & 0x80000000u) post_error(ctrl, kErrNonFinite);
+        }
     } else {
         uint32_t* epoch = &ctrl->epoch;
         // the epoch before this pass (a relaxed read: it cannot see this pass's
@@ -528,6 +568,38 @@ int quantize_blocks_per_sm(const DeviceInfo& di)
     return occ;
 }
 
+// Whether `kern` can run as one cluster of `cl` CTAs of kQuantThreads (cached
+// per device, kernel and size; sizes above 8 are non-portable and opted into).
+template <bool SEARCH>
+bool quantize_cluster_fits(int cl, const DeviceInfo& di)
+{
+    static std::mutex mu;
+    static std::map<std::pair<int, int>, bool> cache;
+    std::lock_guard<std::mutex> lock(mu);
+    const auto key = std::make_pair(di.device, cl);
+    auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+    auto kern = quantize_kernel<SEARCH, false, true>;
+    bool ok = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
+    if (ok) {
+        cudaLaunchConfig_t cfg{};
+        cfg.gridDim = dim3((unsigned)cl, 1, 1);
+        cfg.blockDim = dim3(kQuantThreads, 1, 1);
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)cl;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int clusters = 0;
+        ok = cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) == cudaSuccess && clusters >= 1;
+    }
+    (void)cudaGetLastError();
+    cache[key] = ok;
+    return ok;
+}
+
 cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float* alpha_static, float* alpha_out,
                             uint8_t* codes, uint8_t* scales, int64_t interleave_half, WsControl* ctrl,
                             uint32_t* partials, const DeviceInfo& di, cudaStream_t s, bool scale_search)
@@ -535,12 +607,19 @@ cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float*
     const int64_t tiles = ((rows + 127) / 128) * ((K + 255) / 256);
     const int occ = scale_search ? quantize_blocks_per_sm<true, false>(di) : quantize_blocks_per_sm<false, false>(di);
     const int64_t resident = (int64_t)di.num_sms * std::max(1, occ);
-    // Small tensors (at most one tile per SM): one cooperative launch takes
-    // the amax, hands alpha to every block and quantizes; the two-kernel path
-    // would pay a second launch and its ramp for a few microseconds of work.
-    // Larger tensors: the amax kernel (full occupancy) and then the
-    // quantization kernel with that alpha.
+    // Small tensors (at most one tile per SM): one launch takes the amax,
+    // hands alpha to every block and quantizes; the two-kernel path would pay
+    // a second launch and its ramp for a few microseconds of work.  Up to 16
+    // tiles the grid is one thread-block cluster whose CTAs exchange their
+    // maxima through distributed shared memory; otherwise a cooperative launch
+    // hands alpha over through global memory.  Larger tensors: the amax kernel
+    // (full occupancy) and then the quantization kernel with that alpha.
     const bool single = (alpha_static == nullptr) && tiles <= di.num_sms && occ > 0;
+    const int cl = (single && tiles <= 16 &&
+                    (scale_search ? quantize_cluster_fits<true>((int)tiles, di)
+                                  : quantize_cluster_fits<false>((int)tiles, di)))
+                       ? (int)tiles
+                       : 0;
     const float* alpha_in = alpha_static;
     if (alpha_static == nullptr && !single) {
         cudaError_t e = launch_amax(x, rows * K, alpha_out, ctrl, partials, di, s);
@@ -555,17 +634,27 @@ cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float*
     cfg.blockDim = dim3(kQuantThreads, 1, 1);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    if (single) {   // blocks wait on one another only in the single-launch amax
+    cudaLaunchAttribute attr[2];
+    cfg.attrs = attr;
+    if (cl > 0) {   // one cluster (the grid is `tiles` CTAs); may overlap its predecessor's tail
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)cl;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
+        cfg.numAttrs = 2;
+    } else if (single) {   // blocks wait on one another only in the single-launch amax
         attr[0].id = cudaLaunchAttributeCooperative;
         attr[0].val.cooperative = 1;
+        cfg.numAttrs = 1;
     } else {
         attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.numAttrs = 1;
     }
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    auto kern = scale_search ? quantize_kernel<true, false> : quantize_kernel<false, false>;
+    auto kern = cl > 0 ? (scale_search ? quantize_kernel<true, false, true> : quantize_kernel<false, false, true>)
+                       : (scale_search ? quantize_kernel<true, false> : quantize_kernel<false, false>);
     cudaError_t e = cudaLaunchKernelEx(&cfg, kern, static_cast<const uint16_t*>(x), rows, K, alpha_in, alpha_out,
                                        codes, scales, interleave_half, ctrl, partials, NormArgs{});
     if (e != cudaSuccess) return e;
