@@ -997,12 +997,14 @@ cudaError_t launch_decode_nvfp4_fused(const void* x, int64_t M, const float* alp
     // then the larger grid.
     //   With a partial workspace, the K split runs over independent CTAs (any
     // split 1..8, several CTAs per SM; each CTA takes the amax over all of X,
-    // at most 512K elements); otherwise over a cluster (split a power of two).
+    // so only for at most 64K elements: beyond that every CTA re-reading all
+    // tokens costs more than a cluster's exchange of slice maxima); otherwise
+    // over a cluster (split a power of two).
     constexpr int64_t kSaturateBytes = 16ll << 20;
     int best_split = 0, best_st = 0, best_smem = 0, best_gpart = 0;
     int64_t best_score = -1;
     const bool can_gpart = sw.part != nullptr && M <= kDecodeMaxGpartTokens &&
-                           (p.alpha_static != nullptr || M * K <= (int64_t)1 << 19);
+                           (p.alpha_static != nullptr || M * K <= (int64_t)1 << 16);
     for (int sp = 1; sp <= 8 && sp <= p.k_stages; ++sp) {
         const bool gp = can_gpart && (sp == 1 || (size_t)sp * n_tiles * M * DBM * 4 <= sw.part_bytes);
         if (!gp && (sp & (sp - 1)) != 0) continue;   // a cluster split is a power of two
