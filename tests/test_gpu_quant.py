@@ -40,6 +40,36 @@ def test_quantize_activation_bit_exact(M, K, kind):
     _check_quant(x, t)
 
 
+@pytest.mark.parametrize("M,K", [(7, 2048), (64, 2304), (128, 4096), (8, 4352)])
+def test_small_activation_launch_shapes_bit_exact(M, K):
+    """Small activations are quantized in one launch: up to 16 tiles of 128 x 256 by one
+    thread-block cluster exchanging the block maxima through distributed shared memory (8, 9
+    and 16 CTAs here, 16 being the non-portable maximum), 17 tiles by the cooperative launch.
+    Codes, scales and alpha are bit-exact either way."""
+    x = wl.heavy_tailed_bf16(M, K, 17 + M)
+    t = mq.quantize_activation(to_dev(x))
+    torch.cuda.synchronize()
+    _check_quant(x, t)
+
+
+def test_nonfinite_input_in_a_cluster_quantization():
+    """A NaN in a 16-tile activation (one cluster): reported as MQ_ERR_NONFINITE, excluded from
+    the tensor amax; the other rows' codes and scales match the oracle with that alpha."""
+    x = wl.heavy_tailed_bf16(32, 4096, 23)
+    x[17, 3001] = 0x7FC0
+    ws = mq.workspace(32, 4096)
+    t = mq.quantize_activation(to_dev(x), ws=ws)
+    assert mq.async_status(ws) == 5
+    amax, ax, bad = oracle.tensor_alpha(x)
+    assert bad
+    codes, scales, alpha = nvfp4_host(t)
+    assert np.float32(alpha) == np.float32(ax)
+    ok = np.arange(32) != 17
+    rc, rs = oracle.quantize(x[ok], ax)
+    assert np.array_equal(codes[ok], rc)
+    assert np.array_equal(scales[ok], rs)
+
+
 def test_tiny_workload_quantization():
     """The tiny 128x256x256 workload: X ~ N(0,1), W ~ N(0, 0.02^2), seed 0."""
     p = wl.tiny().projections[0]
