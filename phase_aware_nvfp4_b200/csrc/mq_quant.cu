@@ -706,12 +706,13 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_amax_kernel(const uint16
         if (lane == 0 && r + wstride < rows)
             bulk_prefetch_l2(x + (r + wstride) * K, (uint32_t)std::min<int64_t>(K * 2, (int64_t)1 << 20));
         uint4 v[kNormChunk];
-        // sum of squares: each square of a BF16 value is exact in binary32
-        // (8 significant bits, for |x| in [2^-63, 2^63]) and is added in
-        // binary64 (two running sums per lane, then a butterfly over the warp):
-        // the binary64 sum of the definition up to the order of the additions,
-        // which moves ms only when the sum lies within ~2^-40 relative of an
-        // FP32 rounding boundary.
+        // sum of squares in binary64: x widened exactly, x * x exact (16
+        // significant bits, every BF16 value incl. subnormals and |x| >= 2^64)
+        // and added with one rounding by the fused multiply-add, as in the
+        // definition; four running sums per lane, then a butterfly over the
+        // warp: the definition's sum up to the order of the additions, which
+        // moves ms only when the sum lies within ~2^-40 relative of an FP32
+        // rounding boundary.
         double s[4] = {0.0, 0.0, 0.0, 0.0};   // four independent chains
         for (int64_t c0 = 0; c0 < nv; c0 += chunk) {
 #pragma unroll
@@ -724,11 +725,9 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_amax_kernel(const uint16
                 const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    const float a = bf16_lo(w[j]), b = bf16_hi(w[j]);
-                    float a2, b2;
-                    fmul2v_rn(a, b, a, b, a2, b2);
-                    s[(j & 1) * 2] = __dadd_rn(s[(j & 1) * 2], (double)a2);
-                    s[(j & 1) * 2 + 1] = __dadd_rn(s[(j & 1) * 2 + 1], (double)b2);
+                    const double a = (double)bf16_lo(w[j]), b = (double)bf16_hi(w[j]);
+                    s[(j & 1) * 2] = __fma_rn(a, a, s[(j & 1) * 2]);
+                    s[(j & 1) * 2 + 1] = __fma_rn(b, b, s[(j & 1) * 2 + 1]);
                 }
             }
         }
@@ -738,6 +737,10 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_amax_kernel(const uint16
         const float ms = __double2float_rn(__ddiv_rn(ss, (double)K));
         const float rs = __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(__dadd_rn((double)ms, (double)eps))));
         if (lane == 0) rstd[r] = rs;
+        // |h| maximum of the row over all values (two instructions per pair);
+        // a NaN or Inf among them (magnitude bits 0x7F80 and above, rare) sends
+        // the row through the finite-only fold, which also raises the flag
+        uint32_t mrow = 0;
         for (int64_t c0 = 0; c0 < nv; c0 += chunk) {
             if (nv > chunk) {   // the chunk is no longer in registers
 #pragma unroll
@@ -751,13 +754,25 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_amax_kernel(const uint16
                 const int64_t i = c0 + lane + 32 * u;
                 if (i < nv) {
                     const uint4 g = g_smem ? gr[i] : __ldg(gr + i);
-                    amax_accum(norm_pair(v[u].x, g.x, rs), mx, bad);
-                    amax_accum(norm_pair(v[u].y, g.y, rs), mx, bad);
-                    amax_accum(norm_pair(v[u].z, g.z, rs), mx, bad);
-                    amax_accum(norm_pair(v[u].w, g.w, rs), mx, bad);
+                    mrow = max_u16x2(mrow, norm_pair(v[u].x, g.x, rs) & 0x7FFF7FFFu);
+                    mrow = max_u16x2(mrow, norm_pair(v[u].y, g.y, rs) & 0x7FFF7FFFu);
+                    mrow = max_u16x2(mrow, norm_pair(v[u].z, g.z, rs) & 0x7FFF7FFFu);
+                    mrow = max_u16x2(mrow, norm_pair(v[u].w, g.w, rs) & 0x7FFF7FFFu);
                 }
             }
         }
+        if (__any_sync(0xFFFFFFFFu, max(mrow & 0xFFFFu, mrow >> 16) >= 0x7F80u)) {
+            mrow = 0;
+            for (int64_t i = lane; i < nv; i += 32) {
+                const uint4 xv = __ldg(xr + i);
+                const uint4 g = g_smem ? gr[i] : __ldg(gr + i);
+                amax_accum(norm_pair(xv.x, g.x, rs), mrow, bad);
+                amax_accum(norm_pair(xv.y, g.y, rs), mrow, bad);
+                amax_accum(norm_pair(xv.z, g.z, rs), mrow, bad);
+                amax_accum(norm_pair(xv.w, g.w, rs), mrow, bad);
+            }
+        }
+        mx = max_u16x2(mx, mrow);
     }
     uint32_t m = max(mx & 0xFFFFu, mx >> 16) | (bad ? 0x80000000u : 0u);
 #pragma unroll

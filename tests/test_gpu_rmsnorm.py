@@ -67,3 +67,19 @@ def test_rmsnorm_quantize_closed_form_and_nonfinite():
     mq.rmsnorm_quantize(to_dev(xb), to_dev(g), 1e-6, ws=ws)
     assert mq.async_status(ws) == 5
     assert mq.async_status(ws) == 0
+
+
+def test_rmsnorm_quantize_extreme_magnitudes_bit_exact():
+    """Squares that binary32 cannot hold: rows with one element of 2^64 (x^2 = 2^128, past FP32's
+    range) and rows scaled to ~2^-72 (x^2 ~ 2^-144, FP32 subnormal).  The definition squares and
+    adds in binary64, where both are exact, so h and its NVFP4 tensor stay bit-exact."""
+    M, K = 64, 512
+    base = wl.bf16_bits_to_f32(wl.heavy_tailed_bf16(M, K, 67))
+    big = wl.f32_to_bf16_bits(base[:32])
+    for r in range(32):
+        big[r, (37 * r) % K] = 0x5F80          # 2^64
+    tiny = wl.f32_to_bf16_bits(base[32:] * np.float32(2.0 ** -72))
+    x = np.concatenate([big, tiny])
+    assert np.all((x[32:] & 0x7F80) != 0x7F80)
+    g = wl.normal_bf16(1, K, 1.0, 68)[0]
+    _check(x, g, 0.0)
