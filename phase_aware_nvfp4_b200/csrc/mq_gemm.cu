@@ -658,20 +658,23 @@ __device__ __forceinline__ void epilogue_half_silu_bf16(const EpiScales& es, uin
     }
 }
 
-// KV half-tile (EPI 2) of the pair kernel: the warp's 32 tokens x one
-// 128-column head.  Same arithmetic as kv_rope_store, with the global traffic
-// of a warp coalesced through its 4 KiB staging buffer (rows swizzled by
-// 16-byte chunk, chunk ^ row % 8, so both the row-wise and the column-wise
-// passes are free of bank conflicts):
-//   - for K heads, the cos/sin values of the 32 tokens' positions come in four
-//     chunks of 16 frequencies: per chunk the warp loads 32 rows x (64 B of
-//     cos + 64 B of sin) with 16-byte loads, eight lanes per row
-//     (kv_stage_cos_sin; the first chunk is staged before the accumulator
-//     wait, so its latency overlaps the tile's MMAs), and each lane then reads
-//     its own token's values;
+// KV half-tile (EPI 2) of the pair kernel.  The tile's 256 columns are two
+// 128-column heads, A (columns 0..127) and B (128..255); the warp of half h
+// takes frequencies 32h .. 32h + 31 of both heads, i.e. accumulator columns
+// 32h + {0, 64, 128, 192} + 0..31, so the cos/sin values it needs (the 32
+// tokens' rows at those frequencies) serve both heads.  Same arithmetic as
+// kv_rope_store; the global traffic of a warp goes through its 4 KiB staging
+// buffer (rows swizzled by 16-byte chunk, chunk ^ row % 8, so the row-wise and
+// the column-wise passes are free of bank conflicts):
+//   - the cos/sin values come in two chunks of 16 frequencies: per chunk the
+//     warp loads 32 rows x (64 B of cos + 64 B of sin) with 16-byte loads,
+//     eight lanes per row (kv_stage_cos_sin; the first chunk is staged before
+//     the accumulator wait, so its latency overlaps the tile's MMAs), and each
+//     lane then reads its own token's values;
 //   - each rotated pair of columns is rounded to BF16 at once, and the result
-//     leaves in two 64-column halves: each lane writes its token's 128 bytes,
-//     then the warp stores eight lanes per 128-byte segment of a cache slot.
+//     leaves head by head: each lane writes its token's two 64-byte pieces
+//     (columns 32h .. 32h + 31 and 64 + 32h .. 64 + 32h + 31 of the head row),
+//     then the warp stores four lanes per piece.
 // pos / slot / valid: this lane's token (loaded before the accumulator wait).
 __device__ __forceinline__ void kv_stage_cos_sin(const Params& p, uint8_t* stg, int lane, int32_t pos, int ch)
 {
@@ -690,66 +693,74 @@ __device__ __forceinline__ void kv_stage_cos_sin(const Params& p, uint8_t* stg, 
 
 template <class Barrier>
 __device__ __forceinline__ void epilogue_half_kv(const Params& p, float alpha_ab, uint32_t t_col, int lane,
-                                                 uint8_t* stg, int hh, int32_t pos, int64_t slot, bool valid,
-                                                 Barrier arrive)
+                                                 uint8_t* stg, int half, int n_blk, int32_t pos, int64_t slot,
+                                                 bool valid, Barrier arrive)
 {
-    uint32_t acc[4][32];
+    uint32_t acc[4][32];   // [head A low, head A high, head B low, head B high][frequency 32 half + j]
 #pragma unroll
-    for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(t_col + 32 * c, acc[c]);
+    for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(t_col + 64 * c, acc[c]);
     tmem_wait_ld(acc[0]);
 #pragma unroll
     for (int c = 1; c < 4; ++c) tmem_wait_ld(acc[c]);
     release_acc_warp(lane, arrive);
 
-    const bool is_k = hh < p.n_heads;
-    const int head = is_k ? hh : hh - p.n_heads;
-    uint32_t out[64];   // BF16 pairs: out[w] holds columns 2w, 2w + 1
-    if (is_k) {
+    // K heads come first, so head B is a K head only if head A is one
+    const bool rot_a = 2 * n_blk < p.n_heads, rot_b = 2 * n_blk + 1 < p.n_heads;
+    uint32_t out[4][16];   // BF16 pairs: out[c][w] holds frequencies 32 half + 2w, + 2w + 1 of stream c
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-            if (ch > 0) kv_stage_cos_sin(p, stg, lane, pos, ch);   // chunk 0 was staged before the wait
+    for (int ch = 0; ch < 2; ++ch) {
+        if (rot_a && ch > 0) kv_stage_cos_sin(p, stg, lane, pos, 2 * half + 1);   // chunk 2 half was staged before the wait
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                // cos and sin of frequencies 16 ch + 4 q .. + 3 from this token's staged row
+        for (int q = 0; q < 4; ++q) {
+            float cc[4] = {1.f, 1.f, 1.f, 1.f}, ss[4] = {0.f, 0.f, 0.f, 0.f};
+            if (rot_a) {
+                // cos and sin of frequencies 32 half + 16 ch + 4 q .. + 3 from this token's staged row
                 const float4 cv = *reinterpret_cast<const float4*>(stg + lane * 128 + ((q ^ (lane & 7)) << 4));
                 const float4 sv = *reinterpret_cast<const float4*>(stg + lane * 128 + (((q + 4) ^ (lane & 7)) << 4));
-                const float cc[4] = {cv.x, cv.y, cv.z, cv.w};
-                const float ss[4] = {sv.x, sv.y, sv.z, sv.w};
+                cc[0] = cv.x, cc[1] = cv.y, cc[2] = cv.z, cc[3] = cv.w;
+                ss[0] = sv.x, ss[1] = sv.y, ss[2] = sv.z, ss[3] = sv.w;
+            }
+#pragma unroll
+            for (int hd = 0; hd < 2; ++hd) {
+                const bool rot = hd == 0 ? rot_a : rot_b;
                 float lo[4], hi[4];
 #pragma unroll
                 for (int t = 0; t < 4; ++t) {
-                    const int i = 16 * ch + 4 * q + t;   // frequency: columns i and i + 64
-                    const float a = __fmul_rn(__uint_as_float(acc[i >> 5][i & 31]), alpha_ab);
-                    const float b = __fmul_rn(__uint_as_float(acc[(i + 64) >> 5][(i + 64) & 31]), alpha_ab);
-                    lo[t] = __fsub_rn(__fmul_rn(a, cc[t]), __fmul_rn(b, ss[t]));
-                    hi[t] = __fadd_rn(__fmul_rn(b, cc[t]), __fmul_rn(a, ss[t]));
+                    const int j = 16 * ch + 4 * q + t;
+                    const float a = __fmul_rn(__uint_as_float(acc[2 * hd][j]), alpha_ab);
+                    const float b = __fmul_rn(__uint_as_float(acc[2 * hd + 1][j]), alpha_ab);
+                    if (rot) {
+                        lo[t] = __fsub_rn(__fmul_rn(a, cc[t]), __fmul_rn(b, ss[t]));
+                        hi[t] = __fadd_rn(__fmul_rn(b, cc[t]), __fmul_rn(a, ss[t]));
+                    } else {
+                        lo[t] = a;
+                        hi[t] = b;
+                    }
                 }
-                const int w = 8 * ch + 2 * q;   // column 16 ch + 4 q = 2 w
-                out[w] = pack_bf16x2(lo[0], lo[1]);
-                out[w + 1] = pack_bf16x2(lo[2], lo[3]);
-                out[w + 32] = pack_bf16x2(hi[0], hi[1]);
-                out[w + 33] = pack_bf16x2(hi[2], hi[3]);
+                const int w = 8 * ch + 2 * q;
+                out[2 * hd][w] = pack_bf16x2(lo[0], lo[1]);
+                out[2 * hd][w + 1] = pack_bf16x2(lo[2], lo[3]);
+                out[2 * hd + 1][w] = pack_bf16x2(hi[0], hi[1]);
+                out[2 * hd + 1][w + 1] = pack_bf16x2(hi[2], hi[3]);
             }
-            __syncwarp();   // the next chunk's loads overwrite the staging rows
         }
-    } else {
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-            for (int j = 0; j < 16; ++j)
-                out[16 * c + j] = pack_bf16x2(__fmul_rn(__uint_as_float(acc[c][2 * j]), alpha_ab),
-                                              __fmul_rn(__uint_as_float(acc[c][2 * j + 1]), alpha_ab));
+        __syncwarp();   // the next chunk's loads (or the stores) overwrite the staging rows
     }
-    uint16_t* cache = is_k ? p.k_cache : p.v_cache;
     const int sub = lane >> 3, piece = lane & 7;
+    // destination column of this lane's 16-byte piece: low half (pieces 0..3)
+    // or high half (4..7) of the head row, at the warp's 32 frequencies
+    const int col = (piece < 4 ? 0 : 64) + 32 * half + 8 * (piece & 3);
 #pragma unroll
-    for (int hq = 0; hq < 2; ++hq) {
-        // this token's columns 64 hq .. 64 hq + 63, then eight lanes per cache row segment
+    for (int hd = 0; hd < 2; ++hd) {
+        const int hh = 2 * n_blk + hd;
+        const bool is_k = hh < p.n_heads;
+        const int head = is_k ? hh : hh - p.n_heads;
+        uint16_t* cache = is_k ? p.k_cache : p.v_cache;
+        // this token's two pieces: staged chunks 0..3 = low, 4..7 = high
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
-            const int w = 32 * hq + 4 * q;
-            *reinterpret_cast<uint4*>(stg + lane * 128 + ((q ^ (lane & 7)) << 4)) =
-                make_uint4(out[w], out[w + 1], out[w + 2], out[w + 3]);
+            const uint32_t* o = out[2 * hd + (q >> 2)] + 4 * (q & 3);
+            *reinterpret_cast<uint4*>(stg + lane * 128 + ((q ^ (lane & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
         }
         __syncwarp();
 #pragma unroll
@@ -758,7 +769,7 @@ __device__ __forceinline__ void epilogue_half_kv(const Params& p, float alpha_ab
             const int64_t sr = __shfl_sync(0xFFFFFFFFu, slot, r);
             const int vr = __shfl_sync(0xFFFFFFFFu, valid ? 1 : 0, r);
             if (vr) {
-                uint4* dst = reinterpret_cast<uint4*>(cache + (sr * p.n_heads + head) * 128 + 64 * hq) + piece;
+                uint4* dst = reinterpret_cast<uint4*>(cache + (sr * p.n_heads + head) * 128 + col);
                 *dst = *reinterpret_cast<const uint4*>(stg + r * 128 + ((piece ^ (r & 7)) << 4));
             }
         }
@@ -983,34 +994,46 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_NUM_THREADS, 1)
         const int half = (warp - 2) >> 2;
         EpiScales es = epi_scales<EPI>(p);
         const uint32_t leader_acc_empty = map_to_cta(smem_u32(acc_empty), 0);
-        const uint32_t t_col = tmem_base + ((uint32_t)(32 * lg) << 16) + (uint32_t)(128 * half);
+        // column offset of this warp's accumulator half: 128 columns of the tile,
+        // or (KV) 32 columns in each of the four 64-column quarters
+        const uint32_t t_col = tmem_base + ((uint32_t)(32 * lg) << 16) + (uint32_t)(EPI == 2 ? 32 * half : 128 * half);
         uint8_t* stg = smem + P_OFF_STG + (warp - 2) * P_STG_BYTES;
         auto arrive = [&] { mbar_arrive_cluster(leader_acc_empty); };
         uint32_t acc_phase = 0;
+        // KV epilogue: this lane's token position and cache slot for a tile,
+        // loaded one tile ahead (the loads of the next tile are in flight
+        // during this tile's epilogue) and checked at the top of the tile: an
+        // out-of-range one posts kErrIndex and the token is not written
+        int32_t nx_pos = -1;
+        int64_t nx_slot = -1;
+        bool nx_in = false;
+        auto kv_fetch = [&](int t) {
+            int mb, nb;
+            tile_coords(p, t, mb, nb);
+            const int64_t m = (int64_t)mb * 2 * BM + (int64_t)rank * BM + 32 * lg + lane;
+            nx_in = m < p.M;
+            if (nx_in) {
+                nx_pos = __ldg(p.positions + m);
+                nx_slot = __ldg(p.slots + m);
+            }
+        };
+        if (EPI == 2 && pair < p.num_tiles) kv_fetch(pair);
         for (int tile = pair; tile < p.num_tiles; tile += npairs) {
             int m_blk, n_blk;
             tile_coords(p, tile, m_blk, n_blk);
-            // KV epilogue: this lane's token position and cache slot, fetched
-            // before the accumulator wait; an out-of-range one posts kErrIndex
-            // and the token is not written
             int32_t kv_pos = 0;
             int64_t kv_slot = 0;
             bool kv_valid = false;
-            if (EPI == 2) {
-                const int64_t m = (int64_t)m_blk * 2 * BM + (int64_t)rank * BM + 32 * lg + lane;
-                if (m < p.M) {
-                    const int32_t ps = __ldg(p.positions + m);
-                    const int64_t sl = __ldg(p.slots + m);
-                    kv_valid = ps >= 0 && ps < p.max_pos && sl >= 0 && sl < p.num_slots;
-                    if (kv_valid) {
-                        kv_pos = ps;
-                        kv_slot = sl;
-                    } else {
-                        post_error(p.ctrl, kErrIndex);
-                    }
+            if (EPI == 2 && nx_in) {
+                kv_valid = nx_pos >= 0 && nx_pos < p.max_pos && nx_slot >= 0 && nx_slot < p.num_slots;
+                if (kv_valid) {
+                    kv_pos = nx_pos;
+                    kv_slot = nx_slot;
+                } else {
+                    post_error(p.ctrl, kErrIndex);
                 }
             }
-            if (EPI == 2 && 2 * n_blk + half < p.n_heads) kv_stage_cos_sin(p, stg, lane, kv_pos, 0);
+            if (EPI == 2 && 2 * n_blk < p.n_heads) kv_stage_cos_sin(p, stg, lane, kv_pos, 2 * half);
             if (!warp_wait(acc_full, acc_phase, abort_flag)) {
                 if (lane == 0) {
                     post_error(p.ctrl, kErrTimeout);
@@ -1020,6 +1043,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_NUM_THREADS, 1)
             }
             acc_phase ^= 1u;
             tc_fence_after();
+            if (EPI == 2 && tile + npairs < p.num_tiles) kv_fetch(tile + npairs);
             const int64_t row0 = (int64_t)m_blk * 2 * BM + (int64_t)rank * BM + 32 * lg;
             if (EPI == 0) {
                 epilogue_half_bf16_tma(es, t_col, lane, stg, &tmap_y, n_blk * BN + 128 * half, (int32_t)row0, arrive);
@@ -1029,8 +1053,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_NUM_THREADS, 1)
                 epilogue_half_silu_bf16(es, t_col, lane, stg, &tmap_y, n_blk * (BN / 2) + 64 * half, (int32_t)row0,
                                         arrive);
             } else {
-                epilogue_half_kv(p, es.alpha_ab, t_col, lane, stg, 2 * n_blk + half, kv_pos, kv_slot, kv_valid,
-                                 arrive);
+                epilogue_half_kv(p, es.alpha_ab, t_col, lane, stg, half, n_blk, kv_pos, kv_slot, kv_valid, arrive);
             }
         }
         // every output store has finished before the CTA may leave

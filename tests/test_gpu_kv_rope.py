@@ -100,3 +100,39 @@ def test_kv_rope_bad_position_is_reported():
     torch.cuda.synchronize()
     assert not torch.any(kc[3].view(torch.int16) != 0)          # the bad token was not written
     assert torch.any(kc[2].view(torch.int16) != 0)
+
+
+def test_kv_rope_pair_kernel_skips_bad_tokens_only():
+    """CTA-pair kernel (M > 128), one K/V tile row with a position past the table and one with a
+    negative slot: the call reports MQ_ERR_INDEX, those two tokens write nothing, and every other
+    token's K'/V rows still match the oracle (the tile's index loads run one tile ahead)."""
+    M, K, H, max_pos = 300, 512, 3, 4096
+    rng = np.random.default_rng(94)
+    x = wl.heavy_tailed_bf16(M, K, 95)
+    w = wl.normal_bf16(2 * H * 128, K, 0.02, 96)
+    pos = rng.integers(0, max_pos, size=M).astype(np.int32)
+    num_slots = M + 11
+    slots = rng.permutation(num_slots)[:M].astype(np.int64)
+    bad_pos_row, bad_slot_row = 17, 250
+    freed = slots[bad_slot_row]
+    pos[bad_pos_row] = max_pos
+    slots[bad_slot_row] = -1
+    cs = wl.rope_cos_sin(max_pos)
+    Wq = mq.quantize_weight(to_dev(w))
+    kc = torch.zeros((num_slots, H, 128), dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    ws = mq.workspace(M, K)
+    mq.prefill_kv_rope(to_dev(x), Wq, n_kv_heads=H, positions=torch.from_numpy(pos).cuda(),
+                       cos_sin=torch.from_numpy(cs).cuda(), slots=torch.from_numpy(slots).cuda(), k_cache=kc,
+                       v_cache=vc, ws=ws)
+    torch.cuda.synchronize()
+    assert mq.async_status(ws) == 9                           # MQ_ERR_INDEX
+    good = np.setdiff1d(np.arange(M), [bad_pos_row, bad_slot_row])
+    # the two skipped tokens' rows: the bad-position token's own slot and the slot the
+    # bad-slot token would have had are both left at zero
+    for sl in (slots[bad_pos_row], freed):
+        assert not torch.any(kc[int(sl)].view(torch.int16) != 0)
+        assert not torch.any(vc[int(sl)].view(torch.int16) != 0)
+    slots_chk = slots.copy()
+    slots_chk[bad_slot_row] = freed
+    _check(x, w, pos, slots_chk, cs, kc, vc, num_slots, good)
