@@ -674,6 +674,50 @@ cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float*
 constexpr int kNormThreads = 256;
 constexpr int64_t kNormGammaSmem = 8192;   // gamma elements staged in shared memory (16 KiB)
 
+// End of an RMSNorm first pass: folds the threads' |h| maxima (BF16
+// magnitudes, two per word in mx) and non-finite flags into one word per
+// block (bit 31 = flag), publishes it in partials[block], and the block that
+// takes the last ticket folds every block's word into
+// alpha_h = amax / 2688 (1 if the maximum is 0) and posts kErrNonFinite if
+// any block saw a NaN/Inf.  Every thread of the block calls it.
+template <int WARPS>
+__device__ __forceinline__ void norm_alpha_publish(uint32_t mx, uint32_t bad, float* __restrict__ alpha_out,
+                                                   WsControl* ctrl, uint32_t* __restrict__ partials)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t m = max(mx & 0xFFFFu, mx >> 16) | (bad ? 0x80000000u : 0u);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fold_max_flag(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    __shared__ uint32_t s_red[WARPS];
+    __shared__ bool is_last;
+    if (lane == 0) s_red[warp] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t b = 0;
+        for (int w = 0; w < WARPS; ++w) b = fold_max_flag(b, s_red[w]);
+        partials[blockIdx.x] = b;
+        is_last = (atom_add_acq_rel_gpu(&ctrl->amax_ticket, 1u) == gridDim.x - 1);   // releases the partial
+    }
+    __syncthreads();
+    if (!is_last) return;
+    // the last block folds every block's maximum, all threads at once
+    uint32_t b = 0;
+    for (int j = threadIdx.x; j < (int)gridDim.x; j += WARPS * 32) b = fold_max_flag(b, __ldcg(partials + j));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) b = fold_max_flag(b, __shfl_xor_sync(0xFFFFFFFFu, b, o));
+    __syncthreads();
+    if (lane == 0) s_red[warp] = b;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        b = 0;
+        for (int w = 0; w < WARPS; ++w) b = fold_max_flag(b, s_red[w]);
+        const float amax = __uint_as_float((b & 0x7FFFu) << 16);
+        *alpha_out = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
+        if (b & 0x80000000u) post_error(ctrl, kErrNonFinite);
+        ctrl->amax_ticket = 0;   // visible at kernel end
+    }
+}
+
 __global__ void __launch_bounds__(kNormThreads) rmsnorm_amax_kernel(const uint16_t* __restrict__ x, int64_t rows,
                                                                     int64_t K, const uint16_t* __restrict__ gamma,
                                                                     float eps, float* __restrict__ rstd,
@@ -774,43 +818,148 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_amax_kernel(const uint16
         }
         mx = max_u16x2(mx, mrow);
     }
-    uint32_t m = max(mx & 0xFFFFu, mx >> 16) | (bad ? 0x80000000u : 0u);
+    norm_alpha_publish<kNormThreads / 32>(mx, bad, alpha_out, ctrl, partials);
+}
+
+// Pass 1 with two warps per row, for rows of at most kNormPairMaxK elements:
+// warp 2p + g of the block takes half g of each of its rows (16-byte vectors
+// [g nh, (g + 1) nh), nh = K / 16), so the grid holds twice as many rows in
+// flight as with one warp per row, with half the registers per warp.  The
+// two warps add their binary64 partial sums in a fixed order (half 0 +
+// half 1) through shared memory (double-buffered by row parity, one named
+// barrier per row), so both derive the same rstd; each then takes the |h|
+// maximum of its half.  Arithmetic otherwise as rmsnorm_amax_kernel.
+constexpr int64_t kNormPairMaxK = 4096;
+constexpr int kNormPairChunk = 8;   // 16-byte vectors per lane: half a row of 4096
+static_assert(kNormThreads == 256, "four warp pairs per block: named barriers 1-4");
+#ifndef MQ_NORM_PAIR_MIN_BLOCKS
+#define MQ_NORM_PAIR_MIN_BLOCKS 3
+#endif
+
+__global__ void __launch_bounds__(kNormThreads, MQ_NORM_PAIR_MIN_BLOCKS) rmsnorm_amax_pair_kernel(
+    const uint16_t* __restrict__ x, int64_t rows, int64_t K, const uint16_t* __restrict__ gamma, float eps,
+    float* __restrict__ rstd, float* __restrict__ alpha_out, WsControl* ctrl, uint32_t* __restrict__ partials)
+{
+    grid_dep_wait();   // X may be the previous kernel's output
+    grid_dep_launch_dependents();
+    constexpr int kPairs = kNormThreads / 64;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int g = warp & 1, pr = warp >> 1;
+    const int64_t pstride = (int64_t)gridDim.x * kPairs;
+    const int64_t nv = K / 8, nh = nv / 2;
+    extern __shared__ uint4 s_gamma[];
+    __shared__ double s_part[2][kNormThreads / 32];
+    for (int64_t i = threadIdx.x; i < nv; i += kNormThreads) s_gamma[i] = __ldg(reinterpret_cast<const uint4*>(gamma) + i);
+    __syncthreads();
+    const uint4* gh = s_gamma + g * nh;
+    uint32_t mx = 0, bad = 0;
+    int par = 0;
+    for (int64_t r = (int64_t)blockIdx.x * kPairs + pr; r < rows; r += pstride, par ^= 1) {
+        const uint4* xr = reinterpret_cast<const uint4*>(x + r * K) + g * nh;
+        if (lane == 0 && r + pstride < rows)
+            bulk_prefetch_l2(reinterpret_cast<const uint4*>(x + (r + pstride) * K) + g * nh, (uint32_t)K);
+        uint4 v[kNormPairChunk];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fold_max_flag(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-    __shared__ uint32_t s_red[kNormThreads / 32];
-    __shared__ bool is_last;
-    if (lane == 0) s_red[warp] = m;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        uint32_t b = 0;
-        for (int w = 0; w < kNormThreads / 32; ++w) b = fold_max_flag(b, s_red[w]);
-        partials[blockIdx.x] = b;
-        is_last = (atom_add_acq_rel_gpu(&ctrl->amax_ticket, 1u) == gridDim.x - 1);   // releases the partial
-    }
-    __syncthreads();
-    if (!is_last) return;
-    // the last block folds every block's maximum, all threads at once
-    uint32_t b = 0;
-    for (int j = threadIdx.x; j < (int)gridDim.x; j += kNormThreads) b = fold_max_flag(b, __ldcg(partials + j));
+        for (int u = 0; u < kNormPairChunk; ++u) {
+            const int64_t i = lane + 32 * u;
+            v[u] = (i < nh) ? __ldg(xr + i) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        // binary64 sum of the half's exact squares (four chains, then the warp)
+        double s[4] = {0.0, 0.0, 0.0, 0.0};
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) b = fold_max_flag(b, __shfl_xor_sync(0xFFFFFFFFu, b, o));
-    __syncthreads();
-    if (lane == 0) s_red[warp] = b;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        b = 0;
-        for (int w = 0; w < kNormThreads / 32; ++w) b = fold_max_flag(b, s_red[w]);
-        const float amax = __uint_as_float((b & 0x7FFFu) << 16);
-        *alpha_out = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
-        if (b & 0x80000000u) post_error(ctrl, kErrNonFinite);
-        ctrl->amax_ticket = 0;   // visible at kernel end
+        for (int u = 0; u < kNormPairChunk; ++u) {
+            const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const double a = (double)bf16_lo(w[j]), b = (double)bf16_hi(w[j]);
+                s[(j & 1) * 2] = __fma_rn(a, a, s[(j & 1) * 2]);
+                s[(j & 1) * 2 + 1] = __fma_rn(b, b, s[(j & 1) * 2 + 1]);
+            }
+        }
+        double sp = __dadd_rn(__dadd_rn(s[0], s[1]), __dadd_rn(s[2], s[3]));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sp = __dadd_rn(sp, __shfl_xor_sync(0xFFFFFFFFu, sp, o));
+        if (lane == 0) s_part[par][warp] = sp;
+        // the pair's barrier (ids 1-4; literal ids keep the block's barrier count at five)
+        switch (pr) {
+            case 0: asm volatile("bar.sync 1, 64;" ::: "memory"); break;
+            case 1: asm volatile("bar.sync 2, 64;" ::: "memory"); break;
+            case 2: asm volatile("bar.sync 3, 64;" ::: "memory"); break;
+            default: asm volatile("bar.sync 4, 64;" ::: "memory"); break;
+        }
+        const double ss = __dadd_rn(s_part[par][2 * pr], s_part[par][2 * pr + 1]);
+        const float ms = __double2float_rn(__ddiv_rn(ss, (double)K));
+        const float rs = __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(__dadd_rn((double)ms, (double)eps))));
+        if (g == 0 && lane == 0) rstd[r] = rs;
+        // |h| maximum of the half (two running maxima); NaN/Inf halves take the finite-only fold
+        uint32_t m2[2] = {0u, 0u};
+#pragma unroll
+        for (int u = 0; u < kNormPairChunk; ++u) {
+            const int64_t i = lane + 32 * u;
+            if (i < nh) {
+                const uint4 gv = gh[i];
+                m2[0] = max_u16x2(m2[0], norm_pair(v[u].x, gv.x, rs) & 0x7FFF7FFFu);
+                m2[1] = max_u16x2(m2[1], norm_pair(v[u].y, gv.y, rs) & 0x7FFF7FFFu);
+                m2[0] = max_u16x2(m2[0], norm_pair(v[u].z, gv.z, rs) & 0x7FFF7FFFu);
+                m2[1] = max_u16x2(m2[1], norm_pair(v[u].w, gv.w, rs) & 0x7FFF7FFFu);
+            }
+        }
+        uint32_t mrow = max_u16x2(m2[0], m2[1]);
+        if (__any_sync(0xFFFFFFFFu, max(mrow & 0xFFFFu, mrow >> 16) >= 0x7F80u)) {
+            mrow = 0;
+            for (int64_t i = lane; i < nh; i += 32) {
+                const uint4 xv = __ldg(xr + i), gv = gh[i];
+                amax_accum(norm_pair(xv.x, gv.x, rs), mrow, bad);
+                amax_accum(norm_pair(xv.y, gv.y, rs), mrow, bad);
+                amax_accum(norm_pair(xv.z, gv.z, rs), mrow, bad);
+                amax_accum(norm_pair(xv.w, gv.w, rs), mrow, bad);
+            }
+        }
+        mx = max_u16x2(mx, mrow);
     }
+    norm_alpha_publish<kNormThreads / 32>(mx, bad, alpha_out, ctrl, partials);
+}
+
+// Pass 2: quantize_kernel<false, true> forms h again on load and encodes it
+// with the alpha_h of pass 1.
+static cudaError_t launch_norm_quantize(const void* x, int64_t rows, int64_t K, const void* gamma, float* rstd,
+                                        uint8_t* codes, uint8_t* scales, float* alpha_out, void* h_out,
+                                        WsControl* ctrl, uint32_t* partials, const DeviceInfo& di, cudaStream_t s)
+{
+    const int64_t tiles = ((rows + 127) / 128) * ((K + 255) / 256);
+    const int occ = quantize_blocks_per_sm<false, true>(di);
+    int64_t qb = std::min(tiles, (int64_t)di.num_sms * std::max(1, occ));
+    qb = std::max<int64_t>(qb, 1);
+    NormArgs na{static_cast<const uint16_t*>(gamma), rstd, static_cast<uint16_t*>(h_out)};
+    return launch_pdl(quantize_kernel<false, true>, dim3((unsigned)qb), dim3(kQuantThreads), 0, s,
+                      static_cast<const uint16_t*>(x), rows, K, static_cast<const float*>(alpha_out), alpha_out,
+                      codes, scales, (int64_t)0, ctrl, partials, na);
 }
 
 cudaError_t launch_rmsnorm_quantize(const void* x, int64_t rows, int64_t K, const void* gamma, float eps,
                                     float* rstd, uint8_t* codes, uint8_t* scales, float* alpha_out, void* h_out,
                                     WsControl* ctrl, uint32_t* partials, const DeviceInfo& di, cudaStream_t s)
 {
+    if (K <= kNormPairMaxK) {
+        // two warps per row; one wave of resident blocks
+        const size_t smem = (size_t)K * 2;
+        int per_sm = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rmsnorm_amax_pair_kernel, kNormThreads, smem) !=
+            cudaSuccess) {
+            (void)cudaGetLastError();
+            per_sm = 1;
+        }
+        constexpr int kPairs = kNormThreads / 64;
+        int64_t blocks = (rows + kPairs - 1) / kPairs;
+        blocks = std::min<int64_t>(blocks, (int64_t)di.num_sms * std::max(1, per_sm));
+        blocks = std::min<int64_t>(blocks, kAmaxMaxBlocks);
+        blocks = std::max<int64_t>(blocks, 1);
+        cudaError_t e = launch_pdl(rmsnorm_amax_pair_kernel, dim3((unsigned)blocks), dim3(kNormThreads), smem, s,
+                                   static_cast<const uint16_t*>(x), rows, K, static_cast<const uint16_t*>(gamma), eps,
+                                   rstd, alpha_out, ctrl, partials);
+        if (e != cudaSuccess) return e;
+        return launch_norm_quantize(x, rows, K, gamma, rstd, codes, scales, alpha_out, h_out, ctrl, partials, di, s);
+    }
     // one wave of resident blocks; every warp then walks several rows
     const size_t gsmem = (K <= kNormGammaSmem) ? (size_t)K * 2 : 0;
     int per_sm = 0;
@@ -826,14 +975,7 @@ cudaError_t launch_rmsnorm_quantize(const void* x, int64_t rows, int64_t K, cons
                                static_cast<const uint16_t*>(x), rows, K, static_cast<const uint16_t*>(gamma), eps,
                                rstd, alpha_out, ctrl, partials);
     if (e != cudaSuccess) return e;
-    const int64_t tiles = ((rows + 127) / 128) * ((K + 255) / 256);
-    const int occ = quantize_blocks_per_sm<false, true>(di);
-    int64_t qb = std::min(tiles, (int64_t)di.num_sms * std::max(1, occ));
-    qb = std::max<int64_t>(qb, 1);
-    NormArgs na{static_cast<const uint16_t*>(gamma), rstd, static_cast<uint16_t*>(h_out)};
-    return launch_pdl(quantize_kernel<false, true>, dim3((unsigned)qb), dim3(kQuantThreads), 0, s,
-                      static_cast<const uint16_t*>(x), rows, K, static_cast<const float*>(alpha_out), alpha_out,
-                      codes, scales, (int64_t)0, ctrl, partials, na);
+    return launch_norm_quantize(x, rows, K, gamma, rstd, codes, scales, alpha_out, h_out, ctrl, partials, di, s);
 }
 
 __global__ void selftest_e2m1_kernel(unsigned long long* counts)
