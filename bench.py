@@ -326,7 +326,10 @@ class L2Flush:
 
 
 def _time_calls(torch, fn, reps, flush):
-    """Mean device time (ms) of fn() over reps calls, L2 flushed before each."""
+    """Mean device time (ms) of fn() over reps calls, L2 flushed before each.  One untimed call
+    comes first, so first-launch costs (lazy loading of a kernel's module, tensor-map set-up)
+    stay out of the mean."""
+    fn()
     evs = []
     for _ in range(reps):
         flush()
