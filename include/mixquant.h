@@ -175,10 +175,11 @@ MQ_API size_t mq_decode_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /*
  * The precise decode path (section 3.3: decoding stays on the original BF16
- * weights): Y[M, N] = bf16(sum_k X[m, k] W[n, k]) with FP32 accumulation on
- * the tensor cores.  X BF16 [M, K] with 1 <= M <= 256, W BF16 [N, K], Y BF16
- * [M, N].  ws: >= MQ_WS_CONTROL_BYTES; mq_decode_workspace_bytes(M, N, K)
- * for the fastest launch shape.
+ * weights): Y[M, N] = bf16(sum_k X[m, k] W[n, k]) with FP32 accumulation, on
+ * the tensor cores (a single token: FP32 fused multiply-adds on the CUDA
+ * cores).  X BF16 [M, K] with 1 <= M <= 256, W BF16 [N, K], Y BF16 [M, N].
+ * ws: >= MQ_WS_CONTROL_BYTES; mq_decode_workspace_bytes(M, N, K) for the
+ * fastest launch shape.
  */
 MQ_API mq_status mq_decode_linear(const void* X_bf16, int64_t M, const void* W_bf16, int64_t N, int64_t K, void* Y_bf16,
                            void* ws, size_t ws_bytes, mq_stream_t stream);

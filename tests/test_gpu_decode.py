@@ -32,8 +32,10 @@ def decode_check(y_bits, x, w):
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 256, 256), (8, 1024, 4096), (32, 512, 1024), (64, 768, 2048),
-                                   (17, 272, 320), (200, 256, 512), (256, 128, 128), (1, 4096, 12288)])
+                                   (17, 272, 320), (200, 256, 512), (256, 128, 128), (1, 4096, 12288),
+                                   (1, 16, 64), (1, 400, 1088), (2, 400, 1088)])
 def test_decode_linear_vs_oracle(M, N, K):
+    """M = 1 runs the CUDA-core kernel, larger M the tensor-core kernel."""
     x = wl.heavy_tailed_bf16(M, K, M + K)
     w = wl.normal_bf16(N, K, 0.02, N + K)
     y = mq.decode_linear(to_dev(x), to_dev(w))
@@ -41,9 +43,10 @@ def test_decode_linear_vs_oracle(M, N, K):
     decode_check(to_host_bits(y), x, w)
 
 
-def test_decode_exact_small_integers():
-    rng = np.random.default_rng(0)
-    xi = rng.integers(-4, 5, size=(8, 1024)).astype(np.float32)
+@pytest.mark.parametrize("M", [1, 8])
+def test_decode_exact_small_integers(M):
+    rng = np.random.default_rng(M)
+    xi = rng.integers(-4, 5, size=(M, 1024)).astype(np.float32)
     wi = rng.integers(-4, 5, size=(512, 1024)).astype(np.float32)
     y = mq.decode_linear(to_dev(wl.f32_to_bf16_bits(xi)), to_dev(wl.f32_to_bf16_bits(wi)))
     torch.cuda.synchronize()
