@@ -85,12 +85,13 @@ def test_decode_nvfp4_vs_oracle(M, N, K):
     print(f"nvfp4 decode M={M} N={N} K={K}: rel-Frobenius {rel:.2e}")
 
 
-@pytest.mark.parametrize("M,K", [(16, 512), (3, 2048)])
+@pytest.mark.parametrize("M,K", [(16, 512), (3, 2048), (1, 4096), (1, 192)])
 def test_decode_nvfp4_static_alpha_and_grid_inputs_exact(M, K):
     """Grid-valued inputs whose blocks all hold a 6: X with a static alpha of 1 and W with a 2688
     anchor alone in its block (alpha_w = 1) get block scales of exactly 1 (448 for the anchor), so
     Y = bf16(X W^T) exactly (the FP32 sums stay below 2^24 quarter units), on the quantization
-    kernel + decode GEMM (16 tokens) and on the single kernel (3 tokens)."""
+    kernel + decode GEMM (16 tokens) and on the single kernel (1 and 3 tokens; K = 192 ends in a
+    partial 256-element stage)."""
     rng = np.random.default_rng(3)
     grid = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6], np.float32)
     xi = (rng.choice(grid, size=(M, K)) * rng.choice([-1, 1], size=(M, K))).astype(np.float32)
@@ -162,6 +163,22 @@ def test_decode_nvfp4_reports_nonfinite_tokens():
     ax = oracle.tensor_alpha(x)[1]           # NaN excluded, as on the device
     assert ax == oracle.tensor_alpha(xf)[1]
     _nvfp4_decode_check(x[finite], w, to_host_bits(y)[finite], alpha_x=ax)
+
+
+def test_decode_nvfp4_single_token_nonfinite_and_zero():
+    """One token: a NaN is reported as MQ_ERR_NONFINITE; an all-zero token gives alpha_x = 1, zero
+    codes and an exactly zero output."""
+    w = wl.normal_bf16(256, 1024, 0.02, 93)
+    Wq = mq.quantize_weight(to_dev(w))
+    x = wl.heavy_tailed_bf16(1, 1024, 94)
+    x[0, 5] = 0x7FC0
+    ws = mq.workspace(1, 1024)
+    mq.decode_linear_nvfp4(to_dev(x), Wq, ws=ws)
+    assert mq.async_status(ws) == 5          # MQ_ERR_NONFINITE
+    z = np.zeros((1, 1024), np.uint16)
+    y = mq.decode_linear_nvfp4(to_dev(z), Wq, ws=ws)
+    assert mq.async_status(ws) == 0
+    assert not np.any(to_host_bits(y) & 0x7FFF)
 
 
 @pytest.mark.parametrize("M,N,K", [(8, 1024, 4096), (8, 12288, 4096), (64, 4096, 2048)])
