@@ -518,8 +518,12 @@ __device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v)
 //     (bounded; a wait that runs out posts kErrTimeout and the block stops).
 //     The quantization pass then walks the tiles in the opposite order, so
 //     the lines read last by the amax pass, still in L2, are read first.
-template <bool SEARCH, bool NORM, bool CLUSTER = false, bool LEAN = false>
-__global__ void __launch_bounds__(kQuantThreads, (LEAN || NORM) ? MQ_QUANT_MIN_BLOCKS - 1 : MQ_QUANT_MIN_BLOCKS)
+// LEAN: 0 the regular tile loop; 1 the lean tile loop for tiles inside the
+// tensor and the regular one for its edge tiles, three blocks per SM (the two
+// loops together need more than 64 registers); 2 the lean loop alone, for
+// tensors whose sizes are multiples of 128 x 256, at four blocks per SM.
+template <bool SEARCH, bool NORM, bool CLUSTER = false, int LEAN = 0>
+__global__ void __launch_bounds__(kQuantThreads, (LEAN == 1 || NORM) ? MQ_QUANT_MIN_BLOCKS - 1 : MQ_QUANT_MIN_BLOCKS)
     quantize_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t K, const float* __restrict__ alpha_static,
                     float* __restrict__ alpha_out, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
                     int64_t interleave_half, WsControl* ctrl, uint32_t* __restrict__ partials, NormArgs na)
@@ -656,7 +660,7 @@ __global__ void __launch_bounds__(kQuantThreads, (LEAN || NORM) ? MQ_QUANT_MIN_B
     for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
         const int64_t tile = tiles - 1 - t;
         const int64_t rb = tile / chunks, kc = tile % chunks;
-        if (LEAN && (rb + 1) * 128 <= rows && (kc + 1) * 256 <= K)
+        if (LEAN == 2 || (LEAN == 1 && (rb + 1) * 128 <= rows && (kc + 1) * 256 <= K))
             quant_tile_lean<SEARCH, NORM>(x, rows, K, interleave_half, rb, kc, chunks, qc, enc_tab, dec_tab, sf_stage,
                                           codes, scales, warp, half, blk, na);
         else
@@ -666,7 +670,7 @@ __global__ void __launch_bounds__(kQuantThreads, (LEAN || NORM) ? MQ_QUANT_MIN_B
 }
 
 // Resident blocks per SM of quantize_kernel<SEARCH, NORM, false, LEAN> (cached per device).
-template <bool SEARCH, bool NORM, bool LEAN = false>
+template <bool SEARCH, bool NORM, int LEAN = 0>
 int quantize_blocks_per_sm(const DeviceInfo& di)
 {
     static std::mutex mu;
@@ -742,12 +746,17 @@ cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float*
         if (e != cudaSuccess) return e;
         alpha_in = alpha_out;
     }
-    // Many waves of tiles (at least kQuantLeanTiles): the lean kernel, whose
-    // full tiles skip the per-block bounds checks (8192 x 12288: 84.8 -> 76.9 us
-    // for amax + quantization; at 8192 x 4096 the regular kernel is ahead)
-    const bool lean = !scale_search && !single && tiles >= kQuantLeanTiles;
+    // The lean tile loop skips the per-block bounds checks of tiles inside the
+    // tensor.  From kQuantLeanTiles tiles (several waves) at three blocks per SM
+    // with the regular loop for edge tiles (8192 x 12288: 84.8 -> 75 us for amax
+    // + quantization); below that, for sizes that are multiples of 128 x 256,
+    // alone at four blocks per SM (8192 x 4096: 35.6 -> 33.9 us).
+    const bool aligned = rows % 128 == 0 && K % 256 == 0;
+    const int lean = (scale_search || single) ? 0 : tiles >= kQuantLeanTiles ? 1 : aligned ? 2 : 0;
     const int64_t res =
-        lean ? (int64_t)di.num_sms * std::max(1, quantize_blocks_per_sm<false, false, true>(di)) : resident;
+        lean == 1   ? (int64_t)di.num_sms * std::max(1, quantize_blocks_per_sm<false, false, 1>(di))
+        : lean == 2 ? (int64_t)di.num_sms * std::max(1, quantize_blocks_per_sm<false, false, 2>(di))
+                    : resident;
     int64_t blocks = std::min(tiles, res);
     if (blocks > kAmaxMaxBlocks) blocks = kAmaxMaxBlocks;
     if (blocks < 1) blocks = 1;
@@ -776,7 +785,8 @@ cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float*
         cfg.numAttrs = 1;
     }
     auto kern = cl > 0 ? (scale_search ? quantize_kernel<true, false, true> : quantize_kernel<false, false, true>)
-                : lean ? quantize_kernel<false, false, false, true>
+                : lean == 1 ? quantize_kernel<false, false, false, 1>
+                : lean == 2 ? quantize_kernel<false, false, false, 2>
                        : (scale_search ? quantize_kernel<true, false> : quantize_kernel<false, false>);
     cudaError_t e = cudaLaunchKernelEx(&cfg, kern, static_cast<const uint16_t*>(x), rows, K, alpha_in, alpha_out,
                                        codes, scales, interleave_half, ctrl, partials, NormArgs{});
