@@ -521,7 +521,8 @@ __device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v)
 // LEAN: 0 the regular tile loop; 1 the lean tile loop for tiles inside the
 // tensor and the regular one for its edge tiles, three blocks per SM (the two
 // loops together need more than 64 registers); 2 the lean loop alone, for
-// tensors whose sizes are multiples of 128 x 256, at four blocks per SM.
+// tensors whose sizes are multiples of 128 x 256, at four blocks per SM (three
+// with NORM).
 template <bool SEARCH, bool NORM, bool CLUSTER = false, int LEAN = 0>
 __global__ void __launch_bounds__(kQuantThreads, (LEAN == 1 || NORM) ? MQ_QUANT_MIN_BLOCKS - 1 : MQ_QUANT_MIN_BLOCKS)
     quantize_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t K, const float* __restrict__ alpha_static,
@@ -1060,11 +1061,16 @@ static cudaError_t launch_norm_quantize(const void* x, int64_t rows, int64_t K, 
                                         WsControl* ctrl, uint32_t* partials, const DeviceInfo& di, cudaStream_t s)
 {
     const int64_t tiles = ((rows + 127) / 128) * ((K + 255) / 256);
-    const int occ = quantize_blocks_per_sm<false, true>(di);
+    // sizes that are multiples of 128 x 256: the lean tile loop alone (three
+    // blocks per SM, as every NORM instantiation; 8192 x 4096: 54.5 -> 51.6 us
+    // for the fused pair)
+    const bool aligned = rows % 128 == 0 && K % 256 == 0;
+    const int occ = aligned ? quantize_blocks_per_sm<false, true, 2>(di) : quantize_blocks_per_sm<false, true>(di);
     int64_t qb = std::min(tiles, (int64_t)di.num_sms * std::max(1, occ));
     qb = std::max<int64_t>(qb, 1);
     NormArgs na{static_cast<const uint16_t*>(gamma), rstd, static_cast<uint16_t*>(h_out)};
-    return launch_pdl(quantize_kernel<false, true>, dim3((unsigned)qb), dim3(kQuantThreads), 0, s,
+    return launch_pdl(aligned ? quantize_kernel<false, true, false, 2> : quantize_kernel<false, true>, dim3((unsigned)qb),
+                      dim3(kQuantThreads), 0, s,
                       static_cast<const uint16_t*>(x), rows, K, static_cast<const float*>(alpha_out), alpha_out,
                       codes, scales, (int64_t)0, ctrl, partials, na);
 }
