@@ -449,41 +449,39 @@ __device__ __forceinline__ void quant_block_store(uint32_t (&w)[8], bool ok, flo
 }
 
 template <bool SEARCH, bool NORM>
-__device__ __forceinline__ void quant_tile_lean(const uint16_t* __restrict__ x, int64_t rows, int64_t K,
-                                           int64_t interleave_half, int64_t rb, int64_t kc, int64_t chunks,
-                                           const QuantConsts& qc, const float* enc_tab, const float* dec_tab,
-                                           uint8_t* sf_stage, uint8_t* __restrict__ codes,
-                                           uint8_t* __restrict__ scales, int warp, int half, int blk,
-                                           const NormArgs& na)
+__device__ __forceinline__ void quant_tile_lean(const uint16_t* __restrict__ x, int64_t K, int64_t interleave_half,
+                                                int64_t rb, int64_t kc, int64_t chunks, const QuantConsts& qc,
+                                                const float* enc_tab, const float* dec_tab, uint8_t* sf_stage,
+                                                uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, int warp,
+                                                int half, int blk, const NormArgs& na)
 {
     const int64_t col = kc * 256 + 16 * blk;
     const uint16_t* gp = NORM ? na.gamma + col : nullptr;
-    const int rl0 = 16 * warp + half;
+    const int rl0 = 16 * warp + half;    // the thread's first row in the tile; then every second one
+    const int64_t r0 = rb * 128 + rl0;
+    const uint16_t* xp = x + quant_src_row(r0, interleave_half) * K + col;
+    uint8_t* cp = codes + r0 * (K / 2) + col / 2;
+    uint16_t* hp = (NORM && na.h_out != nullptr) ? na.h_out + r0 * K + col : nullptr;
+    // staging byte of (row rl0 + 2 st, block blk): (rl % 32) * 16 + (rl / 32) * 4 in the atom of
+    // blk / 4, byte blk % 4, so 32 bytes on per step
     uint8_t* sp0 = sf_stage + (blk >> 2) * 512 + (rl0 & 31) * 16 + (rl0 >> 5) * 4 + (blk & 3);
-    {
-        const int64_t r0 = rb * 128 + rl0;
-        const uint16_t* xp = x + quant_src_row(r0, interleave_half) * K + col;
-        uint8_t* cp = codes + r0 * (K / 2) + col / 2;
-        uint16_t* hp = (NORM && na.h_out != nullptr) ? na.h_out + r0 * K + col : nullptr;
 #pragma unroll 1
-        for (int s0 = 0; s0 < 8; s0 += kQuantStepUnroll) {
-            uint4 v[kQuantStepUnroll][2];
+    for (int s0 = 0; s0 < 8; s0 += kQuantStepUnroll) {
+        uint4 v[kQuantStepUnroll][2];
 #pragma unroll
-            for (int u = 0; u < kQuantStepUnroll; ++u) {
-                const uint4* p = reinterpret_cast<const uint4*>(xp + (int64_t)(2 * (s0 + u)) * K);
-                v[u][0] = __ldcs(p);
-                v[u][1] = __ldcs(p + 1);
-            }
+        for (int u = 0; u < kQuantStepUnroll; ++u) {
+            const uint4* p = reinterpret_cast<const uint4*>(xp + (int64_t)(2 * (s0 + u)) * K);
+            v[u][0] = __ldcs(p);
+            v[u][1] = __ldcs(p + 1);
+        }
 #pragma unroll
-            for (int u = 0; u < kQuantStepUnroll; ++u) {
-                const int st = s0 + u;
-                uint32_t w[8] = {v[u][0].x, v[u][0].y, v[u][0].z, v[u][0].w,
-                                 v[u][1].x, v[u][1].y, v[u][1].z, v[u][1].w};
-                const float rs = NORM ? __ldg(na.rstd + r0 + 2 * st) : 0.0f;
-                quant_block_store<SEARCH, NORM>(w, true, rs, gp, hp != nullptr ? hp + (int64_t)(2 * st) * K : nullptr,
-                                                reinterpret_cast<uint2*>(cp + (int64_t)st * K), sp0 + 32 * st, qc,
-                                                enc_tab, dec_tab);
-            }
+        for (int u = 0; u < kQuantStepUnroll; ++u) {
+            const int st = s0 + u;
+            uint32_t w[8] = {v[u][0].x, v[u][0].y, v[u][0].z, v[u][0].w, v[u][1].x, v[u][1].y, v[u][1].z, v[u][1].w};
+            const float rs = NORM ? __ldg(na.rstd + r0 + 2 * st) : 0.0f;
+            quant_block_store<SEARCH, NORM>(w, true, rs, gp, hp != nullptr ? hp + (int64_t)(2 * st) * K : nullptr,
+                                            reinterpret_cast<uint2*>(cp + (int64_t)st * K), sp0 + 32 * st, qc, enc_tab,
+                                            dec_tab);
         }
     }
     __syncthreads();
@@ -662,8 +660,8 @@ __global__ void __launch_bounds__(kQuantThreads, (LEAN == 1 || NORM) ? MQ_QUANT_
         const int64_t tile = tiles - 1 - t;
         const int64_t rb = tile / chunks, kc = tile % chunks;
         if (LEAN == 2 || (LEAN == 1 && (rb + 1) * 128 <= rows && (kc + 1) * 256 <= K))
-            quant_tile_lean<SEARCH, NORM>(x, rows, K, interleave_half, rb, kc, chunks, qc, enc_tab, dec_tab, sf_stage,
-                                          codes, scales, warp, half, blk, na);
+            quant_tile_lean<SEARCH, NORM>(x, K, interleave_half, rb, kc, chunks, qc, enc_tab, dec_tab, sf_stage, codes,
+                                          scales, warp, half, blk, na);
         else
             quant_tile<SEARCH, NORM>(x, rows, K, interleave_half, rb, kc, chunks, qc, enc_tab, dec_tab, sf_stage,
                                      codes, scales, warp, half, blk, na);
