@@ -265,9 +265,9 @@ MQ_API mq_status mq_prefill_kv_rope(const void* X_bf16, const mq_nvfp4* X_q, int
 /* RMSNorm fused with the quantization of its output: the NVFP4 copy of
  *   h[m][k] = bf16( fl32( fl32(x[m][k] * rstd_m) * gamma[k] ) ),
  *   ms_m = fl32( sum_k x^2 (binary64) / K ), rstd_m = fl32( 1/sqrt(ms_m + eps) ),
- *   (the kernel adds the exact binary32 squares in binary64 in its own order,
- *   which gives the same ms for BF16 inputs with 2^-63 <= |x| <= 2^63 except
- *   when the sum lies within ~2^-40 relative of an FP32 rounding boundary),
+ *   (the kernel adds the exact squares of the BF16 values in binary64 in its
+ *   own order, which gives the same ms for every BF16 input except when the
+ *   sum lies within ~2^-40 relative of an FP32 rounding boundary),
  * with a dynamic tensor scale over h (alpha_h = amax|h| / 2688, 1 if 0) and
  * Eq. 2 / Eq. 3 as mq_quantize_activation -- the same codes and scales as an
  * unfused RMSNorm writing BF16 h followed by mq_quantize_activation(h), with
