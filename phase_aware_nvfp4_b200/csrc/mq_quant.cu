@@ -388,9 +388,9 @@ __device__ __forceinline__ void quant_tile(const uint16_t* __restrict__ x, int64
 }
 
 
-// Lean variant of quant_tile for tiles inside the tensor on both axes, used
-// by the quantize kernel for large tensors (many waves of tiles), where the
-// pass is bound by instruction issue: no per-block bounds checks or zeroing,
+// Lean variant of quant_tile for tiles inside the tensor on both axes (see the
+// LEAN parameter of quantize_kernel for where it runs): the pass is bound by
+// instruction issue, and this loop has no per-block bounds checks or zeroing,
 // and the thread's 8 rows are 2 apart in the tile and, with the gate/up
 // interleave too, 2 apart in the source (a warp's 16 rows map onto 16
 // consecutive source rows), so its load, code and staging addresses advance
@@ -802,7 +802,7 @@ cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float*
 // rounding), stores rstd and takes the |h| maximum of the row's
 // h = bf16(fl(fl(x * rstd) * gamma)); the last block folds the per-block
 // maxima into alpha_h = amax/2688 (1 if 0; NaN/Inf excluded and reported).
-// Pass 2 is quantize_kernel<false, true>, which forms h again on load.
+// Pass 2 is quantize_kernel with NORM (launch_norm_quantize), which forms h again on load.
 constexpr int kNormThreads = 256;
 constexpr int64_t kNormGammaSmem = 8192;   // gamma elements staged in shared memory (16 KiB)
 
@@ -1052,7 +1052,7 @@ __global__ void __launch_bounds__(kNormThreads, MQ_NORM_PAIR_MIN_BLOCKS) rmsnorm
     norm_alpha_publish<kNormThreads / 32>(mx, bad, alpha_out, ctrl, partials);
 }
 
-// Pass 2: quantize_kernel<false, true> forms h again on load and encodes it
+// Pass 2: quantize_kernel with NORM forms h again on load and encodes it
 // with the alpha_h of pass 1.
 static cudaError_t launch_norm_quantize(const void* x, int64_t rows, int64_t K, const void* gamma, float* rstd,
                                         uint8_t* codes, uint8_t* scales, float* alpha_out, void* h_out,
