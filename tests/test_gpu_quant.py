@@ -283,3 +283,38 @@ def test_repeated_amax_on_one_workspace():
 def test_e2m1_conversion_instruction_matches_definition():
     """Every FP32 value in [-8, 8]: the hardware E2M1 rounding equals the comparison-chain definition."""
     assert mq.selftest_e2m1() == (0, 0)
+
+
+def _interleave_perm(n_rows):
+    """Stored row r of a gate/up-interleaved weight -> source row (16-row groups, gate then up)."""
+    half = n_rows // 2
+    perm = np.empty(n_rows, np.int64)
+    for r in range(n_rows):
+        c, t = divmod(r, 32)
+        perm[r] = 16 * c + t if t < 16 else half + 16 * c + (t - 16)
+    return perm
+
+
+@pytest.mark.parametrize("M,K,interleave", [(2048, 4096, False), (4096, 2048, True), (4173, 16448, False),
+                                            (16384, 4096, True)])
+def test_lean_quantization_paths_bit_exact(M, K, interleave):
+    """The lean tile loop: alone for 128 x 256-aligned tensors of more tiles than SMs (2048 x 4096,
+    and a 4096 x 2048 gate/up weight whose interleave maps each warp's 16 rows onto 16 consecutive
+    source rows), and for inner tiles beside the regular loop's edge tiles from 2048 tiles (4173 x
+    16448: 33 x 65 tiles with a partial last row block and column chunk; a 16384 x 4096 gate/up
+    weight).  Codes, scales and alpha bit-exact against the oracle on the first and last 128-row
+    blocks and one row in every 128-row block between."""
+    x = wl.heavy_tailed_bf16(M, K, 31 + M) if not interleave else wl.normal_bf16(M, K, 0.02, 37 + M)
+    X = to_dev(x)
+    t = mq.quantize_weight(X, gate_up_interleave=True) if interleave else mq.quantize_activation(X)
+    torch.cuda.synchronize()
+    codes, scales, alpha = nvfp4_host(t)
+    _, a_ref, _ = oracle.tensor_alpha(x)
+    assert np.float32(alpha) == np.float32(a_ref)
+    rows = np.unique(np.concatenate([np.arange(128), np.arange(M - (M % 128 or 128) - 128, M),
+                                     np.arange(128, M, 128) + 37 % 128]))
+    rows = rows[rows < M]
+    src = _interleave_perm(M)[rows] if interleave else rows
+    rc, rs = oracle.quantize(x[src], a_ref)
+    assert np.array_equal(scales[rows], rs), f"{int((scales[rows] != rs).sum())} scale mismatches"
+    assert np.array_equal(codes[rows], rc), f"{int((codes[rows] != rc).sum())} code byte mismatches"
