@@ -33,9 +33,10 @@ def decode_check(y_bits, x, w):
 
 @pytest.mark.parametrize("M,N,K", [(1, 256, 256), (8, 1024, 4096), (32, 512, 1024), (64, 768, 2048),
                                    (17, 272, 320), (200, 256, 512), (256, 128, 128), (1, 4096, 12288),
-                                   (1, 16, 64), (1, 400, 1088), (2, 400, 1088)])
+                                   (1, 16, 64), (1, 400, 1088), (2, 400, 1088), (1, 16, 131072)])
 def test_decode_linear_vs_oracle(M, N, K):
-    """M = 1 runs the CUDA-core kernel, larger M the tensor-core kernel."""
+    """M = 1 runs the CUDA-core kernel (unless the token, 2K bytes, exceeds shared memory, as at
+    K = 131072), larger M the tensor-core kernel."""
     x = wl.heavy_tailed_bf16(M, K, M + K)
     w = wl.normal_bf16(N, K, 0.02, N + K)
     y = mq.decode_linear(to_dev(x), to_dev(w))
@@ -68,7 +69,7 @@ def _nvfp4_decode_check(x, w, y_gpu_bits, alpha_x=None):
                                    (100, 272, 320), (128, 128, 4096), (1, 4096, 12288), (1, 12288, 4096),
                                    (8, 12288, 4096), (16, 12288, 4096), (16, 4096, 12288), (64, 12288, 4096),
                                    (128, 4096, 12288), (2, 400, 1024), (3, 1024, 2048), (4, 12288, 4096),
-                                   (2, 4096, 12288), (1, 272, 8192)])
+                                   (2, 4096, 12288), (1, 272, 8192), (1, 16, 131072)])
 def test_decode_nvfp4_vs_oracle(M, N, K):
     """Ragged tokens (MMA N padded to 32), ragged weight rows (N % 128 != 0) and a partial last
     256-element stage (K % 256 != 0) are all covered, as are the launch shapes the call picks:
